@@ -1,0 +1,238 @@
+"""bf16 activations x NVFP4 weights (mm_bf16_fp4) for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over the C-ABI library ``libfi_nvfp4.so`` (declared in
+``include/fi_nvfp4.h``). This module only marshals arguments: every step of the
+computation runs in the library's CUDA kernels. torch supplies device memory and the
+current CUDA stream. There is no CPU fallback: if the library is missing, every call
+raises.
+
+    Wq, Ws, g = pack_weights(W)                # W: fp32 [n, k] on cuda
+    out = mm_bf16_fp4(A, Wq, Ws, g)            # A: bf16 [m, k] on cuda -> bf16 [m, n]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "FiError", "KIND_GEMV", "KIND_MMA", "TACTIC_DEFAULT", "make_tactic", "tactic_fields",
+    "pack_weights", "mm_bf16_fp4", "splitk_reduce", "resolve_tactic", "default_tactic",
+    "list_tactics", "workspace_bytes", "set_workspace", "last_error", "version", "library",
+    "library_path",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libfi_nvfp4.so"
+
+KIND_GEMV = 0
+KIND_MMA = 1
+TACTIC_DEFAULT = -1
+
+_STATUS = {0: "FI_OK", -1: "FI_ERR_INVALID_ARG", -2: "FI_ERR_UNSUPPORTED_SHAPE",
+           -3: "FI_ERR_UNSUPPORTED_ARCH", -4: "FI_ERR_WORKSPACE", -5: "FI_ERR_CUDA"}
+
+
+class FiError(RuntimeError):
+    """A library call returned a non-zero fi_status."""
+
+    def __init__(self, status: int, where: str, message: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)}: {message}")
+
+
+class TacticInfo(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("splits", ctypes.c_int32),
+                ("ctas_per_sm", ctypes.c_int32), ("variant", ctypes.c_int32),
+                ("grid_x", ctypes.c_int32), ("grid_y", ctypes.c_int32),
+                ("threads", ctypes.c_int32), ("smem_bytes", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_int64)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def library() -> ctypes.CDLL:
+    """Load libfi_nvfp4.so (built by ``python -m bf16_activations_nvfp4_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m bf16_activations_nvfp4_b200.build` "
+                "(there is no fallback implementation)")
+        lib = ctypes.CDLL(path)
+        vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+        lib.fi_nvfp4_pack_weights.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+        lib.fi_mm_bf16_fp4.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
+        lib.fi_mm_bf16_fp4_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp]
+        lib.fi_splitk_reduce.argtypes = [vp, i64, i64, i64, vp, vp, vp]
+        lib.fi_resolve_tactic.argtypes = [i64, i64, i64, i64, ctypes.c_int, ctypes.POINTER(TacticInfo)]
+        lib.fi_default_tactic.argtypes = [i64, i64, i64, ctypes.c_int]
+        lib.fi_default_tactic.restype = i64
+        lib.fi_list_tactics.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.POINTER(i64), ctypes.c_int]
+        lib.fi_mm_workspace_bytes.argtypes = [i64, i64, i64, i64, ctypes.c_int]
+        lib.fi_mm_workspace_bytes.restype = sz
+        lib.fi_set_workspace.argtypes = [vp, sz]
+        lib.fi_last_error.argtypes = []
+        lib.fi_last_error.restype = ctypes.c_char_p
+        lib.fi_version.argtypes = []
+        for name in ("fi_nvfp4_pack_weights", "fi_mm_bf16_fp4", "fi_mm_bf16_fp4_ex", "fi_splitk_reduce",
+                     "fi_resolve_tactic", "fi_list_tactics", "fi_set_workspace", "fi_version"):
+            getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def last_error() -> str:
+    return library().fi_last_error().decode()
+
+
+def version() -> int:
+    return library().fi_version()
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise FiError(status, where, last_error())
+
+
+# ------------------------------------------------------------------------- tactics
+
+def make_tactic(kind: int, splits: int = 0, ctas_per_sm: int = 0, variant: int = 0) -> int:
+    """FI_TACTIC(kind, splits, ctas_per_sm, variant) from include/fi_nvfp4.h."""
+    return (kind << 24) | (splits << 12) | (ctas_per_sm << 8) | variant
+
+
+def tactic_fields(t: int) -> dict:
+    return {"kind": (t >> 24) & 0xF, "splits": (t >> 12) & 0xFFF, "ctas_per_sm": (t >> 8) & 0xF,
+            "variant": t & 0xFF}
+
+
+def resolve_tactic(m: int, n: int, k: int, tactic: int = TACTIC_DEFAULT, num_sms: int = 0) -> dict:
+    info = TacticInfo()
+    _check(library().fi_resolve_tactic(m, n, k, tactic, num_sms, ctypes.byref(info)), "fi_resolve_tactic")
+    return info.as_dict()
+
+
+def default_tactic(m: int, n: int, k: int, num_sms: int = 0) -> int:
+    t = library().fi_default_tactic(m, n, k, num_sms)
+    if t < 0:
+        raise FiError(int(t), "fi_default_tactic", last_error())
+    return int(t)
+
+
+def list_tactics(m: int, n: int, k: int, num_sms: int = 0) -> list[int]:
+    lib = library()
+    count = lib.fi_list_tactics(m, n, k, num_sms, None, 0)
+    if count < 0:
+        raise FiError(count, "fi_list_tactics", last_error())
+    buf = (ctypes.c_int64 * max(count, 1))()
+    lib.fi_list_tactics(m, n, k, num_sms, buf, count)
+    return [int(buf[i]) for i in range(count)]
+
+
+def workspace_bytes(m: int, n: int, k: int, tactic: int = TACTIC_DEFAULT, num_sms: int = 0) -> int:
+    return int(library().fi_mm_workspace_bytes(m, n, k, tactic, num_sms))
+
+
+def set_workspace(buf: torch.Tensor | None) -> None:
+    """Register a caller-owned split-K workspace (a CUDA tensor) for the current device.
+    The caller must keep `buf` alive while calls may use it; None unregisters it."""
+    if buf is None:
+        _check(library().fi_set_workspace(None, 0), "fi_set_workspace")
+    else:
+        _check(library().fi_set_workspace(buf.data_ptr(), buf.numel() * buf.element_size()),
+               "fi_set_workspace")
+
+
+# ---------------------------------------------------------------------- the op
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _require(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+def pack_weights(W: torch.Tensor, out: tuple | None = None):
+    """Quantise fp32 W [n, k] (CUDA) to NVFP4 -> (Wq uint8 [n, k/2], Wscale uint8 [n, k/16],
+    gscale fp32 [1]), all on W's device."""
+    _require(W, "W", torch.float32, 2)
+    n, k = W.shape
+    if out is None:
+        Wq = torch.empty((n, k // 2), dtype=torch.uint8, device=W.device)
+        Ws = torch.empty((n, k // 16), dtype=torch.uint8, device=W.device)
+        g = torch.empty(1, dtype=torch.float32, device=W.device)
+    else:
+        Wq, Ws, g = out
+    with torch.cuda.device(W.device):
+        _check(library().fi_nvfp4_pack_weights(W.data_ptr(), n, k, Wq.data_ptr(), Ws.data_ptr(),
+                                               g.data_ptr(), _stream(W.device)), "fi_nvfp4_pack_weights")
+    return Wq, Ws, g
+
+
+def mm_bf16_fp4(A: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor, gscale: torch.Tensor,
+                tactic: int = TACTIC_DEFAULT, out: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """out[m, n] = A[m, k] . dequant(W)^T, bf16 out (CUDA tensors on one device).
+
+    `workspace` (optional CUDA tensor) is passed to fi_mm_bf16_fp4_ex; without it the call
+    uses the per-device workspace of fi_mm_bf16_fp4.
+    """
+    _require(A, "A", torch.bfloat16, 2)
+    _require(Wq, "Wq", torch.uint8, 2)
+    _require(Wscale, "Wscale", torch.uint8, 2)
+    _require(gscale, "gscale", torch.float32, 1)
+    m, k = A.shape
+    n = Wq.shape[0]
+    if Wq.shape[1] * 2 != k or Wscale.shape != (n, k // 16):
+        raise ValueError(f"shape mismatch: A {tuple(A.shape)}, Wq {tuple(Wq.shape)}, Wscale {tuple(Wscale.shape)}")
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=A.device)
+    else:
+        _require(out, "out", torch.bfloat16, 2)
+    lib = library()
+    with torch.cuda.device(A.device):
+        s = _stream(A.device)
+        if workspace is None:
+            st = lib.fi_mm_bf16_fp4(A.data_ptr(), Wq.data_ptr(), Wscale.data_ptr(), gscale.data_ptr(),
+                                    out.data_ptr(), m, n, k, tactic, s)
+            _check(st, "fi_mm_bf16_fp4")
+        else:
+            st = lib.fi_mm_bf16_fp4_ex(A.data_ptr(), Wq.data_ptr(), Wscale.data_ptr(), gscale.data_ptr(),
+                                       out.data_ptr(), m, n, k, tactic, workspace.data_ptr(),
+                                       workspace.numel() * workspace.element_size(), s)
+            _check(st, "fi_mm_bf16_fp4_ex")
+    return out
+
+
+def splitk_reduce(partials: torch.Tensor, gscale: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16_rn(gscale * fixed-order sum over dim 0) of fp32 partials [S, m, n]."""
+    _require(partials, "partials", torch.float32, 3)
+    _require(gscale, "gscale", torch.float32, 1)
+    S, m, n = partials.shape
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=partials.device)
+    with torch.cuda.device(partials.device):
+        _check(library().fi_splitk_reduce(partials.data_ptr(), S, m, n, gscale.data_ptr(), out.data_ptr(),
+                                          _stream(partials.device)), "fi_splitk_reduce")
+    return out

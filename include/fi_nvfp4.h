@@ -1,0 +1,203 @@
+/*
+ * fi_nvfp4.h - bf16 activations x NVFP4 weights (mm_bf16_fp4) on NVIDIA B200 (sm_100a).
+ *
+ * The operation, after "perf(gemm): split-K, occupancy, and m=1 stream-GEMV decode tactics
+ * for mm_bf16_fp4" (flashinfer PR #4038), Description:
+ *
+ *     out[m, n] = A[m, k] . dequant(W[n, k])^T
+ *
+ * with A in bf16 and W in NVFP4: E2M1 4-bit codes packed two per byte, one E4M3 scale per
+ * 16 contiguous k, one fp32 scale for the whole tensor; fp32 accumulation, bf16 output.
+ * Split-K tactics write fp32 partials that a second kernel sums in a fixed order, so
+ * results are bitwise deterministic run to run (PR #4038, "What it does"); within one
+ * tactic a row's bits do not depend on m (the batch-invariant property of the FlashInfer
+ * v0.7.4 article, "Why identical bits matter").
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library never frees
+ *    or retains them beyond the call. Calls are asynchronous on `stream` (NULL = legacy
+ *    default stream) and never synchronise the host.
+ *  - bf16 tensors are passed as uint16_t bit patterns; layouts are row-major, dense.
+ *  - NVFP4 layout ("canonical", PR #4038 GEMV commit: "(N, K/2) packed layout + linear
+ *    E4M3 scales"): Wq is uint8 [n, k/2], byte j of a row holds code 2j in bits 0-3 and
+ *    code 2j+1 in bits 4-7; Wscale is uint8 [n, k/16] of E4M3 codes, row-major (linear,
+ *    unswizzled); gscale points to one fp32 in device memory (so calls can be captured in
+ *    a CUDA graph without a host read).
+ *  - Return value: FI_OK (0) or a negative fi_status. On error nothing was launched and a
+ *    message is available from fi_last_error() (thread-local). A CUDA launch failure
+ *    returns FI_ERR_CUDA after other work of the same call may already be queued.
+ *  - Supported device: compute capability 10.0 (B200, sm_100a); other devices return
+ *    FI_ERR_UNSUPPORTED_ARCH.
+ */
+#ifndef FI_NVFP4_H_
+#define FI_NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FI_API __attribute__((visibility("default")))
+#else
+#define FI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so this header needs no CUDA headers. */
+typedef struct CUstream_st* fi_stream_t;
+
+typedef enum {
+  FI_OK = 0,
+  FI_ERR_INVALID_ARG = -1,       /* null / misaligned pointer, negative size, bad tactic */
+  FI_ERR_UNSUPPORTED_SHAPE = -2, /* k not a multiple of 32, m beyond the tactic's range */
+  FI_ERR_UNSUPPORTED_ARCH = -3,  /* current device is not compute capability 10.0 */
+  FI_ERR_WORKSPACE = -4,         /* split-K workspace missing or too small */
+  FI_ERR_CUDA = -5               /* a CUDA runtime call or launch failed */
+} fi_status;
+
+/* ------------------------------------------------------------------------- tactics
+ * A tactic is a 32-bit code built by FI_TACTIC(kind, splits, ctas_per_sm, variant):
+ *   kind         FI_KIND_GEMV (streaming GEMV, 1 <= m <= 32) or FI_KIND_MMA (tcgen05
+ *                tensor-core GEMM, 1 <= m <= 256);
+ *   splits       number of K partitions S (1..4095); 0 = device-sized ("knee") split:
+ *                the smallest S that gives the device enough concurrent weight streams
+ *                (PR #4038, "Sizes GEMV split-K from the device");
+ *   ctas_per_sm  co-resident CTAs per SM used to size the grid (1..15); 0 = automatic
+ *                (PR #4038, "Adds occupancy tactics");
+ *   variant      GEMV: weight rows per warp (1, 2 or 4; 0 = automatic). MMA: 0.
+ * Only `kind` and the resolved S change the arithmetic: two tactics with the same kind
+ * and S give bitwise identical outputs, and for a fixed tactic every output row is
+ * bitwise independent of m. FI_TACTIC_DEFAULT (-1) selects from the built-in per-shape
+ * table (PR #4038, "Routes the no-autotune m=1 fallback onto the GEMV"); the table's
+ * choice of kind and S depends on m, so the default is batch-invariant only within the
+ * m range of one table entry.
+ */
+#define FI_KIND_GEMV 0
+#define FI_KIND_MMA 1
+#define FI_TACTIC_DEFAULT ((int64_t)-1)
+#define FI_TACTIC(kind, splits, ctas_per_sm, variant)                          \
+  ((int64_t)(((int64_t)(kind) << 24) | ((int64_t)(splits) << 12) |             \
+             ((int64_t)(ctas_per_sm) << 8) | (int64_t)(variant)))
+#define FI_TACTIC_KIND(t) ((int)(((t) >> 24) & 0xF))
+#define FI_TACTIC_SPLITS(t) ((int)(((t) >> 12) & 0xFFF))
+#define FI_TACTIC_CTAS(t) ((int)(((t) >> 8) & 0xF))
+#define FI_TACTIC_VARIANT(t) ((int)((t) & 0xFF))
+
+/* A tactic resolved for one shape and device (host-side description). */
+typedef struct {
+  int32_t kind;        /* FI_KIND_GEMV or FI_KIND_MMA */
+  int32_t splits;      /* resolved S >= 1 */
+  int32_t ctas_per_sm; /* resolved co-resident CTAs per SM */
+  int32_t variant;     /* resolved variant (GEMV rows per warp) */
+  int32_t grid_x;      /* CTAs along n */
+  int32_t grid_y;      /* CTAs along k (= splits) */
+  int32_t threads;     /* threads per CTA */
+  int32_t smem_bytes;  /* dynamic shared memory per CTA */
+  int64_t workspace_bytes; /* fp32 partials needed (0 when S == 1) */
+} fi_tactic_info;
+
+/* ------------------------------------------------------------------ entry points */
+
+/*
+ * Quantise fp32 weights to NVFP4 (the weight-preparation step; not on the timed path).
+ *   W       device fp32 [n, k], row-major, 16-byte aligned.
+ *   Wq      device uint8 [n, k/2] (output), 16-byte aligned.
+ *   Wscale  device uint8 [n, k/16] (output), 8-byte aligned.
+ *   gscale  device fp32 [1] (output); also used as scratch by the call.
+ * Recipe: gscale = amax(|W|) / (448*6) (one fp32 division); for each 16-block
+ * sf = E4M3_rn_satfinite((amax_block / 6) / gscale); denom = sf * gscale;
+ * code = E2M1_rn_satfinite(w / denom) with the sign of w, or 0 for the whole block when
+ * denom == 0. All arithmetic is IEEE fp32 round-to-nearest-even, so the result is
+ * bit-identical to a CPU implementation of the same steps. Inputs must be finite.
+ * Preconditions: n >= 0, k >= 0, k % 16 == 0 (n == 0 or k == 0 writes gscale = 0).
+ */
+FI_API int fi_nvfp4_pack_weights(const float* W, int64_t n, int64_t k, uint8_t* Wq,
+                          uint8_t* Wscale, float* gscale, fi_stream_t stream);
+
+/*
+ * out[m, n] = bf16_rn(gscale * sum_k A[m, k] * e2m1(Wq) * e4m3(Wscale)), fp32 accumulate
+ * (PR #4038, Description).
+ *   A       device bf16 bits [m, k], 16-byte aligned.
+ *   Wq, Wscale, gscale  NVFP4 weights as produced by fi_nvfp4_pack_weights; Wq 16-byte
+ *           aligned, Wscale 2-byte aligned.
+ *   out     device bf16 bits [m, n], 2-byte aligned; must not overlap the inputs.
+ *   tactic  FI_TACTIC_DEFAULT or an FI_TACTIC(...) code (see above).
+ * Preconditions: m >= 0, n >= 0, k >= 0, k % 32 == 0; m <= 32 for GEMV tactics and
+ * m <= 256 for MMA tactics (FI_ERR_UNSUPPORTED_SHAPE otherwise). m == 0 or n == 0 is a
+ * no-op; k == 0 writes zeros.
+ * Split-K workspace: when the resolved S > 1 the call needs fi_mm_workspace_bytes()
+ * bytes of device memory for fp32 partials. It uses the buffer registered with
+ * fi_set_workspace() for the current device (FI_ERR_WORKSPACE if that is too small); if
+ * none is registered, the library allocates one with cudaMalloc (growing it when needed)
+ * and keeps it until process exit, except while `stream` is capturing a CUDA graph,
+ * where it returns FI_ERR_WORKSPACE instead of allocating.
+ * The per-device workspace is shared: calls that may overlap on different streams must
+ * use fi_mm_bf16_fp4_ex with separate workspaces.
+ */
+FI_API int fi_mm_bf16_fp4(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale,
+                   const float* gscale, uint16_t* out, int64_t m, int64_t n, int64_t k,
+                   int64_t tactic, fi_stream_t stream);
+
+/*
+ * fi_mm_bf16_fp4 with a caller-provided split-K workspace (device, 256-byte aligned,
+ * at least fi_mm_workspace_bytes() bytes; may be NULL when that is 0). Never allocates.
+ */
+FI_API int fi_mm_bf16_fp4_ex(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale,
+                      const float* gscale, uint16_t* out, int64_t m, int64_t n, int64_t k,
+                      int64_t tactic, void* workspace, size_t workspace_bytes,
+                      fi_stream_t stream);
+
+/*
+ * Fixed-order split-K reduction (PR #4038, "a PDL-chained reduce kernel sums them in
+ * fixed order"): for every element e of [m, n],
+ *     s = ((p[0][e] + p[1][e]) + p[2][e]) + ...   (fp32, s = 0 .. splits-1 in order)
+ *     out[e] = bf16_rn(s * gscale[0])             (fp32 product)
+ *   partials  device fp32 [splits, m, n], 16-byte aligned.
+ *   gscale    device fp32 [1].
+ *   out       device bf16 bits [m, n], 2-byte aligned.
+ * Preconditions: 1 <= splits <= 4095, m >= 0, n >= 0.
+ */
+FI_API int fi_splitk_reduce(const float* partials, int64_t splits, int64_t m, int64_t n,
+                     const float* gscale, uint16_t* out, fi_stream_t stream);
+
+/* --------------------------------------------------------------- host helpers
+ * These run on the host only and never launch work. `num_sms` <= 0 means "query the
+ * current device" (which then must exist); a positive value describes a device without
+ * touching CUDA, so the tactic logic can be inspected on any machine.
+ */
+
+/* Resolve a tactic (or FI_TACTIC_DEFAULT) for a shape. Returns FI_OK and fills *info,
+ * or an error status (invalid code, unsupported m for the kind, ...). */
+FI_API int fi_resolve_tactic(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms,
+                      fi_tactic_info* info);
+
+/* The tactic FI_TACTIC_DEFAULT resolves to (the per-shape table). Negative on error. */
+FI_API int64_t fi_default_tactic(int64_t m, int64_t n, int64_t k, int num_sms);
+
+/* Enumerate the valid tactics for a shape into out[0 .. cap-1]; returns how many exist
+ * (which may exceed cap), or a negative status. */
+FI_API int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, int cap);
+
+/* Workspace bytes a call with this shape and tactic needs (0 when S == 1), or 0 for an
+ * invalid tactic. */
+FI_API size_t fi_mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms);
+
+/* Register a caller-owned split-K workspace for the current device (device pointer,
+ * 256-byte aligned; NULL with bytes == 0 unregisters it). The library frees any buffer it
+ * allocated itself for that device. The caller keeps ownership of `ptr` and must keep it
+ * alive while calls that use it may run. */
+FI_API int fi_set_workspace(void* ptr, size_t bytes);
+
+/* Message describing the last error on this host thread ("" if none). */
+FI_API const char* fi_last_error(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+FI_API int fi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FI_NVFP4_H_ */

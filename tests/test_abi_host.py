@@ -1,0 +1,146 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The library must load on a machine without a GPU, export every function that
+include/fi_nvfp4.h declares, resolve tactics from a given SM count without touching CUDA,
+and reject bad arguments before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bf16_activations_nvfp4_b200 as fi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fi_nvfp4.h")
+B200_SMS = 148
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^FI_API\s+[\w\s\*]+?\b(fi_\w+)\s*\(", text, flags=re.M)
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert len(names) >= 11
+    lib = fi.library()
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_version():
+    assert fi.version() >= 100
+
+
+def test_tactic_encoding_matches_header_macros():
+    t = fi.make_tactic(fi.KIND_MMA, 37, 3, 2)
+    assert t == (1 << 24) | (37 << 12) | (3 << 8) | 2
+    assert fi.tactic_fields(t) == {"kind": 1, "splits": 37, "ctas_per_sm": 3, "variant": 2}
+
+
+@pytest.mark.parametrize("n,k", [(2048, 7168), (4096, 4096), (4096, 14336), (14336, 4096), (10304, 2688),
+                                 (512, 2048), (512, 4096), (1024, 2048), (1024, 4096), (2048, 2048),
+                                 (2048, 4096), (152064, 5120)])
+def test_default_gemv_tactic_resolves_for_decode_shapes(n, k):
+    info = fi.resolve_tactic(1, n, k, fi.TACTIC_DEFAULT, B200_SMS)
+    assert info["kind"] == fi.KIND_GEMV
+    assert 1 <= info["splits"] <= k // 32
+    # one wave: the grid never asks for more CTAs than the SMs hold at the tactic's occupancy
+    assert info["grid_x"] * info["grid_y"] <= B200_SMS * info["ctas_per_sm"]
+    # every weight row is covered by some warp of the grid
+    rows_per_cta = 8 * info["variant"]
+    assert info["grid_x"] * rows_per_cta >= min(n, rows_per_cta)
+    assert info["workspace_bytes"] == (info["splits"] * n * 4 if info["splits"] > 1 else 0)
+
+
+def test_device_sized_split_reaches_the_knee_and_is_m_independent():
+    for n, k in [(512, 2048), (1024, 4096), (4096, 14336), (14336, 4096)]:
+        splits = {fi.resolve_tactic(m, n, k, fi.make_tactic(fi.KIND_GEMV, 0, 0, 1), B200_SMS)["splits"]
+                  for m in (1, 2, 4, 8)}
+        assert len(splits) == 1, (n, k, splits)
+        S = splits.pop()
+        warps = n * S  # one row per warp with variant 1
+        assert warps >= 20 * B200_SMS or S == max(1, (k // 32) // 8), (n, k, S)
+        if S > 1:
+            assert n * (S - 1) < 20 * B200_SMS or gemv_smem_needs_split(k, S - 1)
+
+
+def gemv_smem_needs_split(k, S):
+    klen = -(-(k // 32) // S) * 32
+    return 8 * klen * 2 + 8 * (klen // 16) * 4 > 200 * 1024
+
+
+def test_explicit_splits_are_kept():
+    for S in (1, 2, 4, 8):
+        info = fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, S, 0, 2), B200_SMS)
+        assert info["splits"] == S and info["variant"] == 2
+
+
+def test_list_tactics_unique_and_valid():
+    ts = fi.list_tactics(1, 4096, 14336, B200_SMS)
+    assert len(ts) == len(set(ts)) and len(ts) >= 6
+    for t in ts:
+        fi.resolve_tactic(1, 4096, 14336, t, B200_SMS)
+
+
+def test_workspace_bytes():
+    t = fi.make_tactic(fi.KIND_GEMV, 4, 0, 1)
+    assert fi.workspace_bytes(3, 1000, 4096, t, B200_SMS) == 4 * 3 * 1000 * 4
+    assert fi.workspace_bytes(3, 1000, 4096, fi.make_tactic(fi.KIND_GEMV, 1, 0, 1), B200_SMS) == 0
+
+
+@pytest.mark.parametrize("m,n,k,tactic,status", [
+    (1, 64, 48, -1, -2),                                  # k % 32 != 0
+    (33, 64, 64, fi.make_tactic(0, 1, 0, 1), -2),         # GEMV beyond m = 32
+    (1, 64, 64, fi.make_tactic(0, 1, 0, 3), -1),          # rows per warp 3
+    (1, 64, 64, fi.make_tactic(0, 3, 0, 1), -1),          # splits > k/32
+    (1, 64, 64, fi.make_tactic(7, 1, 0, 1), -1),          # unknown kind
+    (1, 64, 64, 1 << 30, -1),                             # out-of-range code
+    (-1, 64, 64, -1, -1),                                 # negative size
+    (32, 64, 14336, fi.make_tactic(0, 1, 0, 1), -2),      # A slice does not fit shared memory
+])
+def test_resolve_rejects(m, n, k, tactic, status):
+    with pytest.raises(fi.FiError) as e:
+        fi.resolve_tactic(m, n, k, tactic, B200_SMS)
+    assert e.value.status == status
+    assert fi.last_error()
+
+
+def _call_mm(A, Wq, Ws, g, out, m, n, k, tactic=-1):
+    lib = fi.library()
+    return lib.fi_mm_bf16_fp4(A, Wq, Ws, g, out, m, n, k, tactic, None)
+
+
+def test_mm_argument_checks_precede_cuda():
+    lib = fi.library()
+    # empty problems are no-ops
+    assert _call_mm(None, None, None, None, None, 0, 64, 64) == 0
+    assert _call_mm(None, None, None, None, None, 4, 0, 64) == 0
+    # shape and pointer errors
+    assert _call_mm(16, 16, 16, 16, 16, 1, 64, 40) == -2
+    assert _call_mm(None, 16, 16, 16, 16, 1, 64, 64) == -1
+    assert "null" in fi.last_error()
+    assert _call_mm(0x1008, 0x2000, 0x3000, 0x4000, 0x5000, 1, 64, 64) == -1  # A misaligned
+    assert "aligned" in fi.last_error()
+    assert _call_mm(0x1000, 0x2000, 0x3001, 0x4000, 0x5000, 1, 64, 64) == -1  # Wscale misaligned
+    assert lib.fi_mm_bf16_fp4_ex(None, None, None, None, None, 0, 1, 32, -1, None, 0, None) == 0
+
+
+def test_pack_and_reduce_argument_checks():
+    lib = fi.library()
+    assert lib.fi_nvfp4_pack_weights(0x1000, 4, 24, 0x2000, 0x3000, 0x4000, None) == -2
+    assert lib.fi_nvfp4_pack_weights(0x1000, 4, 32, 0x2000, 0x3000, None, None) == -1
+    assert lib.fi_nvfp4_pack_weights(0x1004, 4, 32, 0x2000, 0x3000, 0x4000, None) == -1
+    assert lib.fi_splitk_reduce(0x1000, 0, 1, 1, 0x2000, 0x3000, None) == -1
+    assert lib.fi_splitk_reduce(0x1000, 4096, 1, 1, 0x2000, 0x3000, None) == -1
+    assert lib.fi_splitk_reduce(None, 2, 0, 5, None, None, None) == 0
+    assert lib.fi_splitk_reduce(0x1008, 2, 1, 5, 0x2000, 0x3000, None) == -1
+
+
+def test_set_workspace_rejects_bad_arguments():
+    lib = fi.library()
+    assert lib.fi_set_workspace(0x1000, 0) == -1
+    assert lib.fi_set_workspace(None, 64) == -1
+    assert lib.fi_set_workspace(0x1010, 4096) == -1
