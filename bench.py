@@ -1,12 +1,14 @@
 #!/usr/bin/env python
 """Benchmark: m=1 bf16 x NVFP4 decode GEMV on B200 (the serving-class decode shapes).
 
-One step = one call of the library's public op (default tactic) on each of the five
-serving decode shapes n x k in {2048x7168, 4096x4096, 4096x14336, 14336x4096,
-10304x2688} at m=1 (PR #4038, "Split-K on the #3597 decode shapes", first table).
-Every call is a CUDA-graph replay timed with CUDA events on its stream, with L2 flushed
-(a 256 MiB write) before it, as decode serving runs with a cold L2 (PR #4038,
-Performance: "Median GPU time over CUDA-graph replays with a cold L2 cache").
+One step = the five serving decode shapes n x k in {2048x7168, 4096x4096, 4096x14336,
+14336x4096, 10304x2688} at m=1 (PR #4038, "Split-K on the #3597 decode shapes", first
+table), each called through the library's public op with the GEMV tactic at split-K
+S in {1, 2, 4, 8, device-sized}: 25 calls. Every call is a CUDA-graph replay timed with
+CUDA events on its stream, with L2 flushed (a 256 MiB read) before it, as decode serving
+runs with a cold L2 (PR #4038, Performance: "Median GPU time over CUDA-graph replays with
+a cold L2 cache"). The library's default tactic per shape is timed in a second pass and
+reported beside the step.
 
 value = algorithmic bytes of all calls / their summed device time (GB/s); algorithmic
 bytes per call = n*k/2 + n*k/16 + 2*m*k + 2*m*n (packed codes, E4M3 scales, bf16 A and
@@ -37,6 +39,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "µs/call and achieved HBM GB/s (% of B200 peak) for m=1 bf16×NVFP4 GEMV"
 SHAPES = [(2048, 7168), (4096, 4096), (4096, 14336), (14336, 4096), (10304, 2688)]
+SPLITS = [1, 2, 4, 8, 0]  # 0 = device-sized
 M = 1
 FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
@@ -135,46 +138,55 @@ def run_fi(args, rank: int, world: int) -> dict | None:
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(dev)
 
-    cases = []
+    def make_case(n, k, tactic, shared):
+        info = fi.resolve_tactic(M, n, k, tactic)
+        return dict(shared, n=n, k=k, tactic=tactic, info=info, bytes=algorithmic_bytes(M, n, k),
+                    out=torch.empty((M, n), dtype=torch.bfloat16, device=dev))
+
+    cases, defaults = [], []
     for n, k in SHAPES:
         W = torch.from_numpy(inputs.weights(n, k, seed=0)).to(dev)
         Wq, Ws, g = fi.pack_weights(W)
         del W
         a_host = inputs.activations(M, k, seed=0)
-        A = torch.from_numpy(a_host.view(np.int16)).view(torch.bfloat16).to(dev)
-        A_pinned = torch.from_numpy(a_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-        out = torch.empty((M, n), dtype=torch.bfloat16, device=dev)
-        out_pinned = torch.empty((M, n), dtype=torch.bfloat16).pin_memory()
-        tactic = fi.default_tactic(M, n, k)
-        info = fi.resolve_tactic(M, n, k, tactic)
-        cases.append(dict(n=n, k=k, Wq=Wq, Ws=Ws, g=g, A=A, A_pinned=A_pinned, out=out,
-                          out_pinned=out_pinned, tactic=tactic, info=info,
-                          bytes=algorithmic_bytes(M, n, k)))
-    ws_bytes = max(c["info"]["workspace_bytes"] for c in cases)
+        shared = dict(Wq=Wq, Ws=Ws, g=g,
+                      A=torch.from_numpy(a_host.view(np.int16)).view(torch.bfloat16).to(dev),
+                      A_pinned=torch.from_numpy(a_host.view(np.int16)).view(torch.bfloat16).pin_memory(),
+                      out_pinned=torch.empty((M, n), dtype=torch.bfloat16).pin_memory())
+        for S in SPLITS:
+            cases.append(make_case(n, k, fi.make_tactic(fi.KIND_GEMV, S, 0, 0), shared))
+        defaults.append(make_case(n, k, fi.default_tactic(M, n, k), shared))
+    ws_bytes = max(c["info"]["workspace_bytes"] for c in cases + defaults)
     ws = torch.empty(max(ws_bytes, 256) // 4 + 64, dtype=torch.float32, device=dev)
     fi.set_workspace(ws)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_out = torch.empty((), dtype=torch.int32, device=dev)
     torch.cuda.synchronize(dev)
 
     # one CUDA graph per shape holding the library call (1 or 2 kernels)
     with torch.cuda.stream(stream):
-        for c in cases:
+        for c in cases + defaults:
             fi.mm_bf16_fp4(c["A"], c["Wq"], c["Ws"], c["g"], tactic=c["tactic"], out=c["out"])
         torch.cuda.synchronize(dev)
-        for c in cases:
+        for c in cases + defaults:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, stream=stream):
                 fi.mm_bf16_fp4(c["A"], c["Wq"], c["Ws"], c["g"], tactic=c["tactic"], out=c["out"])
             c["graph"] = graph
     torch.cuda.synchronize(dev)
 
-    def device_pass(steps: int, e2e: bool):
+    flush.fill_(1)
+
+    def device_pass(steps: int, e2e: bool, cs=None):
+        cs = cases if cs is None else cs
         evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in cases] for _ in range(steps)]
+                for _ in cs] for _ in range(steps)]
         with torch.cuda.stream(stream):
             for st in range(steps):
-                for ci, c in enumerate(cases):
-                    flush.fill_(st & 0xFF)  # evict L2 (2x its 126 MB) outside the timed interval
+                for ci, c in enumerate(cs):
+                    # evict L2 (2x its 126 MB) with a read, outside the timed interval; a read
+                    # leaves clean lines, so no write-back lands inside the timed call
+                    torch.amax(flush, dim=0, out=flush_out)
                     e0, e1 = evs[st][ci]
                     e0.record(stream)
                     if e2e:
@@ -205,9 +217,9 @@ def run_fi(args, rank: int, world: int) -> dict | None:
         dist.barrier()
     e2e_steps = max(5, args.steps // 4)
     e2e_times = times_us(device_pass(e2e_steps, True))
+    def_times = times_us(device_pass(args.steps, False, defaults))
 
-    per_call = [sum(row[ci] for row in dev_times) for ci in range(len(cases))]  # total us per shape
-    total_us = sum(per_call)
+    total_us = sum(sum(row) for row in dev_times)
     e2e_total_us = sum(sum(row) for row in e2e_times)
     if world > 1:
         t = torch.tensor([total_us, e2e_total_us], dtype=torch.float64, device=dev)
@@ -221,16 +233,26 @@ def run_fi(args, rank: int, world: int) -> dict | None:
 
     if rank != 0:
         return None
-    per_shape = []
-    for ci, c in enumerate(cases):
-        ts = [row[ci] for row in dev_times]
-        med = statistics.median(ts)
-        gbs = c["bytes"] / (med * 1e-6) / 1e9
-        per_shape.append({"n": c["n"], "k": c["k"], "us_median": round(med, 3),
-                          "us_mean": round(statistics.fmean(ts), 3), "gbs_median": round(gbs, 1),
-                          "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                          "tactic": fi.tactic_fields(c["tactic"]) | {"splits": c["info"]["splits"],
-                                                                     "variant": c["info"]["variant"]}})
+
+    def summarize(cs, times):
+        rows = []
+        for ci, c in enumerate(cs):
+            ts = [row[ci] for row in times]
+            med = statistics.median(ts)
+            gbs = c["bytes"] / (med * 1e-6) / 1e9
+            info = c["info"]
+            rows.append({"n": c["n"], "k": c["k"], "splits": info["splits"],
+                         "requested_splits": fi.tactic_fields(c["tactic"])["splits"],
+                         "rows_per_warp": info["variant"] & 0xF, "warps_per_row": info["variant"] >> 4,
+                         "us_median": round(med, 3), "us_mean": round(statistics.fmean(ts), 3),
+                         "gbs_median": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                         "tflops_median": round(2 * M * c["n"] * c["k"] / (med * 1e-6) / 1e12, 4)})
+        return rows
+
+    per_call = summarize(cases, dev_times)
+    default_rows = summarize(defaults, def_times)
+    def_total = sum(sum(row) for row in def_times)
+    def_bytes = sum(c["bytes"] for c in defaults)
     achieved = step_bytes / (total_us / args.steps * 1e-6) / 1e9
     traffic = None
     if NCU_TRAFFIC["source_sha256"] == _gemv_source_sha() and NCU_TRAFFIC["bytes"]:
@@ -250,14 +272,17 @@ def run_fi(args, rank: int, world: int) -> dict | None:
         "data": "synthetic",
         "config": {
             "workload": "serving-class decode GEMV, m=1, n x k in " + ", ".join(f"{n}x{k}" for n, k in SHAPES),
-            "m": M, "tactic": "library default per shape", "weights": "N(0,0.02) -> NVFP4",
+            "m": M, "tactic": "GEMV, split-K S in {1,2,4,8,device-sized} per shape (25 calls per step)",
+            "weights": "N(0,0.02) -> NVFP4",
             "activations": "N(0,1) -> bf16", "seed": 0,
-            "l2": "flushed before every call (256 MiB write, outside the timed interval)",
+            "l2": "flushed before every call (256 MiB read, outside the timed interval)",
             "timing": "CUDA-graph replay per call, CUDA events on the launching stream",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         },
-        "us_per_call": {f"{p['n']}x{p['k']}": p["us_median"] for p in per_shape},
-        "per_shape": per_shape,
+        "us_per_call": {f"{p['n']}x{p['k']}": p["us_median"] for p in default_rows},
+        "default_tactic": {"value": round(def_bytes * args.steps / (def_total * 1e-6) / 1e9, 2), "unit": "GB/s",
+                           "per_shape": default_rows},
+        "per_call": per_call,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": sum(2 * M * c["k"] for c in cases),
                 "d2h_bytes_per_step": sum(2 * M * c["n"] for c in cases),
@@ -334,11 +359,19 @@ def run_reference(args) -> dict:
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["fi", "reference"], default="fi")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
+    ap.add_argument("--shapes", default=None,
+                    help="comma-separated n x k subset of the workload, e.g. 4096x14336 (profiling runs)")
+    ap.add_argument("--splits", default=None, help="comma-separated subset of the split menu (0 = device-sized)")
     args = ap.parse_args(argv)
+    global SHAPES, SPLITS
+    if args.shapes:
+        SHAPES = [tuple(int(v) for v in sh.split("x")) for sh in args.shapes.split(",")]
+    if args.splits:
+        SPLITS = [int(v) for v in args.splits.split(",")]
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 

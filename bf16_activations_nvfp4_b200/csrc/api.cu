@@ -83,69 +83,113 @@ static int check_arch() {
 
 // ----------------------------------------------------------------- tactics
 
-// Device-sized split: the smallest S that puts at least this many weight-streaming warps
-// on every SM (PR #4038 measured saturation at ~20 warps/SM on SM12x; re-measured for B200).
+// Device-sized parallelism: enough weight-streaming warps on every SM to keep HBM busy
+// (PR #4038 measured saturation at ~20 warps/SM on SM12x and sized split-K from the device).
 constexpr int kKneeWarpsPerSm = 20;
-// A split keeps at least this many 32-k chunks so that its warps have work for most lanes.
-constexpr int64_t kMinChunksPerSplit = 8;
+// A warp keeps at least this many 32-k chunks of a row (one full warp step) so that its
+// lanes have work when the k range is divided among warps or splits.
+constexpr int64_t kMinChunksPerWarp = 32;
+// Shared memory per CTA the device-sized split aims for (three CTAs per SM fit).
+constexpr int64_t kKneeSmemPerCta = 72 * 1024;
 // Largest m the default table sends to the GEMV.
 constexpr int64_t kDefaultGemvMaxM = 32;
 
 static int gemv_default_rows(int64_t n) { return n >= 4096 ? 2 : 1; }
 
+// Smallest power of two KW <= maxKW (and <= 8) with RG * KW * S >= target.
+static int64_t auto_kw(int64_t RG, int64_t S, int64_t C, int64_t target) {
+  int64_t KW = 1;
+  while (KW < 8 && RG * KW * S < target && (C / S) / (KW * 2) >= kMinChunksPerWarp) KW *= 2;
+  return KW;
+}
+
+// Device-sized split for rows-per-warp R: the in-CTA split KW first (no second kernel), then
+// the fewest global splits S that reach the target warp count, raised until `m_fit`
+// activation rows of a split fit the shared-memory staging. Depends on (n, k, SMs, m_fit).
+static void gemv_knee(int64_t n, int64_t k, int sms, int64_t m_fit, int R, int64_t KW_req, int64_t* S_out,
+                      int64_t* KW_out) {
+  const int64_t C = k / kChunkK;
+  const int64_t RG = (n + R - 1) / R;
+  const int64_t target = (int64_t)kKneeWarpsPerSm * sms;
+  const int64_t KW = KW_req ? KW_req : auto_kw(RG, 1, C, target);
+  const int64_t want = (target + RG * KW - 1) / (RG * KW > 0 ? RG * KW : 1);
+  int64_t cap = C / (kMinChunksPerWarp * KW);
+  if (cap < 1) cap = 1;
+  int64_t S = want < 1 ? 1 : (want > cap ? cap : want);
+  while (S < C && gemv_smem_bytes(m_fit, ((C + S - 1) / S) * kChunkK, R) > kKneeSmemPerCta) ++S;
+  *S_out = S;
+  *KW_out = KW;
+}
+
 static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms, fi_tactic_info* out);
 
+// The built-in table. m = 1, 2..8 and 9..32 are separate buckets: the tactic (and so the bits
+// of a row) is the same for every m inside a bucket.
 static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms) {
-  (void)n;
-  (void)k;
-  (void)num_sms;
-  if (m <= kDefaultGemvMaxM) return FI_TACTIC(FI_KIND_GEMV, 0, 0, 0);
+  if (m <= kDefaultGemvMaxM) {
+    const int64_t m_fit = m <= 1 ? 1 : (m <= 8 ? 8 : kGemvMaxM);
+    const int R = (m_fit > 16 && gemv_default_rows(n) > 2) ? 2 : gemv_default_rows(n);
+    int64_t S = 1, KW = 1;
+    gemv_knee(n, k, num_sms, m_fit, R, 0, &S, &KW);
+    return FI_TACTIC(FI_KIND_GEMV, S, 0, R | (KW << 4));
+  }
   return FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
 }
 
-static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int R_req,
+// GEMV variant byte: low nibble R (weight rows per warp), high nibble KW (warps per row
+// group inside a CTA); 0 in either means automatic. Splits 0 = device-sized, resolved for
+// m <= 32 so that the resolved S (and the bits) never depend on m.
+static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var,
                         int sms, fi_tactic_info* out) {
   if (m > kGemvMaxM)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV tactics support m <= %d (got m=%lld)",
                      kGemvMaxM, (long long)m);
-  const int R = R_req ? R_req : gemv_default_rows(n);
+  const int R = (var & 0xF) ? (var & 0xF) : gemv_default_rows(n);
   if (R != 1 && R != 2 && R != 4)
-    return set_error(FI_ERR_INVALID_ARG, "GEMV variant (rows per warp) must be 0, 1, 2 or 4");
+    return set_error(FI_ERR_INVALID_ARG, "GEMV rows per warp must be 0 (auto), 1, 2 or 4");
+  if (R == 4 && m > 16)
+    return set_error(FI_ERR_INVALID_ARG, "GEMV with 4 rows per warp supports m <= 16");
+  const int KW_req = var >> 4;
+  if (KW_req != 0 && KW_req != 1 && KW_req != 2 && KW_req != 4 && KW_req != 8)
+    return set_error(FI_ERR_INVALID_ARG, "GEMV warps per row group must be 0 (auto), 1, 2, 4 or 8");
   const int64_t C = k / kChunkK;
-  const int64_t row_groups = (n + R - 1) / R;
+  const int64_t RG = (n + R - 1) / R;
+  int64_t KW = KW_req;
   int64_t S = S_req;
   if (S == 0) {
-    const int64_t want = ((int64_t)kKneeWarpsPerSm * sms + row_groups - 1) / (row_groups > 0 ? row_groups : 1);
-    int64_t cap = C / kMinChunksPerSplit;
-    if (cap < 1) cap = 1;
-    S = want < 1 ? 1 : (want > cap ? cap : want);
-    // keep the shared-memory staging of 8 activation rows within budget without making S
-    // depend on m (so the device-sized split is the same for every m <= 8)
-    while (S < C && gemv_smem_bytes(8, ((C + S - 1) / S) * kChunkK) > kSmemBudget) ++S;
-  } else if (C > 0 && S > C) {
-    return set_error(FI_ERR_INVALID_ARG, "splits=%lld exceeds k/32=%lld", (long long)S, (long long)C);
+    gemv_knee(n, k, sms, kGemvMaxM, R, KW_req, &S, &KW);
+  } else {
+    if (C > 0 && S > C)
+      return set_error(FI_ERR_INVALID_ARG, "splits=%lld exceeds k/32=%lld", (long long)S, (long long)C);
+    if (KW == 0) KW = auto_kw(RG, S, C, (int64_t)kKneeWarpsPerSm * sms);
   }
   if (S < 1) S = 1;
+  if (C > 0 && KW > C / S)
+    return set_error(FI_ERR_INVALID_ARG, "warps per row group (%lld) exceeds the %lld k-chunks of a split",
+                     (long long)KW, (long long)(C / S));
   const int64_t klen_max = ((C + S - 1) / S) * kChunkK;
-  const int64_t smem = gemv_smem_bytes(m, klen_max);
+  const int64_t smem = gemv_smem_bytes(m, klen_max, R);
   if (smem > kSmemBudget)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE,
                      "GEMV: m=%lld with k/splits=%lld needs %lld B of shared memory (> %d); use more splits",
                      (long long)m, (long long)klen_max, (long long)smem, kSmemBudget);
   int ctas = ctas_req;
   if (ctas == 0) {
-    ctas = (int)((227 * 1024) / (smem + 1024));
-    if (ctas > 4) ctas = 4;
+    // leave room on every SM for the PDL-launched reduce when the tactic splits
+    ctas = S > 1 ? 3 : 4;
+    const int fit = (int)((227 * 1024) / (smem + 1024));
+    if (ctas > fit) ctas = fit;
     if (ctas < 1) ctas = 1;
   }
-  const int64_t cta_rows = (row_groups + kGemvWarps - 1) / kGemvWarps;
+  const int64_t NS = kGemvWarps / KW;
+  const int64_t cta_rows = (RG + NS - 1) / NS;
   int64_t slots = ((int64_t)sms * ctas) / S;
   if (slots < 1) slots = 1;
   const int64_t grid_x = cta_rows < slots ? cta_rows : slots;
   out->kind = FI_KIND_GEMV;
   out->splits = (int32_t)S;
   out->ctas_per_sm = ctas;
-  out->variant = R;
+  out->variant = (int32_t)(R | (KW << 4));
   out->grid_x = (int32_t)(grid_x > 0 ? grid_x : 1);
   out->grid_y = (int32_t)S;
   out->threads = kGemvThreads;
@@ -234,6 +278,14 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
   if (m < 0 || n < 0 || k < 0) return set_error(FI_ERR_INVALID_ARG, "negative size");
   if (k % 32 != 0) return set_error(FI_ERR_UNSUPPORTED_SHAPE, "k=%lld is not a multiple of 32", (long long)k);
   if (m == 0 || n == 0) return FI_OK;
+  if (k == 0) {  // the empty sum: out = 0; A and the weights are empty and may be null
+    if (!out) return set_error(FI_ERR_INVALID_ARG, "null pointer argument");
+    int rc0 = check_arch();
+    if (rc0 != FI_OK) return rc0;
+    if (cudaMemsetAsync(out, 0, (size_t)(m * n) * sizeof(uint16_t), stream) != cudaSuccess)
+      return set_cuda_error("cudaMemsetAsync(out)");
+    return FI_OK;
+  }
   if (!A || !Wq || !Wscale || !gscale || !out) return set_error(FI_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned(A, 16) || !aligned(Wq, 16)) return set_error(FI_ERR_INVALID_ARG, "A and Wq must be 16-byte aligned");
   if (!aligned(Wscale, 2) || !aligned(out, 2) || !aligned(gscale, 4))
@@ -245,11 +297,6 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
   fi_tactic_info info;
   rc = resolve(m, n, k, tactic, sms, &info);
   if (rc != FI_OK) return rc;
-  if (k == 0) {
-    if (cudaMemsetAsync(out, 0, (size_t)(m * n) * sizeof(uint16_t), stream) != cudaSuccess)
-      return set_cuda_error("cudaMemsetAsync(out)");
-    return FI_OK;
-  }
   float* partials = nullptr;
   if (info.workspace_bytes > 0) {
     const size_t need = (size_t)info.workspace_bytes;
@@ -277,8 +324,11 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.n = n;
     a.k = k;
     a.splits = info.splits;
-    a.rows_per_warp = info.variant;
+    a.kw = info.variant >> 4;
+    a.rows_per_warp = info.variant & 0xF;
     a.grid_x = info.grid_x;
+    a.ctas_per_sm = info.ctas_per_sm;
+    a.num_sms = sms;
     a.smem_bytes = info.smem_bytes;
     rc = launch_gemv(a, stream);
     if (rc != FI_OK) return rc;
@@ -356,23 +406,27 @@ int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, 
   clear_error();
   const int sms = sms_or_device(num_sms);
   if (sms <= 0) return set_error(FI_ERR_CUDA, "no device to query the SM count from");
-  int count = 0;
+  // the split menu {1, 2, 4, 8, device-sized} for each rows-per-warp choice, plus every
+  // in-CTA split for one row per warp; entries resolving to the same launch are listed once
+  int64_t cand[32];
+  int nc = 0;
   const int splits[] = {1, 2, 4, 8, 0};
-  const int rows[] = {1, 2, 4};
-  for (int R : rows) {
-    int64_t seen[8];
-    int nseen = 0;
-    for (int S : splits) {
-      const int64_t t = FI_TACTIC(FI_KIND_GEMV, S, 0, R);
-      fi_tactic_info info;
-      if (resolve(m, n, k, t, sms, &info) != FI_OK) continue;
-      bool dup = false;  // the device-sized split may coincide with a power of two
-      for (int i = 0; i < nseen; ++i) dup |= (seen[i] == info.splits);
-      if (dup) continue;
-      seen[nseen++] = info.splits;
-      if (count < cap && out) out[count] = t;
-      ++count;
-    }
+  for (int R : {1, 2, 4})
+    for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, R);
+  for (int KW : {1, 2, 4, 8}) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, 1, 0, 1 | (KW << 4));
+  fi_tactic_info seen[32];
+  int nseen = 0, count = 0;
+  for (int c = 0; c < nc; ++c) {
+    fi_tactic_info info;
+    if (resolve(m, n, k, cand[c], sms, &info) != FI_OK) continue;
+    bool dup = false;
+    for (int i = 0; i < nseen; ++i)
+      dup |= seen[i].kind == info.kind && seen[i].splits == info.splits && seen[i].variant == info.variant &&
+             seen[i].ctas_per_sm == info.ctas_per_sm;
+    if (dup) continue;
+    seen[nseen++] = info;
+    if (count < cap && out) out[count] = cand[c];
+    ++count;
   }
   clear_error();
   return count;

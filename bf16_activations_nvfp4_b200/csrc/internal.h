@@ -28,9 +28,19 @@ constexpr int kWarpK = 32 * kChunkK;          // k per warp step (512 code bytes
 constexpr int kGemvMaxM = 32;
 constexpr int kSmemBudget = 200 * 1024;       // dynamic shared memory we allow per CTA
 
-// Shared memory the GEMV needs for m activation rows over klen k (f16 values plus one
-// fp32 power-of-two scale per 16-block).
-inline int64_t gemv_smem_bytes(int64_t m, int64_t klen) { return m * klen * 2 + m * (klen / 16) * 4; }
+// Activation rows the GEMV kernel instance for m is compiled for (1, 2, 4, ..., 32).
+inline int gemv_mt(int64_t m) {
+  int mt = 1;
+  while (mt < m) mt *= 2;
+  return mt;
+}
+
+// Shared memory the GEMV needs: m activation rows over klen k (f16 values plus one fp32
+// power-of-two scale per 16-block) and the in-CTA split-K combine buffer
+// (2 parities x 8 warps x R rows x MT activation rows, fp32).
+inline int64_t gemv_smem_bytes(int64_t m, int64_t klen, int R) {
+  return m * klen * 2 + m * (klen / 16) * 4 + 2 * 8 * (int64_t)R * gemv_mt(m) * 4;
+}
 
 struct GemvArgs {
   const uint16_t* A;
@@ -40,9 +50,12 @@ struct GemvArgs {
   uint16_t* out;       // used when splits == 1
   float* partials;     // [splits, m, n] when splits > 1
   int64_t m, n, k;
-  int splits;
-  int rows_per_warp;
-  int grid_x;
+  int splits;         // S: global K splits (grid.y)
+  int kw;             // KW: warps sharing one row group inside a CTA (1, 2, 4, 8)
+  int rows_per_warp;  // R
+  int grid_x;         // CTAs per split wanted by the tactic (capped by occupancy at launch)
+  int ctas_per_sm;
+  int num_sms;
   int smem_bytes;
 };
 int launch_gemv(const GemvArgs& a, cudaStream_t stream);

@@ -49,33 +49,48 @@ def test_default_gemv_tactic_resolves_for_decode_shapes(n, k):
     assert 1 <= info["splits"] <= k // 32
     # one wave: the grid never asks for more CTAs than the SMs hold at the tactic's occupancy
     assert info["grid_x"] * info["grid_y"] <= B200_SMS * info["ctas_per_sm"]
-    # every weight row is covered by some warp of the grid
-    rows_per_cta = 8 * info["variant"]
-    assert info["grid_x"] * rows_per_cta >= min(n, rows_per_cta)
+    # the grid has a CTA for every 8/KW row groups of R rows, up to one wave
+    R, KW = info["variant"] & 0xF, info["variant"] >> 4
+    rows_per_cta_pass = (8 // KW) * R
+    assert info["grid_x"] == min(-(-n // rows_per_cta_pass), B200_SMS * info["ctas_per_sm"] // info["splits"])
     assert info["workspace_bytes"] == (info["splits"] * n * 4 if info["splits"] > 1 else 0)
 
 
 def test_device_sized_split_reaches_the_knee_and_is_m_independent():
-    for n, k in [(512, 2048), (1024, 4096), (4096, 14336), (14336, 4096)]:
-        splits = {fi.resolve_tactic(m, n, k, fi.make_tactic(fi.KIND_GEMV, 0, 0, 1), B200_SMS)["splits"]
-                  for m in (1, 2, 4, 8)}
-        assert len(splits) == 1, (n, k, splits)
-        S = splits.pop()
-        warps = n * S  # one row per warp with variant 1
-        assert warps >= 20 * B200_SMS or S == max(1, (k // 32) // 8), (n, k, S)
-        if S > 1:
-            assert n * (S - 1) < 20 * B200_SMS or gemv_smem_needs_split(k, S - 1)
+    """The device-sized tactic (splits=0) resolves to the same S and in-CTA split KW for every
+    m the GEMV takes, and gives the device at least ~20 streaming warps per SM unless the
+    k range cannot be divided further."""
+    for n, k in [(512, 2048), (1024, 4096), (4096, 14336), (14336, 4096), (2048, 7168), (10304, 2688)]:
+        for R in (1, 2):
+            t = fi.make_tactic(fi.KIND_GEMV, 0, 0, R)
+            got = {(i["splits"], i["variant"]) for i in
+                   (fi.resolve_tactic(m, n, k, t, B200_SMS) for m in (1, 2, 3, 8, 16, 32 if R < 4 else 16))}
+            assert len(got) == 1, (n, k, R, got)
+            S, var = got.pop()
+            KW = var >> 4
+            warps = -(-n // R) * KW * S
+            assert warps >= 20 * B200_SMS or (k // 32) // (S * KW) < 64, (n, k, R, S, KW)
 
 
-def gemv_smem_needs_split(k, S):
-    klen = -(-(k // 32) // S) * 32
-    return 8 * klen * 2 + 8 * (klen // 16) * 4 > 200 * 1024
+def test_default_table_is_constant_within_m_buckets():
+    for n, k in [(4096, 14336), (14336, 4096), (512, 2048)]:
+        for bucket in ([1], [2, 3, 5, 8], [9, 16, 31, 32]):
+            ts = {fi.default_tactic(m, n, k, B200_SMS) for m in bucket}
+            assert len(ts) == 1, (n, k, bucket, ts)
+
+
+def test_default_m1_serving_shapes_need_no_second_kernel():
+    for n, k in [(2048, 7168), (4096, 4096), (4096, 14336), (14336, 4096), (10304, 2688), (152064, 5120)]:
+        info = fi.resolve_tactic(1, n, k, fi.default_tactic(1, n, k, B200_SMS), B200_SMS)
+        assert info["splits"] == 1 and info["workspace_bytes"] == 0, (n, k, info)
 
 
 def test_explicit_splits_are_kept():
     for S in (1, 2, 4, 8):
         info = fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, S, 0, 2), B200_SMS)
-        assert info["splits"] == S and info["variant"] == 2
+        assert info["splits"] == S and info["variant"] & 0xF == 2
+    info = fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, 2, 3, 1 | (4 << 4)), B200_SMS)
+    assert (info["splits"], info["ctas_per_sm"], info["variant"]) == (2, 3, 0x41)
 
 
 def test_list_tactics_unique_and_valid():
@@ -100,6 +115,9 @@ def test_workspace_bytes():
     (1, 64, 64, 1 << 30, -1),                             # out-of-range code
     (-1, 64, 64, -1, -1),                                 # negative size
     (32, 64, 14336, fi.make_tactic(0, 1, 0, 1), -2),      # A slice does not fit shared memory
+    (32, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),       # 4 rows per warp only up to m = 16
+    (1, 64, 4096, fi.make_tactic(0, 1, 0, 1 | (3 << 4)), -1),   # KW must be a power of two <= 8
+    (1, 64, 128, fi.make_tactic(0, 1, 0, 1 | (8 << 4)), -1),    # KW > k/32 chunks
 ])
 def test_resolve_rejects(m, n, k, tactic, status):
     with pytest.raises(fi.FiError) as e:

@@ -64,9 +64,11 @@ def test_parity_spanning_tiles(m, n, k, seed):
 
 
 def _exact_case(m, n, k, seed):
-    """Small-integer activations and weights e2m1 * 2^e * 2^-9 (gscale 2^-9): every product is
-    a multiple of 2^-10 and every partial sum of <= k terms stays far below 2^14, so fp32
-    accumulation is exact in any order and the result is a bf16-representable value."""
+    """Small-integer activations (|a| <= 2) and weights e2m1 * 448 * 2^-j * 2^-9 with one
+    block at the tensor maximum, so gscale = 2^-9 exactly and every block scale is 448 * 2^-j.
+    Every product is then a multiple of 7 * 2^(5-jmax) * gscale-free units and every partial
+    sum of <= k terms stays below 2^24 of those units: fp32 accumulation is exact in any
+    order, so every tactic must return exactly bf16_rn(exact result)."""
     rng = np.random.default_rng(seed)
     A = inputs.to_bf16_bits(rng.integers(-2, 3, (m, k)).astype(np.float32))
     E2M1 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
@@ -74,7 +76,7 @@ def _exact_case(m, n, k, seed):
     W[:, ::16] = 6.0
     e = rng.integers(-2, 1, (n, k // 16)).astype(np.float32)
     W *= np.repeat(np.exp2(e), 16, axis=1) * np.float32(448 * 2.0 ** -9)
-    W[0, 0] = np.float32(6 * 448 * 2.0 ** -9)
+    W[0, 0:16] = np.abs(W[0, 0:16]) / np.exp2(e[0, 0])  # block 0 at scale 448: tensor amax 5.25
     return A, W
 
 
@@ -84,8 +86,8 @@ def test_integer_exact_bitwise(m, n, k):
     Wq, Ws, g = oracle.pack(W)
     assert g == np.float32(2.0 ** -9)
     ref = oracle.mm(A, Wq, Ws, g)
+    assert np.array_equal(ref.astype(np.float32).astype(np.float64), ref)  # exact in fp32
     want = np.array([[oracle.f32_to_bf16_bits(v) for v in row] for row in ref.astype(np.float32)], np.uint16)
-    assert np.array_equal(_gpu.bits_to_f64(want), ref)  # the exact result is bf16-representable
     dw = fi.pack_weights(torch.from_numpy(W).cuda())
     for t in _tactics(m, n, k):
         got = _mm(A, dw, t)
@@ -122,13 +124,27 @@ def test_batch_invariance_rows_do_not_depend_on_m(splits):
 
 
 def test_rows_per_warp_and_occupancy_do_not_change_bits():
+    """Only the kind, S and the in-CTA split KW fix the arithmetic: rows per warp and CTAs per
+    SM only move work between warps and CTAs."""
     m, n, k = 2, 2048, 7168
     A = inputs.activations(m, k, seed=9)
     dw = _gpu.device_weights(n, k, 0)
     for S in (1, 3):
-        outs = [_mm(A, dw, fi.make_tactic(GEMV, S, c, R)) for R in (1, 2, 4) for c in (1, 2, 4)]
-        for o in outs[1:]:
-            assert np.array_equal(o, outs[0]), S
+        for KW in (1, 2):
+            outs = [_mm(A, dw, fi.make_tactic(GEMV, S, c, R | (KW << 4))) for R in (1, 2, 4) for c in (1, 2, 4)]
+            for o in outs[1:]:
+                assert np.array_equal(o, outs[0]), (S, KW)
+
+
+def test_in_cta_split_counts_agree_within_tolerance():
+    m, n, k = 3, 1024, 8192
+    A = inputs.activations(m, k, seed=2, outliers=True)
+    W, (Wq, Ws, g) = _gpu.weights(n, k, 2)
+    ref = oracle.mm(A, Wq, Ws, g)
+    dw = _gpu.device_weights(n, k, 2)
+    for S in (1, 2):
+        for KW in (1, 2, 4, 8):
+            _gpu.assert_within_tolerance(_mm(A, dw, fi.make_tactic(GEMV, S, 0, 1 | (KW << 4))), ref, f"S={S} KW={KW}")
 
 
 def test_split_counts_agree_within_tolerance():
