@@ -1,18 +1,24 @@
 #!/usr/bin/env python
 """Benchmark: m=1 bf16 x NVFP4 decode GEMV on B200 (the serving-class decode shapes).
 
-One step = the five serving decode shapes n x k in {2048x7168, 4096x4096, 4096x14336,
-14336x4096, 10304x2688} at m=1 (PR #4038, "Split-K on the #3597 decode shapes", first
-table), each called through the library's public op with the GEMV tactic at split-K
-S in {1, 2, 4, 8, device-sized}: 25 calls. Every call is a CUDA-graph replay timed with
-CUDA events on its stream, with L2 flushed (a 256 MiB read) before it, as decode serving
-runs with a cold L2 (PR #4038, Performance: "Median GPU time over CUDA-graph replays with
-a cold L2 cache"). The library's default tactic per shape is timed in a second pass and
-reported beside the step.
+Workload (PR #4038, "Split-K on the #3597 decode shapes", first table): the five serving
+decode shapes n x k in {2048x7168, 4096x4096, 4096x14336, 14336x4096, 10304x2688} at m=1,
+each called through the library's public op with the GEMV tactic at split-K
+S in {1, 2, 4, 8, device-sized}. One step = those 25 calls.
 
-value = algorithmic bytes of all calls / their summed device time (GB/s); algorithmic
-bytes per call = n*k/2 + n*k/16 + 2*m*k + 2*m*n (packed codes, E4M3 scales, bf16 A and
-out). Inputs are synthetic, seeded (A ~ N(0,1) in bf16, W ~ N(0, 0.02) quantised to NVFP4).
+Method (PR #4038, Performance: "Median GPU time over CUDA-graph replays with a cold L2
+cache, as in serving"):
+  * the step is captured once as a CUDA graph; consecutive calls are chained with
+    programmatic dependent launch, as in a decode step where one GEMV follows another;
+  * L2 is kept cold without flushing by rotating every call over its own copy of the packed
+    weights; the copies of each shape total >= 300 MB (> 2x the 126 MB L2), so no weight byte
+    is in L2 when it is read (inputs larger than L2);
+  * K replays of the step graph are timed with CUDA events on the launching stream;
+  * per-call µs: a graph of repeated calls of one (shape, split) over its rotating copies.
+
+value = algorithmic bytes of all calls / their device time (GB/s); algorithmic bytes per call
+= n*k/2 + n*k/16 + 2*m*k + 2*m*n (packed codes, E4M3 scales, bf16 A and out). Synthetic
+seeded inputs: A ~ N(0,1) in bf16, W ~ N(0, 0.02) quantised to NVFP4 by the library.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fi|reference]
 
@@ -27,9 +33,8 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
+import threading
 import time
 
 import numpy as np
@@ -41,7 +46,7 @@ METRIC = "µs/call and achieved HBM GB/s (% of B200 peak) for m=1 bf16×NVFP4 GE
 SHAPES = [(2048, 7168), (4096, 4096), (4096, 14336), (14336, 4096), (10304, 2688)]
 SPLITS = [1, 2, 4, 8, 0]  # 0 = device-sized
 M = 1
-FLUSH_BYTES = 256 << 20
+COLD_BYTES = 300 << 20  # per-shape footprint of the rotating weight copies
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes per launch of the GEMV kernel (dram__bytes_read.sum + dram__bytes_write.sum)
@@ -76,53 +81,51 @@ def _gemv_source_sha() -> str:
 # ------------------------------------------------------------------ clock sampling
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+    """NVML sampling (every 10 ms) of SM clock and throttle reasons while the timed region runs."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, index: int):
         self.index = index
-        self.proc = None
-        self.file = None
+        self.samples = []
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+
+    def _run(self, handle, nvml):
+        while not self._stop.is_set():
+            try:
+                mhz = nvml.nvmlDeviceGetClockInfo(handle, nvml.NVML_CLOCK_SM)
+                reasons = nvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(0.01)
 
     def __enter__(self):
-        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.file, stderr=subprocess.DEVNULL)
+            import pynvml as nvml
+            nvml.nvmlInit()
+            handle = nvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = nvml.nvmlDeviceGetMaxClockInfo(handle, nvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, args=(handle, nvml), daemon=True)
+            self._thread.start()
         except Exception:
-            self.proc = None
-        time.sleep(0.3)
+            self._thread = None
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-        self.file.flush()
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=2)
 
     def summary(self) -> dict | None:
-        try:
-            with open(self.file.name) as f:
-                rows = [[c.strip() for c in line.split(",")] for line in f if line.strip()]
-            os.unlink(self.file.name)
-        except Exception:
+        if not self.samples:
             return None
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({name for _, r in self.samples for name, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "NVML, 10 ms"}
 
 
 # ------------------------------------------------------------------------ fi arm
@@ -137,127 +140,143 @@ def run_fi(args, rank: int, world: int) -> dict | None:
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(dev)
+    peaks = _peaks()
 
-    def make_case(n, k, tactic, shared):
-        info = fi.resolve_tactic(M, n, k, tactic)
-        return dict(shared, n=n, k=k, tactic=tactic, info=info, bytes=algorithmic_bytes(M, n, k),
-                    out=torch.empty((M, n), dtype=torch.bfloat16, device=dev))
-
-    cases, defaults = [], []
+    # ---- inputs: packed weights (with rotating copies), activations, outputs
+    shapes = []
     for n, k in SHAPES:
         W = torch.from_numpy(inputs.weights(n, k, seed=0)).to(dev)
         Wq, Ws, g = fi.pack_weights(W)
         del W
+        b = algorithmic_bytes(M, n, k)
+        ncopy = max(len(SPLITS), -(-COLD_BYTES // b))
+        copies = [(Wq, Ws)] + [(Wq.clone(), Ws.clone()) for _ in range(ncopy - 1)]
         a_host = inputs.activations(M, k, seed=0)
-        shared = dict(Wq=Wq, Ws=Ws, g=g,
-                      A=torch.from_numpy(a_host.view(np.int16)).view(torch.bfloat16).to(dev),
-                      A_pinned=torch.from_numpy(a_host.view(np.int16)).view(torch.bfloat16).pin_memory(),
-                      out_pinned=torch.empty((M, n), dtype=torch.bfloat16).pin_memory())
-        for S in SPLITS:
-            cases.append(make_case(n, k, fi.make_tactic(fi.KIND_GEMV, S, 0, 0), shared))
-        defaults.append(make_case(n, k, fi.default_tactic(M, n, k), shared))
-    ws_bytes = max(c["info"]["workspace_bytes"] for c in cases + defaults)
+        shapes.append(dict(n=n, k=k, g=g, copies=copies, bytes=b,
+                           A=torch.from_numpy(a_host.view(np.int16)).view(torch.bfloat16).to(dev),
+                           A_pinned=torch.from_numpy(a_host.view(np.int16)).view(torch.bfloat16).pin_memory(),
+                           out=torch.empty((M, n), dtype=torch.bfloat16, device=dev),
+                           out_pinned=torch.empty((M, n), dtype=torch.bfloat16).pin_memory()))
+    calls = []  # the step: every shape at every split
+    for si, sh in enumerate(shapes):
+        for ci, S in enumerate(SPLITS):
+            t = fi.make_tactic(fi.KIND_GEMV, S, 0, 0)
+            calls.append(dict(shape=si, copy=ci, tactic=t, info=fi.resolve_tactic(M, sh["n"], sh["k"], t)))
+    defaults = [dict(shape=si, tactic=fi.default_tactic(M, sh["n"], sh["k"])) for si, sh in enumerate(shapes)]
+    for d in defaults:
+        sh = shapes[d["shape"]]
+        d["info"] = fi.resolve_tactic(M, sh["n"], sh["k"], d["tactic"])
+    ws_bytes = max(c["info"]["workspace_bytes"] for c in calls + defaults)
     ws = torch.empty(max(ws_bytes, 256) // 4 + 64, dtype=torch.float32, device=dev)
     fi.set_workspace(ws)
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
-    flush_out = torch.empty((), dtype=torch.int32, device=dev)
     torch.cuda.synchronize(dev)
 
-    # one CUDA graph per shape holding the library call (1 or 2 kernels)
-    with torch.cuda.stream(stream):
-        for c in cases + defaults:
-            fi.mm_bf16_fp4(c["A"], c["Wq"], c["Ws"], c["g"], tactic=c["tactic"], out=c["out"])
-        torch.cuda.synchronize(dev)
-        for c in cases + defaults:
+    def call(si, copy, tactic):
+        sh = shapes[si]
+        Wq, Ws = sh["copies"][copy % len(sh["copies"])]
+        fi.mm_bf16_fp4(sh["A"], Wq, Ws, sh["g"], tactic=tactic, out=sh["out"])
+
+    def capture(fn):
+        with torch.cuda.stream(stream):
+            fn()  # warm-up outside capture (sets kernel attributes, checks arguments)
+            torch.cuda.synchronize(dev)
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, stream=stream):
-                fi.mm_bf16_fp4(c["A"], c["Wq"], c["Ws"], c["g"], tactic=c["tactic"], out=c["out"])
-            c["graph"] = graph
-    torch.cuda.synchronize(dev)
-
-    flush.fill_(1)
-
-    def device_pass(steps: int, e2e: bool, cs=None):
-        cs = cases if cs is None else cs
-        evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in cs] for _ in range(steps)]
-        with torch.cuda.stream(stream):
-            for st in range(steps):
-                for ci, c in enumerate(cs):
-                    # evict L2 (2x its 126 MB) with a read, outside the timed interval; a read
-                    # leaves clean lines, so no write-back lands inside the timed call
-                    torch.amax(flush, dim=0, out=flush_out)
-                    e0, e1 = evs[st][ci]
-                    e0.record(stream)
-                    if e2e:
-                        c["A"].copy_(c["A_pinned"], non_blocking=True)
-                        fi.mm_bf16_fp4(c["A"], c["Wq"], c["Ws"], c["g"], tactic=c["tactic"], out=c["out"])
-                        c["out_pinned"].copy_(c["out"], non_blocking=True)
-                    else:
-                        c["graph"].replay()
-                    e1.record(stream)
-        return evs
-
-    def times_us(evs):
+                fn()
         torch.cuda.synchronize(dev)
-        return [[e0.elapsed_time(e1) * 1e3 for (e0, e1) in row] for row in evs]
+        return graph
 
-    times_us(device_pass(args.warmup, False))
-    times_us(device_pass(max(3, args.warmup // 2), True))
+    def time_replays(graph, reps: int) -> list[float]:
+        """Per-replay device time in us, each replay bracketed by events on the stream."""
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        with torch.cuda.stream(stream):
+            for e0, e1 in evs:
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return [e0.elapsed_time(e1) * 1e3 for e0, e1 in evs]
+
+    # ---- the step graph (25 calls)
+    step_graph = capture(lambda: [call(c["shape"], c["copy"], c["tactic"]) for c in calls])
+
+    # ---- per-call graphs: one (shape, tactic) repeated over its rotating copies
+    def per_call_graph(si, tactic):
+        nrep = 2 * len(shapes[si]["copies"])
+        return capture(lambda: [call(si, r, tactic) for r in range(nrep)]), nrep
+
+    case_graphs = [per_call_graph(c["shape"], c["tactic"]) for c in calls]
+    default_graphs = [per_call_graph(d["shape"], d["tactic"]) for d in defaults]
+
+    time_replays(step_graph, args.warmup)
+    for g_, _ in case_graphs + default_graphs:
+        time_replays(g_, 2)
 
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clocks:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         wall0 = time.perf_counter()
-        dev_times = times_us(device_pass(args.steps, False))
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                step_graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
         wall1 = time.perf_counter()
-    torch.cuda.synchronize(dev)
+        total_us = e0.elapsed_time(e1) * 1e3
+        case_us = [statistics.median(time_replays(g_, 15)) / nrep for g_, nrep in case_graphs]
+        default_us = [statistics.median(time_replays(g_, 15)) / nrep for g_, nrep in default_graphs]
     if world > 1:
         dist.barrier()
-    e2e_steps = max(5, args.steps // 4)
-    e2e_times = times_us(device_pass(e2e_steps, True))
-    def_times = times_us(device_pass(args.steps, False, defaults))
 
-    total_us = sum(sum(row) for row in dev_times)
-    e2e_total_us = sum(sum(row) for row in e2e_times)
+    # ---- end to end through the public op with host buffers (eager calls)
+    e2e_steps = max(5, args.steps // 10)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for it in range(2 + e2e_steps):
+            if it == 2:
+                x0.record(stream)
+            for c in calls:
+                sh = shapes[c["shape"]]
+                sh["A"].copy_(sh["A_pinned"], non_blocking=True)
+                call(c["shape"], c["copy"], c["tactic"])
+                sh["out_pinned"].copy_(sh["out"], non_blocking=True)
+        x1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_us = x0.elapsed_time(x1) * 1e3
+
     if world > 1:
-        t = torch.tensor([total_us, e2e_total_us], dtype=torch.float64, device=dev)
+        t = torch.tensor([total_us, e2e_us], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_us, e2e_total_us = float(t[0]), float(t[1])
-    step_bytes = sum(c["bytes"] for c in cases)
+        total_us, e2e_us = float(t[0]), float(t[1])
+    step_bytes = sum(shapes[c["shape"]]["bytes"] for c in calls)
     value = world * step_bytes * args.steps / (total_us * 1e-6) / 1e9
-    e2e_value = world * step_bytes * e2e_steps / (e2e_total_us * 1e-6) / 1e9
-    peaks = _peaks()
-    launches_per_step = sum(1 + (c["info"]["splits"] > 1) for c in cases)
-
+    e2e_value = world * step_bytes * e2e_steps / (e2e_us * 1e-6) / 1e9
+    launches_per_step = sum(1 + (c["info"]["splits"] > 1) for c in calls)
     if rank != 0:
         return None
 
-    def summarize(cs, times):
-        rows = []
-        for ci, c in enumerate(cs):
-            ts = [row[ci] for row in times]
-            med = statistics.median(ts)
-            gbs = c["bytes"] / (med * 1e-6) / 1e9
-            info = c["info"]
-            rows.append({"n": c["n"], "k": c["k"], "splits": info["splits"],
-                         "requested_splits": fi.tactic_fields(c["tactic"])["splits"],
-                         "rows_per_warp": info["variant"] & 0xF, "warps_per_row": info["variant"] >> 4,
-                         "us_median": round(med, 3), "us_mean": round(statistics.fmean(ts), 3),
-                         "gbs_median": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                         "tflops_median": round(2 * M * c["n"] * c["k"] / (med * 1e-6) / 1e12, 4)})
-        return rows
+    def row(si, info, tactic, us):
+        sh = shapes[si]
+        gbs = sh["bytes"] / (us * 1e-6) / 1e9
+        return {"n": sh["n"], "k": sh["k"], "requested_splits": fi.tactic_fields(tactic)["splits"],
+                "splits": info["splits"], "rows_per_warp": info["variant"] & 0xF,
+                "warps_per_row": info["variant"] >> 4, "us": round(us, 3), "gbs": round(gbs, 1),
+                "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                "tflops": round(2 * M * sh["n"] * sh["k"] / (us * 1e-6) / 1e12, 4)}
 
-    per_call = summarize(cases, dev_times)
-    default_rows = summarize(defaults, def_times)
-    def_total = sum(sum(row) for row in def_times)
-    def_bytes = sum(c["bytes"] for c in defaults)
-    achieved = step_bytes / (total_us / args.steps * 1e-6) / 1e9
+    per_call = [row(c["shape"], c["info"], c["tactic"], us) for c, us in zip(calls, case_us)]
+    default_rows = [row(d["shape"], d["info"], d["tactic"], us) for d, us in zip(defaults, default_us)]
+    # dominant kernel: the GEMV alone (split 1: one launch per call, no reduce)
+    s1 = [(shapes[c["shape"]]["bytes"], us) for c, us in zip(calls, case_us) if c["info"]["splits"] == 1]
+    achieved = sum(b for b, _ in s1) / (sum(u for _, u in s1) * 1e-6) / 1e9
     traffic = None
     if NCU_TRAFFIC["source_sha256"] == _gemv_source_sha() and NCU_TRAFFIC["bytes"]:
         traffic = statistics.fmean(NCU_TRAFFIC["bytes"].values())
-    line = {
+    def_bytes = sum(shapes[d["shape"]]["bytes"] for d in defaults)
+    return {
         "metric": METRIC,
         "value": round(value, 2),
         "unit": "GB/s",
@@ -272,44 +291,92 @@ def run_fi(args, rank: int, world: int) -> dict | None:
         "data": "synthetic",
         "config": {
             "workload": "serving-class decode GEMV, m=1, n x k in " + ", ".join(f"{n}x{k}" for n, k in SHAPES),
-            "m": M, "tactic": "GEMV, split-K S in {1,2,4,8,device-sized} per shape (25 calls per step)",
-            "weights": "N(0,0.02) -> NVFP4",
-            "activations": "N(0,1) -> bf16", "seed": 0,
-            "l2": "flushed before every call (256 MiB read, outside the timed interval)",
-            "timing": "CUDA-graph replay per call, CUDA events on the launching stream",
+            "m": M, "calls_per_step": len(calls),
+            "tactics": "GEMV at split-K S in {1,2,4,8,device-sized} for every shape",
+            "weights": "N(0,0.02) -> NVFP4 (library pack)", "activations": "N(0,1) -> bf16", "seed": 0,
+            "l2": "inputs larger than L2: every call reads its own weight copy, >= 300 MB of copies per shape",
+            "timing": "CUDA-graph replays (calls chained with programmatic dependent launch), CUDA events",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         },
-        "us_per_call": {f"{p['n']}x{p['k']}": p["us_median"] for p in default_rows},
-        "default_tactic": {"value": round(def_bytes * args.steps / (def_total * 1e-6) / 1e9, 2), "unit": "GB/s",
+        "us_per_call": {f"{r['n']}x{r['k']}": r["us"] for r in default_rows},
+        "default_tactic": {"value": round(def_bytes / (sum(default_us) * 1e-6) / 1e9, 2), "unit": "GB/s",
                            "per_shape": default_rows},
         "per_call": per_call,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": sum(2 * M * c["k"] for c in cases),
-                "d2h_bytes_per_step": sum(2 * M * c["n"] for c in cases),
-                "how": "public op on device weights; per call: pinned H2D copy of A, the op, D2H copy of out, "
-                       "all between the CUDA events; L2 flushed before each call"},
+                "h2d_bytes_per_step": sum(2 * M * shapes[c["shape"]]["k"] for c in calls),
+                "d2h_bytes_per_step": sum(2 * M * shapes[c["shape"]]["n"] for c in calls),
+                "how": "eager public-op calls; per call a pinned H2D copy of A, the op, a D2H copy of out"},
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-                     "peak_source": peaks["source"] + " (copy bandwidth, burst)",
-                     "note": "per library call: GEMV kernel plus the split-K reduce where the tactic splits"},
+                     "peak_source": peaks["source"] + " copy bandwidth (burst)",
+                     "kernel": "gemv_nvfp4_kernel, split 1 on the five shapes (one launch per call)"},
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall1 - wall0, 3),
     }
-    return line
+
+
+def sweep(args) -> None:
+    """Print per-call µs of every listed tactic for each shape (cold-L2 graph method)."""
+    import torch
+
+    import bf16_activations_nvfp4_b200 as fi
+    from bf16_activations_nvfp4_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    for n, k in SHAPES:
+        W = torch.from_numpy(inputs.weights(n, k, seed=0)).to(dev)
+        Wq, Ws, g = fi.pack_weights(W)
+        del W
+        b = algorithmic_bytes(args.m, n, k)
+        copies = [(Wq, Ws)] + [(Wq.clone(), Ws.clone()) for _ in range(-(-COLD_BYTES // b) - 1)]
+        A = torch.from_numpy(inputs.activations(args.m, k, seed=0).view(np.int16)).view(torch.bfloat16).to(dev)
+        out = torch.empty((args.m, n), dtype=torch.bfloat16, device=dev)
+        tactics = fi.list_tactics(args.m, n, k) + [fi.default_tactic(args.m, n, k)]
+        ws = torch.empty(max(fi.workspace_bytes(args.m, n, k, t) for t in tactics) // 4 + 64, device=dev)
+        for t in tactics:
+            info = fi.resolve_tactic(args.m, n, k, t)
+            nrep = 2 * len(copies)
+            with torch.cuda.stream(stream):
+                fi.mm_bf16_fp4(A, Wq, Ws, g, tactic=t, out=out, workspace=ws)
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=stream):
+                    for r in range(nrep):
+                        q, s_ = copies[r % len(copies)]
+                        fi.mm_bf16_fp4(A, q, s_, g, tactic=t, out=out, workspace=ws)
+                ts = []
+                for _ in range(12):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    graph.replay()
+                    e1.record(stream)
+                    e1.synchronize()
+                    ts.append(e0.elapsed_time(e1) * 1e3 / nrep)
+            us = statistics.median(ts[2:])
+            print(json.dumps({"m": args.m, "n": n, "k": k, "tactic": fi.tactic_fields(t), "resolved": info,
+                              "us": round(us, 3), "gbs": round(b / (us * 1e-6) / 1e9, 1)}), flush=True)
+            del graph
+        del copies
 
 
 # -------------------------------------------------------------- oracle (CPU) timing
 
-def oracle_sample(target_s: float) -> dict:
-    """Time the CPU oracle's product (dequantise + fp64 dot) on the same five shapes."""
+def _oracle_packed():
     import oracle
     from bf16_activations_nvfp4_b200 import inputs
-
     packed = []
     for n, k in SHAPES:
         Wq, Ws, g = oracle.pack(inputs.weights(n, k, seed=0))
         packed.append((inputs.activations(M, k, seed=0), Wq, Ws, g, algorithmic_bytes(M, n, k)))
+    return packed
+
+
+def oracle_sample(target_s: float) -> dict:
+    """Time the CPU oracle's product (dequantise + fp64 dot) on the same five shapes."""
+    import oracle
+    packed = _oracle_packed()
     reps, elapsed, nbytes = 0, 0.0, 0
     while elapsed < target_s and reps < 200:
         for A, Wq, Ws, g, b in packed:
@@ -320,17 +387,12 @@ def oracle_sample(target_s: float) -> dict:
         reps += 1
     return {"value": round(nbytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
             "kind": "oracle", "reps": reps, "seconds": round(elapsed, 2),
-            "sample": f"{reps} full passes over the five m=1 shapes (pack excluded)"}
+            "sample": f"{reps} full passes over the five m=1 products (pack excluded)"}
 
 
 def run_reference(args) -> dict:
     import oracle
-    from bf16_activations_nvfp4_b200 import inputs
-
-    packed = []
-    for n, k in SHAPES:
-        Wq, Ws, g = oracle.pack(inputs.weights(n, k, seed=0))
-        packed.append((inputs.activations(M, k, seed=0), Wq, Ws, g, algorithmic_bytes(M, n, k)))
+    packed = _oracle_packed()
     # each step is one of the five products, in rotation, so K steps stay within minutes
     for st in range(args.warmup):
         A, Wq, Ws, g, _ = packed[st % len(packed)]
@@ -359,21 +421,23 @@ def run_reference(args) -> dict:
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["fi", "reference"], default="fi")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     ap.add_argument("--shapes", default=None,
                     help="comma-separated n x k subset of the workload, e.g. 4096x14336 (profiling runs)")
     ap.add_argument("--splits", default=None, help="comma-separated subset of the split menu (0 = device-sized)")
+    ap.add_argument("--sweep", action="store_true", help="print per-call µs of every listed tactic and exit")
+    ap.add_argument("--m", type=int, default=1, help="activation rows for --sweep")
     args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
     global SHAPES, SPLITS
     if args.shapes:
         SHAPES = [tuple(int(v) for v in sh.split("x")) for sh in args.shapes.split(",")]
     if args.splits:
         SPLITS = [int(v) for v in args.splits.split(",")]
-    if args.warmup < 3:
-        ap.error("--warmup must be at least 3")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -381,6 +445,9 @@ def main(argv=None) -> int:
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if args.sweep:
+        sweep(args)
         return 0
 
     if world > 1:

@@ -330,6 +330,7 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.ctas_per_sm = info.ctas_per_sm;
     a.num_sms = sms;
     a.smem_bytes = info.smem_bytes;
+    a.pdl = 1;
     rc = launch_gemv(a, stream);
     if (rc != FI_OK) return rc;
   } else {

@@ -37,10 +37,15 @@ namespace fi {
 
 namespace {
 
-// Stage A[0:m, kbase : kbase + klen] as f16 (scaled per 16-block) plus fp32 block scales.
+// Shared-memory image of the activations for one K split, laid out for conflict-free reads:
+// chunk c (32 k) of row r lives in 4 16-byte quads at uint4 index
+//     ((r * G + c / 32) * 4 + q) * 32 + c % 32,        G = ceil(nch / 32)
+// so the 32 lanes of a warp, reading chunks 32t .. 32t+31, touch 512 contiguous bytes per
+// quad. Values are f16 with one power-of-two scale per 16-block (fp32, linear As[r][2c+h]).
 __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A, int64_t k, int m,
-                                                  int64_t kbase, int klen, uint32_t* Ah, float* As) {
-  const int blocks_per_row = klen / 16;
+                                                  int64_t kbase, int nch, uint4* Ah4, float* As) {
+  const int G = (nch + 31) / 32;
+  const int blocks_per_row = nch * 2;
   const int nblk = m * blocks_per_row;
   for (int bi = threadIdx.x; bi < nblk; bi += blockDim.x) {
     const int r = bi / blocks_per_row;
@@ -67,9 +72,10 @@ __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A
       const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * up;
       h[i] = f32x2_to_f16x2(lo, hi);
     }
-    uint4* dst = reinterpret_cast<uint4*>(Ah + (int64_t)r * (klen / 2) + b * 8);
+    const int c = b >> 1, half = b & 1;
+    uint4* dst = Ah4 + ((int64_t)(r * G + c / 32) * 4 + 2 * half) * 32 + (c % 32);
     dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
-    dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+    dst[32] = make_uint4(h[4], h[5], h[6], h[7]);
     As[r * blocks_per_row + b] = down;
   }
 }
@@ -97,10 +103,18 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
 
 }  // namespace
 
+// Occupancy target per instance (register budget per thread = 65536 / (256 * CTAs)): the
+// small-m streaming instances keep three CTAs (24 warps) per SM resident.
+template <int MT, int R>
+constexpr int gemv_min_ctas() {
+  return (MT * R <= 2) ? 3 : (MT * R <= 8 && MT <= 4) ? 2 : 1;
+}
+
 template <int MT, int R, int D>
-__global__ void __launch_bounds__(kGemvThreads) gemv_nvfp4_kernel(GemvArgs p) {
+__global__ void __launch_bounds__(kGemvThreads, gemv_min_ctas<MT, R>()) gemv_nvfp4_kernel(GemvArgs p) {
   extern __shared__ __align__(16) uint8_t smem[];
-  // let a PDL-launched split-K reduce get scheduled; it waits for this grid to finish
+  // a PDL-launched successor (the split-K reduce, or the next op) may be scheduled now; it
+  // waits for this grid's completion before touching what this grid writes
   pdl_launch_dependents();
 
   const int lane = threadIdx.x & 31;
@@ -118,12 +132,13 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nvfp4_kernel(GemvArgs p) {
   const int64_t C = k / kChunkK;
   const int64_t c0 = (int64_t)s * C / S;
   const int nch = (int)((int64_t)(s + 1) * C / S - c0);
-  const int klen = nch * kChunkK;
+  const int G = (nch + 31) / 32;
   const int w0 = kw * nch / KW;
   const int wch = (kw + 1) * nch / KW - w0;
   // at least one (possibly empty) step per row group, so every warp of a slot meets the
   // slot's barrier once per row group even when its share of k is empty
   const int T = wch > 0 ? (wch + 31) / 32 : 1;
+  const int climit = wch - lane;  // step t is live for this lane iff 32 * t < climit
 
   // row groups of this CTA, and of this warp's slot
   const int64_t RG = (n + R - 1) / R;
@@ -132,39 +147,61 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nvfp4_kernel(GemvArgs p) {
   const int nrg = (rg_lo + slot < rg_hi) ? (int)((rg_hi - rg_lo - slot + NS - 1) / NS) : 0;
   const int F = nrg * T;
 
-  uint32_t* Ah = reinterpret_cast<uint32_t*>(smem);
-  float* As = reinterpret_cast<float*>(smem + (int64_t)m * klen * 2);
-  float* comb = As + m * (klen / 16);  // [2][NS][KW][R*MT], used when KW > 1
+  uint4* Ah4 = reinterpret_cast<uint4*>(smem);
+  float* As = reinterpret_cast<float*>(smem + (int64_t)m * G * 32 * 64);
+  float* comb = As + m * nch * 2;  // [2][NS][KW][R*MT], used when KW > 1
 
-  const uint8_t* wq_base = p.Wq + (c0 + w0) * 16;
-  const uint8_t* ws_base = p.Ws + (c0 + w0) * 2;
-  const int64_t wq_row = k / 2, ws_row = k / 16;
-
-  auto load_step = [&](Step<R>& st, int li, int lt) {
-    const int c = lt * 32 + lane;
-    const bool ok = li < nrg && c < wch;
-    const int64_t j0 = (rg_lo + slot + (int64_t)li * NS) * R;
+  // load cursor: one pointer per row, advanced 32 chunks per step and jumped to the next
+  // row group of this slot (NS * R rows further) after T steps
+  const int64_t rs_q = k / 2, rs_s = k / 16;
+  const uint8_t* lq[R];
+  const uint8_t* ls[R];
+  {
+    const int64_t j0 = (rg_lo + slot) * R;
 #pragma unroll
     for (int i = 0; i < R; ++i) {
-      if (ok && j0 + i < n) {
-        st.q[i] = ldg_stream_v4(wq_base + (j0 + i) * wq_row + (int64_t)c * 16);
-        st.sc[i] = ldg_stream_u16(ws_base + (j0 + i) * ws_row + (int64_t)c * 2);
+      lq[i] = p.Wq + (j0 + i) * rs_q + (c0 + w0 + lane) * 16;
+      ls[i] = p.Ws + (j0 + i) * rs_s + (c0 + w0 + lane) * 2;
+    }
+  }
+  const int64_t jump_q = (int64_t)NS * R * rs_q - (int64_t)T * 32 * 16;
+  const int64_t jump_s = (int64_t)NS * R * rs_s - (int64_t)T * 32 * 2;
+  // rows of the row group being fetched that exist (0 once past this warp's row groups)
+  int64_t l_left = nrg > 0 ? n - (rg_lo + slot) * R : 0;
+  int l_t = 0, l_g = 0;
+  auto issue = [&](Step<R>& st) {
+    const bool live = 32 * l_t < climit && l_g < nrg;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      if (live && i < l_left) {
+        st.q[i] = ldg_stream_v4(lq[i]);
+        st.sc[i] = ldg_stream_u16(ls[i]);
       } else {
         st.q[i] = make_uint4(0, 0, 0, 0);
         st.sc[i] = 0;
       }
+      lq[i] += 32 * 16;
+      ls[i] += 32 * 2;
+    }
+    if (++l_t == T) {
+      l_t = 0;
+      ++l_g;
+      l_left -= (int64_t)NS * R;
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        lq[i] += jump_q;
+        ls[i] += jump_s;
+      }
     }
   };
 
-  // prologue: put the first D steps of the weight stream in flight, then stage A
+  // prologue: put the first D steps of the weight stream in flight (weights are never written
+  // by the preceding kernel), then wait for the producer of A and stage it
   Step<R> ring[D];
-  int li = 0, lt = 0;
 #pragma unroll
-  for (int d = 0; d < D; ++d) {
-    load_step(ring[d], li, lt);
-    if (++lt == T) { lt = 0; ++li; }
-  }
-  stage_activations(p.A, k, m, c0 * kChunkK, klen, Ah, As);
+  for (int d = 0; d < D; ++d) issue(ring[d]);
+  pdl_wait();
+  stage_activations(p.A, k, m, c0 * kChunkK, nch, Ah4, As);
   __syncthreads();
 
   const float g = (S == 1) ? *p.gscale : 1.0f;
@@ -174,14 +211,49 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nvfp4_kernel(GemvArgs p) {
 #pragma unroll
     for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
 
-  int ci = 0, ct = 0;
+  // compute cursor: this lane's activation quads and block scales for step t
+  const int ca0 = w0 + lane;
+  const uint4* a_base = Ah4 + (int64_t)(ca0 / 32) * 4 * 32 + (ca0 % 32);
+  const float2* s_base = reinterpret_cast<const float2*>(As) + ca0;
+  int ct = 0, cg = 0;
   for (int f0 = 0; f0 < F; f0 += D) {
 #pragma unroll
     for (int d = 0; d < D; ++d) {
       if (f0 + d < F) {
         Step<R>& cur = ring[d];
-        const int c = ct * 32 + lane;
-        if (c < wch) {
+        if (MT == 1 && 32 * ct < climit) {
+          // one activation row: decode each weight word straight into the FMAs (same
+          // element order as below, fewer live registers)
+          const uint4* ap = a_base + (int64_t)ct * 4 * 32;
+          const uint4 a0 = ap[0], a1 = ap[32], a2 = ap[64], a3 = ap[96];
+          const uint32_t a[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                                  a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+          const float2 sa = s_base[ct * 32];
+#pragma unroll
+          for (int i = 0; i < R; ++i) {
+            const uint32_t words[4] = {cur.q[i].x, cur.q[i].y, cur.q[i].z, cur.q[i].w};
+            float pb[2] = {0.0f, 0.0f};
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+              const uint32_t h0 = e2m1x2_byte_to_f16x2<0>(words[wd]);
+              const uint32_t h1 = e2m1x2_byte_to_f16x2<1>(words[wd]);
+              const uint32_t h2 = e2m1x2_byte_to_f16x2<2>(words[wd]);
+              const uint32_t h3 = e2m1x2_byte_to_f16x2<3>(words[wd]);
+              float& pp = pb[wd >> 1];
+              pp = fma_lo_f16(a[wd * 4 + 0], h0, pp);
+              pp = fma_hi_f16(a[wd * 4 + 0], h0, pp);
+              pp = fma_lo_f16(a[wd * 4 + 1], h1, pp);
+              pp = fma_hi_f16(a[wd * 4 + 1], h1, pp);
+              pp = fma_lo_f16(a[wd * 4 + 2], h2, pp);
+              pp = fma_hi_f16(a[wd * 4 + 2], h2, pp);
+              pp = fma_lo_f16(a[wd * 4 + 3], h3, pp);
+              pp = fma_hi_f16(a[wd * 4 + 3], h3, pp);
+            }
+            const uint32_t sh = e4m3x2_to_f16x2(cur.sc[i]);
+            acc[i][0] = fmaf(pb[0], f16_lo_to_f32(sh) * sa.x, acc[i][0]);
+            acc[i][0] = fmaf(pb[1], f16_hi_to_f32(sh) * sa.y, acc[i][0]);
+          }
+        } else if (MT > 1 && 32 * ct < climit) {
           uint32_t wf[R][16];
           float sw[R][2];
 #pragma unroll
@@ -198,15 +270,14 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nvfp4_kernel(GemvArgs p) {
             sw[i][0] = f16_lo_to_f32(sh);
             sw[i][1] = f16_hi_to_f32(sh);
           }
-          const int ca = w0 + c;  // chunk index inside the staged split
 #pragma unroll
           for (int r = 0; r < MT; ++r) {
             if (r < m) {
-              const uint4* ap = reinterpret_cast<const uint4*>(Ah + (int64_t)r * (klen / 2) + ca * 16);
-              const uint4 a0 = ap[0], a1 = ap[1], a2 = ap[2], a3 = ap[3];
+              const uint4* ap = a_base + ((int64_t)r * G + ct) * 4 * 32;
+              const uint4 a0 = ap[0], a1 = ap[32], a2 = ap[64], a3 = ap[96];
               const uint32_t a[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
                                       a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-              const float2 sa = *reinterpret_cast<const float2*>(As + r * (klen / 16) + ca * 2);
+              const float2 sa = s_base[r * nch + ct * 32];
 #pragma unroll
               for (int i = 0; i < R; ++i) {
                 const float p0 = dot16(a, wf[i]);
@@ -218,13 +289,12 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nvfp4_kernel(GemvArgs p) {
           }
         }
         // refill this ring slot with the step D ahead (predicated off past the end)
-        load_step(cur, li, lt);
-        if (++lt == T) { lt = 0; ++li; }
+        issue(cur);
 
         if (ct == T - 1) {
-          // row group ci is complete: reduce over lanes, then over the slot's KW warps
-          const int64_t j0 = (rg_lo + slot + (int64_t)ci * NS) * R;
-          const int par = ci & 1;
+          // row group cg is complete: reduce over lanes, then over the slot's KW warps
+          const int64_t j0 = (rg_lo + slot + (int64_t)cg * NS) * R;
+          const int par = cg & 1;
 #pragma unroll
           for (int i = 0; i < R; ++i) {
 #pragma unroll
@@ -275,7 +345,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_nvfp4_kernel(GemvArgs p) {
 #pragma unroll
             for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
         }
-        if (++ct == T) { ct = 0; ++ci; }
+        if (++ct == T) {
+          ct = 0;
+          ++cg;
+        }
       }
     }
   }
@@ -312,9 +385,17 @@ int launch_one(const GemvArgs& a, cudaStream_t stream) {
   int64_t gx = (int64_t)a.num_sms * ctas / a.splits;
   if (gx < 1) gx = 1;
   if (gx > a.grid_x) gx = a.grid_x;
-  dim3 grid((unsigned)gx, (unsigned)a.splits);
-  kern<<<grid, kGemvThreads, a.smem_bytes, stream>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return set_cuda_error("gemv kernel launch");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)gx, (unsigned)a.splits);
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = (size_t)a.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return set_cuda_error("gemv kernel launch");
   return FI_OK;
 }
 
@@ -324,7 +405,9 @@ int launch_rows(const GemvArgs& a, cudaStream_t stream) {
   switch (a.rows_per_warp) {
     case 1: return launch_one<MT, 1, D1>(a, stream);
     case 2: return launch_one<MT, 2, 2>(a, stream);
-    case 4: return launch_one<MT, 4, 2>(a, stream);
+    case 4:
+      if constexpr (MT <= 16) return launch_one<MT, 4, 2>(a, stream);
+      return set_error(FI_ERR_INVALID_ARG, "GEMV with 4 rows per warp supports m <= 16");
     default: return set_error(FI_ERR_INVALID_ARG, "GEMV rows per warp must be 1, 2 or 4");
   }
 }

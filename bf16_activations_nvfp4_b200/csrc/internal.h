@@ -35,11 +35,12 @@ inline int gemv_mt(int64_t m) {
   return mt;
 }
 
-// Shared memory the GEMV needs: m activation rows over klen k (f16 values plus one fp32
-// power-of-two scale per 16-block) and the in-CTA split-K combine buffer
-// (2 parities x 8 warps x R rows x MT activation rows, fp32).
+// Shared memory the GEMV needs: m activation rows over klen k as f16, padded to whole warp
+// steps of 1024 k, plus one fp32 power-of-two scale per 16-block, plus the in-CTA split-K
+// combine buffer (2 parities x 8 warps x R rows x MT activation rows, fp32).
 inline int64_t gemv_smem_bytes(int64_t m, int64_t klen, int R) {
-  return m * klen * 2 + m * (klen / 16) * 4 + 2 * 8 * (int64_t)R * gemv_mt(m) * 4;
+  const int64_t padded = (klen + 1023) / 1024 * 1024;
+  return m * padded * 2 + m * (klen / 16) * 4 + 2 * 8 * (int64_t)R * gemv_mt(m) * 4;
 }
 
 struct GemvArgs {
@@ -57,6 +58,7 @@ struct GemvArgs {
   int ctas_per_sm;
   int num_sms;
   int smem_bytes;
+  int pdl;            // launch with programmatic stream serialization
 };
 int launch_gemv(const GemvArgs& a, cudaStream_t stream);
 

@@ -20,6 +20,7 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
                                                              const float* __restrict__ gscale,
                                                              uint16_t* __restrict__ out,
                                                              bool vec4) {
+  pdl_launch_dependents();
   pdl_wait();
   const float g = *gscale;
   const int64_t e0 = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 4;

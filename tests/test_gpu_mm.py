@@ -113,14 +113,24 @@ def test_batch_invariance_rows_do_not_depend_on_m(splits):
     n, k = 4096, 14336
     A32 = inputs.activations(32, k, seed=0, outliers=True)
     dw = _gpu.device_weights(n, k, 0)
-    ms = [1, 2, 4, 8, 16, 32] if splits else [1, 2, 4, 8]
-    for R in (1, 2, 4):
+    ms = [1, 2, 4, 8, 16, 32]
+    for R in (1, 2):
         t = fi.make_tactic(GEMV, splits, 0, R)
         base = _mm(A32[:ms[-1]], dw, t)
         for m in ms:
             for _ in range(10 if m in (1, ms[-1]) else 2):
                 got = _mm(A32[:m], dw, t)
                 assert np.array_equal(got, base[:m]), (R, splits, m)
+
+
+def test_batch_invariance_four_rows_per_warp_up_to_m16():
+    n, k = 4096, 14336
+    A16 = inputs.activations(16, k, seed=1, outliers=True)
+    dw = _gpu.device_weights(n, k, 0)
+    t = fi.make_tactic(GEMV, 8, 0, 4)
+    base = _mm(A16, dw, t)
+    for m in (1, 3, 8, 16):
+        assert np.array_equal(_mm(A16[:m], dw, t), base[:m]), m
 
 
 def test_rows_per_warp_and_occupancy_do_not_change_bits():
