@@ -21,7 +21,7 @@ __all__ = [
     "FiError", "KIND_GEMV", "KIND_MMA", "TACTIC_DEFAULT", "make_tactic", "tactic_fields",
     "pack_weights", "mm_bf16_fp4", "splitk_reduce", "resolve_tactic", "default_tactic",
     "list_tactics", "workspace_bytes", "set_workspace", "last_error", "version", "library",
-    "library_path",
+    "library_path", "get_device_error", "debug_set", "DEBUG_STALL_PRODUCER", "DEBUG_WAIT_TIMEOUT_NS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -89,8 +89,11 @@ def library() -> ctypes.CDLL:
         lib.fi_last_error.argtypes = []
         lib.fi_last_error.restype = ctypes.c_char_p
         lib.fi_version.argtypes = []
+        lib.fi_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        lib.fi_debug_set.argtypes = [ctypes.c_int, i64]
         for name in ("fi_nvfp4_pack_weights", "fi_mm_bf16_fp4", "fi_mm_bf16_fp4_ex", "fi_splitk_reduce",
-                     "fi_resolve_tactic", "fi_list_tactics", "fi_set_workspace", "fi_version"):
+                     "fi_resolve_tactic", "fi_list_tactics", "fi_set_workspace", "fi_version",
+                     "fi_get_device_error", "fi_debug_set"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -107,6 +110,22 @@ def version() -> int:
 def _check(status: int, where: str) -> None:
     if status != 0:
         raise FiError(status, where, last_error())
+
+
+DEBUG_STALL_PRODUCER = 1
+DEBUG_WAIT_TIMEOUT_NS = 2
+
+
+def get_device_error() -> int:
+    """Read and clear the current device's sticky kernel error word (0 = no error)."""
+    code = ctypes.c_uint(0)
+    _check(library().fi_get_device_error(ctypes.byref(code)), "fi_get_device_error")
+    return int(code.value)
+
+
+def debug_set(key: int, value: int) -> None:
+    """Test hooks of fi_debug_set (stall the producer of the next launches, wait limit)."""
+    _check(library().fi_debug_set(int(key), int(value)), "fi_debug_set")
 
 
 # ------------------------------------------------------------------------- tactics

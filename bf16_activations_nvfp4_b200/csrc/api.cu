@@ -2,6 +2,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "fi_nvfp4.h"
@@ -83,42 +85,83 @@ static int check_arch() {
 
 // ----------------------------------------------------------------- tactics
 
-// Device-sized parallelism: enough weight-streaming warps on every SM to keep HBM busy
-// (PR #4038 measured saturation at ~20 warps/SM on SM12x and sized split-K from the device).
-constexpr int kKneeWarpsPerSm = 20;
-// A warp keeps at least this many 32-k chunks of a row (one full warp step) so that its
-// lanes have work when the k range is divided among warps or splits.
-constexpr int64_t kMinChunksPerWarp = 32;
-// Shared memory per CTA the device-sized split aims for (three CTAs per SM fit).
-constexpr int64_t kKneeSmemPerCta = 72 * 1024;
 // Largest m the default table sends to the GEMV.
 constexpr int64_t kDefaultGemvMaxM = 32;
+// Rows per consumer warp when the tactic leaves it open.
+constexpr int kGemvDefaultRows = 2;
 
-static int gemv_default_rows(int64_t n) { return n >= 4096 ? 2 : 1; }
-
-// Smallest power of two KW <= maxKW (and <= 8) with RG * KW * S >= target.
-static int64_t auto_kw(int64_t RG, int64_t S, int64_t C, int64_t target) {
-  int64_t KW = 1;
-  while (KW < 8 && RG * KW * S < target && (C / S) / (KW * 2) >= kMinChunksPerWarp) KW *= 2;
-  return KW;
+int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int R, int ctas_per_sm, int sms, GemvGeometry* g) {
+  const int64_t C = k / kChunkK;
+  const int64_t nch = (C + S - 1) / S;  // chunks of the largest split
+  // KW: the largest power of two <= min(8, warp steps of a split)
+  const int64_t steps = (nch + 31) / 32;
+  int KW = 1;
+  while (KW * 2 <= kGemvConsumerWarps && KW * 2 <= steps) KW *= 2;
+  const int TR = (kGemvConsumerWarps / KW) * R;
+  const int ctas = ctas_per_sm > 0 ? ctas_per_sm : 1;
+  const int64_t per_cta = std::min<int64_t>(kSmemBudget, (228 * 1024) / ctas - 2048);
+  const int64_t a_bytes = round_up(m * ((nch + 31) / 32) * 2048, 128);
+  const int64_t as_bytes = round_up(m * nch * 8, 128);
+  const int64_t comb_bytes = round_up(2 * kGemvConsumerWarps * (int64_t)R * gemv_mt(m) * 4, 128);
+  const int64_t bar_bytes = round_up(2 * kGemvMaxStages * 8, 128);
+  const int64_t fixed = a_bytes + as_bytes + comb_bytes + bar_bytes;
+  const int64_t avail = per_cta - fixed;
+  auto stage_of = [&](int64_t sl) { return round_up(TR * (sl * 16 + gemv_scales_stride(sl)), 128); };
+  int64_t target = std::min<int64_t>(kGemvStageTarget, avail / 4);
+  int64_t slab;
+  if (stage_of(nch) <= target) {
+    slab = nch;
+  } else {
+    const int64_t unit = 32 * KW;
+    slab = unit;
+    while (slab + unit < nch && stage_of(slab + unit) <= target) slab += unit;
+  }
+  const int64_t stage_bytes = stage_of(slab);
+  const int64_t stages = std::min<int64_t>(kGemvMaxStages, avail > 0 ? avail / stage_bytes : 0);
+  if (stages < 2)
+    return set_error(FI_ERR_UNSUPPORTED_SHAPE,
+                     "GEMV: m=%lld over %lld k per split leaves no room for the weight ring in shared "
+                     "memory; use more splits",
+                     (long long)m, (long long)(nch * kChunkK));
+  const int64_t tiles = (n + TR - 1) / TR;
+  int64_t gx = std::max<int64_t>(1, (int64_t)sms * ctas / S);
+  if (gx > tiles) gx = tiles;
+  g->S = S;
+  g->R = R;
+  g->KW = KW;
+  g->TR = TR;
+  g->slab = (int)slab;
+  g->stages = (int)stages;
+  g->ctas_per_sm = ctas;
+  g->grid_x = (int)std::max<int64_t>(1, gx);
+  g->stage_bytes = stage_bytes;
+  g->off_as = a_bytes;
+  g->off_comb = a_bytes + as_bytes;
+  g->off_bar = a_bytes + as_bytes + comb_bytes;
+  g->off_ring = fixed;
+  g->smem_bytes = fixed + stages * stage_bytes;
+  return FI_OK;
 }
 
-// Device-sized split for rows-per-warp R: the in-CTA split KW first (no second kernel), then
-// the fewest global splits S that reach the target warp count, raised until `m_fit`
-// activation rows of a split fit the shared-memory staging. Depends on (n, k, SMs, m_fit).
-static void gemv_knee(int64_t n, int64_t k, int sms, int64_t m_fit, int R, int64_t KW_req, int64_t* S_out,
-                      int64_t* KW_out) {
+// Device-sized split (PR #4038, "Sizes GEMV split-K from the device"): the fewest splits S
+// that give every SM a CTA with rows to stream while `m_fit` activation rows of a split fit
+// the shared-memory staging. Depends on (n, k, SMs, R, m_fit) only.
+static int gemv_knee(int64_t n, int64_t k, int sms, int64_t m_fit, int R, int ctas, int* S_out) {
   const int64_t C = k / kChunkK;
-  const int64_t RG = (n + R - 1) / R;
-  const int64_t target = (int64_t)kKneeWarpsPerSm * sms;
-  const int64_t KW = KW_req ? KW_req : auto_kw(RG, 1, C, target);
-  const int64_t want = (target + RG * KW - 1) / (RG * KW > 0 ? RG * KW : 1);
-  int64_t cap = C / (kMinChunksPerWarp * KW);
-  if (cap < 1) cap = 1;
-  int64_t S = want < 1 ? 1 : (want > cap ? cap : want);
-  while (S < C && gemv_smem_bytes(m_fit, ((C + S - 1) / S) * kChunkK, R) > kKneeSmemPerCta) ++S;
-  *S_out = S;
-  *KW_out = KW;
+  const int64_t maxS = std::max<int64_t>(1, std::min<int64_t>(C, 4095));
+  for (int64_t S = 1; S <= maxS; ++S) {
+    GemvGeometry g;
+    if (gemv_geometry(m_fit, n, k, (int)S, R, ctas, sms, &g) != FI_OK) continue;
+    const int64_t tiles = (n + g.TR - 1) / g.TR;
+    const bool enough = tiles * S >= (int64_t)sms * g.ctas_per_sm;
+    const bool last = S == maxS || (C / (S + 1)) < 32;  // a split keeps at least one warp step
+    if (enough || last) {
+      *S_out = (int)S;
+      clear_error();
+      return FI_OK;
+    }
+  }
+  return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV: no split count fits m=%lld in shared memory", (long long)m_fit);
 }
 
 static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms, fi_tactic_info* out);
@@ -128,73 +171,56 @@ static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms,
 static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms) {
   if (m <= kDefaultGemvMaxM) {
     const int64_t m_fit = m <= 1 ? 1 : (m <= 8 ? 8 : kGemvMaxM);
-    const int R = (m_fit > 16 && gemv_default_rows(n) > 2) ? 2 : gemv_default_rows(n);
-    int64_t S = 1, KW = 1;
-    gemv_knee(n, k, num_sms, m_fit, R, 0, &S, &KW);
-    return FI_TACTIC(FI_KIND_GEMV, S, 0, R | (KW << 4));
+    int S = 1;
+    if (gemv_knee(n, k, num_sms, m_fit, kGemvDefaultRows, 1, &S) != FI_OK) S = 1;
+    return FI_TACTIC(FI_KIND_GEMV, S, 0, kGemvDefaultRows);
   }
   return FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
 }
 
-// GEMV variant byte: low nibble R (weight rows per warp), high nibble KW (warps per row
-// group inside a CTA); 0 in either means automatic. Splits 0 = device-sized, resolved for
-// m <= 32 so that the resolved S (and the bits) never depend on m.
+// GEMV variant byte: R, the weight rows per consumer warp (1, 2 or 4; 0 = automatic).
+// Splits 0 = device-sized, resolved for m <= 32 so that the resolved S (and the bits) never
+// depend on m.
 static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var,
                         int sms, fi_tactic_info* out) {
   if (m > kGemvMaxM)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV tactics support m <= %d (got m=%lld)",
                      kGemvMaxM, (long long)m);
-  const int R = (var & 0xF) ? (var & 0xF) : gemv_default_rows(n);
+  const int R = var ? var : kGemvDefaultRows;
   if (R != 1 && R != 2 && R != 4)
     return set_error(FI_ERR_INVALID_ARG, "GEMV rows per warp must be 0 (auto), 1, 2 or 4");
   if (R == 4 && m > 16)
     return set_error(FI_ERR_INVALID_ARG, "GEMV with 4 rows per warp supports m <= 16");
-  const int KW_req = var >> 4;
-  if (KW_req != 0 && KW_req != 1 && KW_req != 2 && KW_req != 4 && KW_req != 8)
-    return set_error(FI_ERR_INVALID_ARG, "GEMV warps per row group must be 0 (auto), 1, 2, 4 or 8");
   const int64_t C = k / kChunkK;
-  const int64_t RG = (n + R - 1) / R;
-  int64_t KW = KW_req;
-  int64_t S = S_req;
+  const int ctas = ctas_req ? ctas_req : 1;
+  int S = S_req;
   if (S == 0) {
-    gemv_knee(n, k, sms, kGemvMaxM, R, KW_req, &S, &KW);
+    const int rc = gemv_knee(n, k, sms, kGemvMaxM, R, ctas, &S);
+    if (rc != FI_OK) return rc;
+  } else if (C > 0 && S > C) {
+    return set_error(FI_ERR_INVALID_ARG, "splits=%lld exceeds k/32=%lld", (long long)S, (long long)C);
+  }
+  GemvGeometry g;
+  if (C == 0) {  // k == 0: nothing to stream; the caller writes zeros
+    memset(&g, 0, sizeof(g));
+    g.S = 1;
+    g.R = R;
+    g.KW = 1;
+    g.ctas_per_sm = ctas;
+    g.grid_x = 1;
   } else {
-    if (C > 0 && S > C)
-      return set_error(FI_ERR_INVALID_ARG, "splits=%lld exceeds k/32=%lld", (long long)S, (long long)C);
-    if (KW == 0) KW = auto_kw(RG, S, C, (int64_t)kKneeWarpsPerSm * sms);
+    const int rc = gemv_geometry(m, n, k, S, R, ctas, sms, &g);
+    if (rc != FI_OK) return rc;
   }
-  if (S < 1) S = 1;
-  if (C > 0 && KW > C / S)
-    return set_error(FI_ERR_INVALID_ARG, "warps per row group (%lld) exceeds the %lld k-chunks of a split",
-                     (long long)KW, (long long)(C / S));
-  const int64_t klen_max = ((C + S - 1) / S) * kChunkK;
-  const int64_t smem = gemv_smem_bytes(m, klen_max, R);
-  if (smem > kSmemBudget)
-    return set_error(FI_ERR_UNSUPPORTED_SHAPE,
-                     "GEMV: m=%lld with k/splits=%lld needs %lld B of shared memory (> %d); use more splits",
-                     (long long)m, (long long)klen_max, (long long)smem, kSmemBudget);
-  int ctas = ctas_req;
-  if (ctas == 0) {
-    // leave room on every SM for the PDL-launched reduce when the tactic splits
-    ctas = S > 1 ? 3 : 4;
-    const int fit = (int)((227 * 1024) / (smem + 1024));
-    if (ctas > fit) ctas = fit;
-    if (ctas < 1) ctas = 1;
-  }
-  const int64_t NS = kGemvWarps / KW;
-  const int64_t cta_rows = (RG + NS - 1) / NS;
-  int64_t slots = ((int64_t)sms * ctas) / S;
-  if (slots < 1) slots = 1;
-  const int64_t grid_x = cta_rows < slots ? cta_rows : slots;
   out->kind = FI_KIND_GEMV;
-  out->splits = (int32_t)S;
-  out->ctas_per_sm = ctas;
-  out->variant = (int32_t)(R | (KW << 4));
-  out->grid_x = (int32_t)(grid_x > 0 ? grid_x : 1);
-  out->grid_y = (int32_t)S;
+  out->splits = g.S;
+  out->ctas_per_sm = g.ctas_per_sm;
+  out->variant = R;
+  out->grid_x = g.grid_x;
+  out->grid_y = g.S;
   out->threads = kGemvThreads;
-  out->smem_bytes = (int32_t)smem;
-  out->workspace_bytes = S > 1 ? S * m * n * (int64_t)sizeof(float) : 0;
+  out->smem_bytes = (int32_t)g.smem_bytes;
+  out->workspace_bytes = g.S > 1 ? (int64_t)g.S * m * n * (int64_t)sizeof(float) : 0;
   return FI_OK;
 }
 
@@ -267,6 +293,15 @@ static int get_workspace(size_t need, cudaStream_t stream, void** ptr) {
   return FI_OK;
 }
 
+// ------------------------------------------------------------------ test hooks
+
+namespace {
+// launches whose producer warp is told to issue nothing (consumer waits then time out)
+std::atomic<int> g_debug_stall_launches{0};
+// limit of every mbarrier wait inside the kernels
+std::atomic<uint64_t> g_wait_timeout_ns{1000000000ull};
+}  // namespace
+
 // ------------------------------------------------------------------ checks
 
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -287,9 +322,10 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     return FI_OK;
   }
   if (!A || !Wq || !Wscale || !gscale || !out) return set_error(FI_ERR_INVALID_ARG, "null pointer argument");
-  if (!aligned(A, 16) || !aligned(Wq, 16)) return set_error(FI_ERR_INVALID_ARG, "A and Wq must be 16-byte aligned");
-  if (!aligned(Wscale, 2) || !aligned(out, 2) || !aligned(gscale, 4))
-    return set_error(FI_ERR_INVALID_ARG, "Wscale/out must be 2-byte and gscale 4-byte aligned");
+  if (!aligned(A, 16) || !aligned(Wq, 16) || !aligned(Wscale, 16))
+    return set_error(FI_ERR_INVALID_ARG, "A, Wq and Wscale must be 16-byte aligned");
+  if (!aligned(out, 2) || !aligned(gscale, 4))
+    return set_error(FI_ERR_INVALID_ARG, "out must be 2-byte and gscale 4-byte aligned");
   int rc = check_arch();
   if (rc != FI_OK) return rc;
   const int sms = device_sm_count();
@@ -313,7 +349,11 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     }
   }
   if (info.kind == FI_KIND_GEMV) {
+    GemvGeometry g;
+    rc = gemv_geometry(m, n, k, info.splits, info.variant, info.ctas_per_sm, sms, &g);
+    if (rc != FI_OK) return rc;
     GemvArgs a;
+    memset(&a, 0, sizeof(a));
     a.A = A;
     a.Wq = Wq;
     a.Ws = Wscale;
@@ -323,14 +363,22 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.m = m;
     a.n = n;
     a.k = k;
-    a.splits = info.splits;
-    a.kw = info.variant >> 4;
-    a.rows_per_warp = info.variant & 0xF;
-    a.grid_x = info.grid_x;
-    a.ctas_per_sm = info.ctas_per_sm;
-    a.num_sms = sms;
-    a.smem_bytes = info.smem_bytes;
+    a.splits = g.S;
+    a.kw = g.KW;
+    a.rows_per_warp = g.R;
+    a.slab = g.slab;
+    a.stages = g.stages;
+    a.grid_x = g.grid_x;
     a.pdl = 1;
+    a.debug_stall = g_debug_stall_launches > 0 ? 1 : 0;
+    if (g_debug_stall_launches > 0) --g_debug_stall_launches;
+    a.stage_bytes = g.stage_bytes;
+    a.off_as = g.off_as;
+    a.off_comb = g.off_comb;
+    a.off_bar = g.off_bar;
+    a.off_ring = g.off_ring;
+    a.smem_bytes = g.smem_bytes;
+    a.timeout_ns = g_wait_timeout_ns;
     rc = launch_gemv(a, stream);
     if (rc != FI_OK) return rc;
   } else {
@@ -353,8 +401,8 @@ int fi_nvfp4_pack_weights(const float* W, int64_t n, int64_t k, uint8_t* Wq, uin
   if (k % 16 != 0) return set_error(FI_ERR_UNSUPPORTED_SHAPE, "k=%lld is not a multiple of 16", (long long)k);
   if (!gscale) return set_error(FI_ERR_INVALID_ARG, "gscale must not be null");
   if (n * k > 0 && (!W || !Wq || !Wscale)) return set_error(FI_ERR_INVALID_ARG, "null pointer argument");
-  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(Wscale, 8) || !aligned(gscale, 4))
-    return set_error(FI_ERR_INVALID_ARG, "W/Wq must be 16-byte, Wscale 8-byte, gscale 4-byte aligned");
+  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(Wscale, 16) || !aligned(gscale, 4))
+    return set_error(FI_ERR_INVALID_ARG, "W, Wq and Wscale must be 16-byte, gscale 4-byte aligned");
   const int rc = check_arch();
   if (rc != FI_OK) return rc;
   return launch_pack(W, n, k, Wq, Wscale, gscale, reinterpret_cast<cudaStream_t>(stream));
@@ -407,14 +455,13 @@ int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, 
   clear_error();
   const int sms = sms_or_device(num_sms);
   if (sms <= 0) return set_error(FI_ERR_CUDA, "no device to query the SM count from");
-  // the split menu {1, 2, 4, 8, device-sized} for each rows-per-warp choice, plus every
-  // in-CTA split for one row per warp; entries resolving to the same launch are listed once
+  // the split menu {1, 2, 4, 8, device-sized} for each rows-per-warp choice; entries
+  // resolving to the same launch are listed once
   int64_t cand[32];
   int nc = 0;
   const int splits[] = {1, 2, 4, 8, 0};
   for (int R : {1, 2, 4})
     for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, R);
-  for (int KW : {1, 2, 4, 8}) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, 1, 0, 1 | (KW << 4));
   fi_tactic_info seen[32];
   int nseen = 0, count = 0;
   for (int c = 0; c < nc; ++c) {
@@ -455,6 +502,31 @@ int fi_set_workspace(void* ptr, size_t bytes) {
   w.bytes = bytes;
   w.owned = false;
   return FI_OK;
+}
+
+int fi_get_device_error(unsigned* code) {
+  clear_error();
+  if (!code) return set_error(FI_ERR_INVALID_ARG, "code must not be null");
+  *code = 0;
+  const int rc = check_arch();
+  if (rc != FI_OK) return rc;
+  return gemv_read_error(code);
+}
+
+int fi_debug_set(int key, int64_t value) {
+  clear_error();
+  switch (key) {
+    case FI_DEBUG_STALL_PRODUCER:
+      if (value < 0) return set_error(FI_ERR_INVALID_ARG, "launch count must be >= 0");
+      g_debug_stall_launches = (int)value;
+      return FI_OK;
+    case FI_DEBUG_WAIT_TIMEOUT_NS:
+      if (value <= 0) return set_error(FI_ERR_INVALID_ARG, "timeout must be > 0 ns");
+      g_wait_timeout_ns = (uint64_t)value;
+      return FI_OK;
+    default:
+      return set_error(FI_ERR_INVALID_ARG, "unknown debug key %d", key);
+  }
 }
 
 const char* fi_last_error(void) { return g_err; }

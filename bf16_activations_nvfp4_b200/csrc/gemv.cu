@@ -1,33 +1,38 @@
 // Streaming GEMV for bf16 activations x NVFP4 weights, m <= 32 (sm_100a).
 //
-// After PR #4038's streaming GEMV ("weights stream from global memory to registers with
-// latency hidden by warp count", "one output row per warp, warp-shuffle reduction", and the
-// v2 commit's "A-in-SMEM staging" lever for m > 1), re-designed for B200:
+// After PR #4038's streaming GEMV ("weights stream from global memory ... latency hidden by
+// warp count", "one output row per warp, warp-shuffle reduction", the v2 commit's
+// "A-in-SMEM staging"), re-designed for B200, where an m=1 GEMV has to keep ~100 KB of
+// weights in flight per SM to run at HBM speed:
 //
-//  * Grid (G, S): blockIdx.y is the global K split s; the G CTAs of a split take balanced,
-//    contiguous ranges of weight row groups (R rows each) and persist over them.
-//  * Inside a CTA the 8 warps form 8/KW slots of KW warps. The KW warps of a slot share one
-//    row group and split its k range KW ways (in-CTA split-K); their partials are combined
-//    through shared memory in fixed order kw = 0..KW-1, so narrow-n shapes fill the GPU
-//    without a second kernel.
-//  * A warp streams R rows at once: lane L reads the 16 code bytes (32 k, two scale blocks) of
-//    chunk t*32+L with one coalesced 128-bit load per row plus the two E4M3 scale bytes. D steps
-//    are kept in flight in a register ring, across row-group boundaries, and the first D are
-//    issued before the activations are staged, so the weight stream starts at once.
-//  * The CTA stages A[0:m, split] in shared memory as f16 with one power-of-two scale per
-//    16-block (block floating point). A bf16 value has 8 significant bits, so the f16 copy is
-//    exact for every element within 2^28 of its block maximum; smaller ones are rounded at
-//    2^-39 of the block maximum.
-//  * Decode is the hardware cvt.rn.f16x2.e2m1x2 (two codes per instruction, exact) and the dot
-//    product the mixed-precision fma.rn.f32.f16 (f16 x f16 product, fp32 accumulate), one
-//    instruction per code; an 8-bit-significand activation times an E2M1 value is exact, so the
-//    only roundings are fp32 accumulation steps.
-//  * Per 16-block: p = sum_{i in block} a_i * e2m1_i (sequential, fp32), then
-//    acc = fma(p, sf_w * sf_a, acc). Lanes combine through a fixed xor butterfly (every lane
-//    ends with the same bits), then the KW warps in fixed order. The k order of every output is
-//    fixed by (k, S, KW) alone: bits do not depend on m, R, D, G or the CTAs per SM.
-//  * S == 1 writes bf16_rn(acc * gscale); S > 1 writes the fp32 partial for the fixed-order
-//    reduce kernel.
+//  * Warp specialisation. One producer warp per CTA streams weight tiles HBM -> shared memory
+//    with bulk asynchronous copies (cp.async.bulk, completion counted on an mbarrier) into an
+//    NST-stage ring; 8 consumer warps decode from shared memory. In-flight bytes live in
+//    shared memory, not registers, and cost the producer one instruction per copy.
+//  * Programmatic dependent launch. The producer issues the first NST stages before the
+//    grid-dependency wait (weights are never written by the preceding kernel); the consumers
+//    wait, then stage the activations, so the weight stream overlaps the previous kernel's
+//    tail and the activation staging.
+//  * Tiles. Grid (G, S): blockIdx.y is the K split s. The split's weight rows are cut into
+//    tiles of TR = NS * R rows; the G CTAs of a split own balanced contiguous tile ranges. A
+//    tile's rows are fetched in slabs of SL 32-k chunks (one ring stage per slab): one bulk
+//    copy per row for the codes and one per row for the E4M3 scales (a 16-byte-aligned
+//    superset of the scale bytes, indexed from the remainder; the bytes past the end of the
+//    scale tensor, where a superset would overrun it, are copied with plain loads).
+//  * Work split. The 8 consumer warps form NS = 8 / KW slots of KW warps, KW = the largest
+//    power of two <= min(8, ceil(chunks / 32)). Slot `slot` computes rows slot*R .. slot*R+R-1
+//    of the tile; inside a slot, lane L of warp kw takes chunks c = 32*KW*t + 32*kw + L.
+//  * Arithmetic (fixed by k and S alone, hence bitwise identical for every m, R, TR, SL,
+//    NST, G and CTAs per SM): A is staged as f16 with one power-of-two scale per 16-block
+//    (exact for every element within 2^28 of its block maximum); codes are decoded by
+//    cvt.rn.f16x2.e2m1x2 (exact) and multiplied by the mixed-precision fma.rn.f32.f16 (exact
+//    product, fp32 accumulate); per 16-block p = sum_i a_i * e2m1_i in element order, then
+//    acc = fma(p, sf_w * sf_a, acc) over the lane's chunks in order; lanes combine through a
+//    fixed xor butterfly (all lanes end with the same bits), the KW warps in order kw = 0..KW-1.
+//    S == 1 writes bf16_rn(acc * gscale); S > 1 writes fp32 partials for the reduce kernel.
+//  * Bounded waits. Every mbarrier wait gives up after a time limit (%globaltimer): it sets a
+//    device error flag and a CTA-wide abort flag, the CTA finishes its control flow without
+//    computing, and the producer waits (bounded) for the copies it issued before exiting.
 #include <cstdint>
 
 #include "common.cuh"
@@ -35,19 +40,90 @@
 
 namespace fi {
 
+// Sticky device error word: bit 0 = a consumer wait timed out, bit 1 = a producer wait timed
+// out, bit 2 = the producer's final drain timed out. Read and cleared by gemv_read_error().
+__device__ unsigned int g_gemv_error = 0;
+
 namespace {
 
-// Shared-memory image of the activations for one K split, laid out for conflict-free reads:
-// chunk c (32 k) of row r lives in 4 16-byte quads at uint4 index
-//     ((r * G + c / 32) * 4 + q) * 32 + c % 32,        G = ceil(nch / 32)
-// so the 32 lanes of a warp, reading chunks 32t .. 32t+31, touch 512 contiguous bytes per
-// quad. Values are f16 with one power-of-two scale per 16-block (fp32, linear As[r][2c+h]).
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete. Returns false (and raises the abort flag and
+// the device error bit) if it has not after timeout_ns, or at once if the CTA has aborted.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  uint64_t timeout_ns, unsigned err_bit) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if ((it & 63) == 63) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > timeout_ns) {
+        *abort_flag = 1;
+        atomicOr(&g_gemv_error, err_bit);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Stage A[0:m, kbase : kbase + 32*nch] for the consumer warps. Layout for conflict-free reads:
+// chunk c (32 k) of row r is 4 16-byte quads at uint4 index ((r * GA + c / 32) * 4 + q) * 32 +
+// c % 32 (GA = ceil(nch / 32)), so a warp reading 32 consecutive chunks touches 512
+// contiguous bytes per quad. Values are f16 scaled by a power of two per 16-block that puts
+// the block maximum in [2^14, 2^15); As[r][b] holds the inverse scale.
 __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A, int64_t k, int m,
-                                                  int64_t kbase, int nch, uint4* Ah4, float* As) {
-  const int G = (nch + 31) / 32;
+                                                  int64_t kbase, int nch, uint4* Ah4, float* As, int tid,
+                                                  int nthreads) {
+  const int GA = (nch + 31) / 32;
   const int blocks_per_row = nch * 2;
   const int nblk = m * blocks_per_row;
-  for (int bi = threadIdx.x; bi < nblk; bi += blockDim.x) {
+  for (int bi = tid; bi < nblk; bi += nthreads) {
     const int r = bi / blocks_per_row;
     const int b = bi - r * blocks_per_row;
     const uint16_t* src = A + (int64_t)r * k + kbase + (int64_t)b * 16;
@@ -60,8 +136,7 @@ __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A
       e = max(e, (w[i] >> 7) & 0xFFu);
       e = max(e, (w[i] >> 23) & 0xFFu);
     }
-    // scale the block maximum into [2^14, 2^15): biased exponent E -> shift 141 - E
-    int sh = 141 - (int)e;
+    int sh = 141 - (int)e;  // biased exponent E -> block maximum in [2^14, 2^15)
     sh = sh < -126 ? -126 : (sh > 126 ? 126 : sh);
     const float up = __uint_as_float((uint32_t)(sh + 127) << 23);
     const float down = __uint_as_float((uint32_t)(127 - sh) << 23);
@@ -73,16 +148,15 @@ __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A
       h[i] = f32x2_to_f16x2(lo, hi);
     }
     const int c = b >> 1, half = b & 1;
-    uint4* dst = Ah4 + ((int64_t)(r * G + c / 32) * 4 + 2 * half) * 32 + (c % 32);
+    uint4* dst = Ah4 + ((int64_t)(r * GA + c / 32) * 4 + 2 * half) * 32 + (c % 32);
     dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
     dst[32] = make_uint4(h[4], h[5], h[6], h[7]);
     As[r * blocks_per_row + b] = down;
   }
 }
 
-// Sum of 16 products a_i * w_i (8 f16x2 words each), sequential in element order.
-__device__ __forceinline__ float dot16(const uint32_t* a, const uint32_t* w) {
-  float p = 0.0f;
+// p += a_i * w_i for the 8 f16 pairs of one 16-block, in element order.
+__device__ __forceinline__ float dot16(const uint32_t* a, const uint32_t* w, float p) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     p = fma_lo_f16(a[i], w[i], p);
@@ -91,284 +165,272 @@ __device__ __forceinline__ float dot16(const uint32_t* a, const uint32_t* w) {
   return p;
 }
 
-template <int R>
-struct Step {
-  uint4 q[R];
-  uint32_t sc[R];
-};
-
-__device__ __forceinline__ void named_barrier(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+// Decode one 16-byte code quad (32 E2M1 codes) into 16 f16x2 words.
+__device__ __forceinline__ void decode32(const uint4 q, uint32_t* wf) {
+  const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int wd = 0; wd < 4; ++wd) {
+    wf[wd * 4 + 0] = e2m1x2_byte_to_f16x2<0>(words[wd]);
+    wf[wd * 4 + 1] = e2m1x2_byte_to_f16x2<1>(words[wd]);
+    wf[wd * 4 + 2] = e2m1x2_byte_to_f16x2<2>(words[wd]);
+    wf[wd * 4 + 3] = e2m1x2_byte_to_f16x2<3>(words[wd]);
+  }
 }
 
 }  // namespace
 
-// Occupancy target per instance (register budget per thread = 65536 / (256 * CTAs)): the
-// small-m streaming instances keep three CTAs (24 warps) per SM resident.
 template <int MT, int R>
-constexpr int gemv_min_ctas() {
-  return (MT * R <= 2) ? 3 : (MT * R <= 8 && MT <= 4) ? 2 : 1;
-}
+__global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ volatile int abort_flag;
 
-template <int MT, int R, int D>
-__global__ void __launch_bounds__(kGemvThreads, gemv_min_ctas<MT, R>()) gemv_nvfp4_kernel(GemvArgs p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  // a PDL-launched successor (the split-K reduce, or the next op) may be scheduled now; it
-  // waits for this grid's completion before touching what this grid writes
-  pdl_launch_dependents();
-
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const bool producer = warp == kGemvConsumerWarps;
   const int m = (int)p.m;
   const int64_t n = p.n, k = p.k;
   const int S = p.splits;
   const int s = blockIdx.y;
-  const int KW = p.kw;
-  const int NS = kGemvWarps / KW;  // row-group slots per CTA
-  const int slot = warp / KW;
-  const int kw = warp - slot * KW;
+  const int KW = p.kw, NS = kGemvConsumerWarps / KW;
+  const int TR = NS * R;
+  const int SL = p.slab, NST = p.stages;
 
-  // K range of this split (in 32-k chunks) and of this warp inside it
+  // K range of this split, in 32-k chunks
   const int64_t C = k / kChunkK;
   const int64_t c0 = (int64_t)s * C / S;
   const int nch = (int)((int64_t)(s + 1) * C / S - c0);
-  const int G = (nch + 31) / 32;
-  const int w0 = kw * nch / KW;
-  const int wch = (kw + 1) * nch / KW - w0;
-  // at least one (possibly empty) step per row group, so every warp of a slot meets the
-  // slot's barrier once per row group even when its share of k is empty
-  const int T = wch > 0 ? (wch + 31) / 32 : 1;
-  const int climit = wch - lane;  // step t is live for this lane iff 32 * t < climit
+  const int nslab = (nch + SL - 1) / SL;
 
-  // row groups of this CTA, and of this warp's slot
-  const int64_t RG = (n + R - 1) / R;
-  const int64_t rg_lo = (int64_t)blockIdx.x * RG / gridDim.x;
-  const int64_t rg_hi = (int64_t)(blockIdx.x + 1) * RG / gridDim.x;
-  const int nrg = (rg_lo + slot < rg_hi) ? (int)((rg_hi - rg_lo - slot + NS - 1) / NS) : 0;
-  const int F = nrg * T;
+  // tiles (TR rows) of this CTA
+  const int64_t tiles = (n + TR - 1) / TR;
+  const int64_t t_lo = (int64_t)blockIdx.x * tiles / gridDim.x;
+  const int64_t t_hi = (int64_t)(blockIdx.x + 1) * tiles / gridDim.x;
+  const int64_t Q = (t_hi - t_lo) * nslab;  // ring stages this CTA consumes
 
+  // shared memory carve-up (offsets computed on the host, 128-byte aligned)
   uint4* Ah4 = reinterpret_cast<uint4*>(smem);
-  float* As = reinterpret_cast<float*>(smem + (int64_t)m * G * 32 * 64);
-  float* comb = As + m * nch * 2;  // [2][NS][KW][R*MT], used when KW > 1
+  float* As = reinterpret_cast<float*>(smem + p.off_as);
+  float* comb = reinterpret_cast<float*>(smem + p.off_comb);  // [2][8 warps][R * MT]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  uint64_t* empty = full + NST;
+  uint8_t* ring = smem + p.off_ring;
+  const int codes_stride = SL * 16;           // bytes per row of codes in a stage
+  const int scales_stride = SL * 2 + 32;      // bytes per row of scales (+ alignment slack)
+  const int scales_off = TR * codes_stride;   // start of the scale rows in a stage
 
-  // load cursor: one pointer per row, advanced 32 chunks per step and jumped to the next
-  // row group of this slot (NS * R rows further) after T steps
-  const int64_t rs_q = k / 2, rs_s = k / 16;
-  const uint8_t* lq[R];
-  const uint8_t* ls[R];
-  {
-    const int64_t j0 = (rg_lo + slot) * R;
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-      lq[i] = p.Wq + (j0 + i) * rs_q + (c0 + w0 + lane) * 16;
-      ls[i] = p.Ws + (j0 + i) * rs_s + (c0 + w0 + lane) * 2;
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kGemvConsumerWarps);
     }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  const int64_t jump_q = (int64_t)NS * R * rs_q - (int64_t)T * 32 * 16;
-  const int64_t jump_s = (int64_t)NS * R * rs_s - (int64_t)T * 32 * 2;
-  // rows of the row group being fetched that exist (0 once past this warp's row groups)
-  int64_t l_left = nrg > 0 ? n - (rg_lo + slot) * R : 0;
-  int l_t = 0, l_g = 0;
-  auto issue = [&](Step<R>& st) {
-    const bool live = 32 * l_t < climit && l_g < nrg;
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-      if (live && i < l_left) {
-        st.q[i] = ldg_stream_v4(lq[i]);
-        st.sc[i] = ldg_stream_u16(ls[i]);
-      } else {
-        st.q[i] = make_uint4(0, 0, 0, 0);
-        st.sc[i] = 0;
-      }
-      lq[i] += 32 * 16;
-      ls[i] += 32 * 2;
-    }
-    if (++l_t == T) {
-      l_t = 0;
-      ++l_g;
-      l_left -= (int64_t)NS * R;
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        lq[i] += jump_q;
-        ls[i] += jump_s;
-      }
-    }
-  };
-
-  // prologue: put the first D steps of the weight stream in flight (weights are never written
-  // by the preceding kernel), then wait for the producer of A and stage it
-  Step<R> ring[D];
-#pragma unroll
-  for (int d = 0; d < D; ++d) issue(ring[d]);
-  pdl_wait();
-  stage_activations(p.A, k, m, c0 * kChunkK, nch, Ah4, As);
   __syncthreads();
+  // a PDL-launched successor may be scheduled now; it waits for this grid's completion
+  pdl_launch_dependents();
 
-  const float g = (S == 1) ? *p.gscale : 1.0f;
-  float acc[R][MT];
-#pragma unroll
-  for (int i = 0; i < R; ++i)
-#pragma unroll
-    for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
+  const int64_t rs_q = k / 2, rs_s = k / 16;
+  const int64_t scale_bytes_total = n * rs_s;
 
-  // compute cursor: this lane's activation quads and block scales for step t
-  const int ca0 = w0 + lane;
-  const uint4* a_base = Ah4 + (int64_t)(ca0 / 32) * 4 * 32 + (ca0 % 32);
-  const float2* s_base = reinterpret_cast<const float2*>(As) + ca0;
-  int ct = 0, cg = 0;
-  for (int f0 = 0; f0 < F; f0 += D) {
-#pragma unroll
-    for (int d = 0; d < D; ++d) {
-      if (f0 + d < F) {
-        Step<R>& cur = ring[d];
-        if (MT == 1 && 32 * ct < climit) {
-          // one activation row: decode each weight word straight into the FMAs (same
-          // element order as below, fewer live registers)
-          const uint4* ap = a_base + (int64_t)ct * 4 * 32;
-          const uint4 a0 = ap[0], a1 = ap[32], a2 = ap[64], a3 = ap[96];
-          const uint32_t a[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
-                                  a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-          const float2 sa = s_base[ct * 32];
-#pragma unroll
-          for (int i = 0; i < R; ++i) {
-            const uint32_t words[4] = {cur.q[i].x, cur.q[i].y, cur.q[i].z, cur.q[i].w};
-            float pb[2] = {0.0f, 0.0f};
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {
-              const uint32_t h0 = e2m1x2_byte_to_f16x2<0>(words[wd]);
-              const uint32_t h1 = e2m1x2_byte_to_f16x2<1>(words[wd]);
-              const uint32_t h2 = e2m1x2_byte_to_f16x2<2>(words[wd]);
-              const uint32_t h3 = e2m1x2_byte_to_f16x2<3>(words[wd]);
-              float& pp = pb[wd >> 1];
-              pp = fma_lo_f16(a[wd * 4 + 0], h0, pp);
-              pp = fma_hi_f16(a[wd * 4 + 0], h0, pp);
-              pp = fma_lo_f16(a[wd * 4 + 1], h1, pp);
-              pp = fma_hi_f16(a[wd * 4 + 1], h1, pp);
-              pp = fma_lo_f16(a[wd * 4 + 2], h2, pp);
-              pp = fma_hi_f16(a[wd * 4 + 2], h2, pp);
-              pp = fma_lo_f16(a[wd * 4 + 3], h3, pp);
-              pp = fma_hi_f16(a[wd * 4 + 3], h3, pp);
-            }
-            const uint32_t sh = e4m3x2_to_f16x2(cur.sc[i]);
-            acc[i][0] = fmaf(pb[0], f16_lo_to_f32(sh) * sa.x, acc[i][0]);
-            acc[i][0] = fmaf(pb[1], f16_hi_to_f32(sh) * sa.y, acc[i][0]);
+  if (producer) {
+    // ------------------------------------------------------------------ producer warp
+    int64_t issued = 0;
+    if (lane == 0 && !p.debug_stall) {
+      for (int64_t q = 0; q < Q; ++q) {
+        const int slot = (int)(q % NST);
+        if (q >= NST && !mbar_wait_bounded(&empty[slot], (uint32_t)((q / NST - 1) & 1), &abort_flag,
+                                           p.timeout_ns, 2u))
+          break;
+        const int64_t tile = t_lo + q / nslab;
+        const int sb = (int)(q % nslab);
+        const int a = sb * SL;
+        const int len = min(SL, nch - a);
+        uint8_t* stage = ring + (int64_t)slot * p.stage_bytes;
+        uint32_t bytes = 0;
+        const int64_t j0 = tile * TR;
+        const int rows = (int)min((int64_t)TR, n - j0);
+        // plain-load tail first (only a scale superset that would overrun the tensor)
+        for (int r = 0; r < rows; ++r) {
+          const int64_t st = (j0 + r) * rs_s + (c0 + a) * 2;
+          const int64_t al = st & ~(int64_t)15;
+          const int64_t ae = (st + (int64_t)len * 2 + 15) & ~(int64_t)15;
+          if (ae > scale_bytes_total) {
+            uint8_t* dst = stage + scales_off + r * scales_stride;
+            for (int64_t b = al; b < st + (int64_t)len * 2; ++b) dst[b - al] = p.Ws[b];
+          } else {
+            bytes += (uint32_t)(ae - al);
           }
-        } else if (MT > 1 && 32 * ct < climit) {
-          uint32_t wf[R][16];
-          float sw[R][2];
-#pragma unroll
-          for (int i = 0; i < R; ++i) {
-            const uint32_t words[4] = {cur.q[i].x, cur.q[i].y, cur.q[i].z, cur.q[i].w};
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {
-              wf[i][wd * 4 + 0] = e2m1x2_byte_to_f16x2<0>(words[wd]);
-              wf[i][wd * 4 + 1] = e2m1x2_byte_to_f16x2<1>(words[wd]);
-              wf[i][wd * 4 + 2] = e2m1x2_byte_to_f16x2<2>(words[wd]);
-              wf[i][wd * 4 + 3] = e2m1x2_byte_to_f16x2<3>(words[wd]);
-            }
-            const uint32_t sh = e4m3x2_to_f16x2(cur.sc[i]);
-            sw[i][0] = f16_lo_to_f32(sh);
-            sw[i][1] = f16_hi_to_f32(sh);
-          }
-#pragma unroll
-          for (int r = 0; r < MT; ++r) {
-            if (r < m) {
-              const uint4* ap = a_base + ((int64_t)r * G + ct) * 4 * 32;
-              const uint4 a0 = ap[0], a1 = ap[32], a2 = ap[64], a3 = ap[96];
-              const uint32_t a[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
-                                      a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-              const float2 sa = s_base[r * nch + ct * 32];
-#pragma unroll
-              for (int i = 0; i < R; ++i) {
-                const float p0 = dot16(a, wf[i]);
-                const float p1 = dot16(a + 8, wf[i] + 8);
-                acc[i][r] = fmaf(p0, sw[i][0] * sa.x, acc[i][r]);
-                acc[i][r] = fmaf(p1, sw[i][1] * sa.y, acc[i][r]);
-              }
-            }
-          }
+          bytes += (uint32_t)len * 16;
         }
-        // refill this ring slot with the step D ahead (predicated off past the end)
-        issue(cur);
+        mbar_arrive_expect_tx(&full[slot], bytes);
+        for (int r = 0; r < rows; ++r) {
+          const int64_t j = j0 + r;
+          bulk_g2s(stage + r * codes_stride, p.Wq + j * rs_q + (c0 + a) * 16, (uint32_t)len * 16, &full[slot]);
+          const int64_t st = j * rs_s + (c0 + a) * 2;
+          const int64_t al = st & ~(int64_t)15;
+          const int64_t ae = (st + (int64_t)len * 2 + 15) & ~(int64_t)15;
+          if (ae <= scale_bytes_total)
+            bulk_g2s(stage + scales_off + r * scales_stride, p.Ws + al, (uint32_t)(ae - al), &full[slot]);
+        }
+        issued = q + 1;
+      }
+      // drain: every copy this CTA issued must have landed before the CTA exits
+      const int64_t first = issued > NST ? issued - NST : 0;
+      for (int64_t q = first; q < issued; ++q)
+        mbar_wait_bounded(&full[q % NST], (uint32_t)((q / NST) & 1), &abort_flag, p.timeout_ns, 4u);
+    }
+    return;
+  }
 
-        if (ct == T - 1) {
-          // row group cg is complete: reduce over lanes, then over the slot's KW warps
-          const int64_t j0 = (rg_lo + slot + (int64_t)cg * NS) * R;
-          const int par = cg & 1;
+  // -------------------------------------------------------------------- consumer warps
+  const int slot_id = warp / KW;
+  const int kw = warp - slot_id * KW;
+  pdl_wait();
+  const int GA = (nch + 31) / 32;
+  stage_activations(p.A, k, m, c0 * kChunkK, nch, Ah4, As, tid, kGemvConsumerWarps * 32);
+  named_barrier(1, kGemvConsumerWarps * 32);
+  const float g = (S == 1) ? *p.gscale : 1.0f;
+
+  float acc[R][MT];
+  int64_t q = 0;
+  for (int64_t tile = t_lo; tile < t_hi; ++tile) {
 #pragma unroll
-          for (int i = 0; i < R; ++i) {
+    for (int i = 0; i < R; ++i)
 #pragma unroll
-            for (int r = 0; r < MT; ++r) {
-              float v = acc[i][r];
+      for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
+    const int64_t j0 = tile * TR + slot_id * R;  // first row of this warp's slot
+    const int rows = (int)max((int64_t)0, min((int64_t)R, n - j0));
+    for (int sb = 0; sb < nslab; ++sb, ++q) {
+      const int slot = (int)(q % NST);
+      const bool ok = mbar_wait_bounded(&full[slot], (uint32_t)((q / NST) & 1), &abort_flag, p.timeout_ns, 1u);
+      const int a = sb * SL;
+      const int len = min(SL, nch - a);
+      if (ok) {
+        const uint8_t* stage = ring + (int64_t)slot * p.stage_bytes;
+        // scale superset offset of each of this warp's rows
+        int soff[R];
 #pragma unroll
-              for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-              acc[i][r] = v;
-            }
-          }
-          if (KW > 1) {
-            float* mine = comb + ((par * NS + slot) * KW + kw) * (R * MT);
-#pragma unroll
-            for (int i = 0; i < R; ++i)
-#pragma unroll
-              for (int r = 0; r < MT; ++r)
-                if (lane == ((i * MT + r) & 31)) mine[i * MT + r] = acc[i][r];
-            named_barrier(1 + slot, KW * 32);
-            if (kw == 0) {
-              const float* all = comb + (par * NS + slot) * KW * (R * MT);
-#pragma unroll
-              for (int i = 0; i < R; ++i)
-#pragma unroll
-                for (int r = 0; r < MT; ++r) {
-                  float v = acc[i][r];
-                  for (int q = 1; q < KW; ++q) v += all[q * (R * MT) + i * MT + r];
-                  acc[i][r] = v;
-                }
-            }
-          }
-          if (KW == 1 || kw == 0) {
+        for (int i = 0; i < R; ++i) soff[i] = (int)((((j0 + i) * rs_s) + (c0 + a) * 2) & 15);
+        for (int lc = 32 * kw + lane; lc < len; lc += 32 * KW) {
+          const int c = a + lc;  // chunk inside the split
+          // activations: 4 quads per activation row, and the two block scales
+          const uint4* ap = Ah4 + ((int64_t)(c / 32) * 4) * 32 + (c % 32);
+          const float2* sp = reinterpret_cast<const float2*>(As) + c;
+          if (MT == 1) {
+            const uint4 a0 = ap[0], a1 = ap[32], a2 = ap[64], a3 = ap[96];
+            const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                                     a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+            const float2 sa = sp[0];
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-              const int64_t j = j0 + i;
+              if (i < rows) {
+                const int rr = slot_id * R + i;
+                const uint4 cq = *reinterpret_cast<const uint4*>(stage + rr * codes_stride + lc * 16);
+                const uint32_t sc = *reinterpret_cast<const uint16_t*>(stage + scales_off + rr * scales_stride +
+                                                                       soff[i] + lc * 2);
+                uint32_t wf[16];
+                decode32(cq, wf);
+                const float p0 = dot16(av, wf, 0.0f);
+                const float p1 = dot16(av + 8, wf + 8, 0.0f);
+                const uint32_t sh = e4m3x2_to_f16x2(sc);
+                acc[i][0] = fmaf(p0, f16_lo_to_f32(sh) * sa.x, acc[i][0]);
+                acc[i][0] = fmaf(p1, f16_hi_to_f32(sh) * sa.y, acc[i][0]);
+              }
+            }
+          } else {
+            uint32_t wf[R][16];
+            float sw[R][2];
 #pragma unroll
-              for (int r = 0; r < MT; ++r) {
-                if (r < m && j < n && lane == ((i * MT + r) & 31)) {
-                  if (S == 1)
-                    p.out[(int64_t)r * n + j] = f32_to_bf16_rn(acc[i][r] * g);
-                  else
-                    p.partials[((int64_t)s * m + r) * n + j] = acc[i][r];
+            for (int i = 0; i < R; ++i) {
+              const int rr = slot_id * R + i;
+              uint4 cq = make_uint4(0, 0, 0, 0);
+              uint32_t sc = 0;
+              if (i < rows) {
+                cq = *reinterpret_cast<const uint4*>(stage + rr * codes_stride + lc * 16);
+                sc = *reinterpret_cast<const uint16_t*>(stage + scales_off + rr * scales_stride + soff[i] + lc * 2);
+              }
+              decode32(cq, wf[i]);
+              const uint32_t sh = e4m3x2_to_f16x2(sc);
+              sw[i][0] = f16_lo_to_f32(sh);
+              sw[i][1] = f16_hi_to_f32(sh);
+            }
+#pragma unroll
+            for (int r = 0; r < MT; ++r) {
+              if (r < m) {
+                const uint4* apr = ap + (int64_t)r * GA * 4 * 32;
+                const uint4 a0 = apr[0], a1 = apr[32], a2 = apr[64], a3 = apr[96];
+                const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                                         a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+                const float2 sa = sp[(int64_t)r * nch];
+#pragma unroll
+                for (int i = 0; i < R; ++i) {
+                  const float p0 = dot16(av, wf[i], 0.0f);
+                  const float p1 = dot16(av + 8, wf[i] + 8, 0.0f);
+                  acc[i][r] = fmaf(p0, sw[i][0] * sa.x, acc[i][r]);
+                  acc[i][r] = fmaf(p1, sw[i][1] * sa.y, acc[i][r]);
                 }
               }
             }
           }
-#pragma unroll
-          for (int i = 0; i < R; ++i)
-#pragma unroll
-            for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
-        }
-        if (++ct == T) {
-          ct = 0;
-          ++cg;
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+    // the tile is done: lanes, then the slot's KW warps in order
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+      for (int r = 0; r < MT; ++r) {
+        float v = acc[i][r];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        acc[i][r] = v;
+      }
+    const int par = (int)((tile - t_lo) & 1);
+    if (KW > 1) {
+      float* mine = comb + ((par * kGemvConsumerWarps) + warp) * (R * MT);
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int r = 0; r < MT; ++r)
+          if (lane == ((i * MT + r) & 31)) mine[i * MT + r] = acc[i][r];
+      named_barrier(2 + slot_id, KW * 32);
+      if (kw == 0) {
+        const float* all = comb + (par * kGemvConsumerWarps + warp) * (R * MT);
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+#pragma unroll
+          for (int r = 0; r < MT; ++r) {
+            float v = acc[i][r];
+            for (int w = 1; w < KW; ++w) v += all[w * (R * MT) + i * MT + r];
+            acc[i][r] = v;
+          }
+      }
+    }
+    if (kw == 0 && !abort_flag) {
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int r = 0; r < MT; ++r)
+          if (i < rows && r < m && lane == ((i * MT + r) & 31)) {
+            const int64_t j = j0 + i;
+            if (S == 1)
+              p.out[(int64_t)r * n + j] = f32_to_bf16_rn(acc[i][r] * g);
+            else
+              p.partials[((int64_t)s * m + r) * n + j] = acc[i][r];
+          }
     }
   }
 }
 
 namespace {
 
-template <typename K>
-int occupancy(K kern, int smem_bytes) {
-  int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvThreads, smem_bytes) != cudaSuccess) {
-    cudaGetLastError();
-    return 1;
-  }
-  return occ > 0 ? occ : 1;
-}
-
-template <int MT, int R, int D>
+template <int MT, int R>
 int launch_one(const GemvArgs& a, cudaStream_t stream) {
-  auto kern = gemv_nvfp4_kernel<MT, R, D>;
+  auto kern = gemv_nvfp4_kernel<MT, R>;
   // the opt-in shared memory limit is a per-device function attribute; raise it once
   static int configured[kMaxDevices] = {};
   int dev = 0;
@@ -379,14 +441,8 @@ int launch_one(const GemvArgs& a, cudaStream_t stream) {
       return set_cuda_error("cudaFuncSetAttribute(gemv smem)");
     configured[dev] = 1;
   }
-  // the grid is persistent: never ask for more CTAs than fit at once
-  const int occ = occupancy(kern, a.smem_bytes);
-  const int ctas = a.ctas_per_sm < occ ? a.ctas_per_sm : occ;
-  int64_t gx = (int64_t)a.num_sms * ctas / a.splits;
-  if (gx < 1) gx = 1;
-  if (gx > a.grid_x) gx = a.grid_x;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)gx, (unsigned)a.splits);
+  cfg.gridDim = dim3((unsigned)a.grid_x, (unsigned)a.splits);
   cfg.blockDim = dim3(kGemvThreads);
   cfg.dynamicSmemBytes = (size_t)a.smem_bytes;
   cfg.stream = stream;
@@ -401,12 +457,11 @@ int launch_one(const GemvArgs& a, cudaStream_t stream) {
 
 template <int MT>
 int launch_rows(const GemvArgs& a, cudaStream_t stream) {
-  constexpr int D1 = MT <= 4 ? 4 : 2;
   switch (a.rows_per_warp) {
-    case 1: return launch_one<MT, 1, D1>(a, stream);
-    case 2: return launch_one<MT, 2, 2>(a, stream);
+    case 1: return launch_one<MT, 1>(a, stream);
+    case 2: return launch_one<MT, 2>(a, stream);
     case 4:
-      if constexpr (MT <= 16) return launch_one<MT, 4, 2>(a, stream);
+      if constexpr (MT <= 16) return launch_one<MT, 4>(a, stream);
       return set_error(FI_ERR_INVALID_ARG, "GEMV with 4 rows per warp supports m <= 16");
     default: return set_error(FI_ERR_INVALID_ARG, "GEMV rows per warp must be 1, 2 or 4");
   }
@@ -422,6 +477,16 @@ int launch_gemv(const GemvArgs& a, cudaStream_t stream) {
   if (a.m <= 16) return launch_rows<16>(a, stream);
   if (a.m <= 32) return launch_rows<32>(a, stream);
   return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV supports m <= %d", kGemvMaxM);
+}
+
+int gemv_read_error(unsigned* bits) {
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_gemv_error, sizeof(v)) != cudaSuccess)
+    return set_cuda_error("cudaMemcpyFromSymbol(gemv error)");
+  if (v && cudaMemcpyToSymbol(g_gemv_error, &zero, sizeof(zero)) != cudaSuccess)
+    return set_cuda_error("cudaMemcpyToSymbol(gemv error)");
+  *bits = v;
+  return FI_OK;
 }
 
 }  // namespace fi

@@ -20,13 +20,13 @@ void clear_error();
 int device_sm_count();
 
 // ------------------------------------------------------------------------ GEMV
-// Geometry shared by the tactic resolver and the GEMV launcher.
-constexpr int kGemvWarps = 8;                 // warps per CTA
-constexpr int kGemvThreads = kGemvWarps * 32;
-constexpr int kChunkK = 32;                   // k per lane per step (16 code bytes)
-constexpr int kWarpK = 32 * kChunkK;          // k per warp step (512 code bytes)
+constexpr int kGemvConsumerWarps = 8;                     // warps that decode and multiply
+constexpr int kGemvThreads = (kGemvConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kChunkK = 32;                                // k per lane per step (16 code bytes)
 constexpr int kGemvMaxM = 32;
-constexpr int kSmemBudget = 200 * 1024;       // dynamic shared memory we allow per CTA
+constexpr int kSmemBudget = 227 * 1024 - 1024;             // dynamic shared memory per CTA we allow
+constexpr int kGemvMaxStages = 8;
+constexpr int kGemvStageTarget = 32 * 1024;                // preferred bytes per ring stage
 
 // Activation rows the GEMV kernel instance for m is compiled for (1, 2, 4, ..., 32).
 inline int gemv_mt(int64_t m) {
@@ -35,13 +35,20 @@ inline int gemv_mt(int64_t m) {
   return mt;
 }
 
-// Shared memory the GEMV needs: m activation rows over klen k as f16, padded to whole warp
-// steps of 1024 k, plus one fp32 power-of-two scale per 16-block, plus the in-CTA split-K
-// combine buffer (2 parities x 8 warps x R rows x MT activation rows, fp32).
-inline int64_t gemv_smem_bytes(int64_t m, int64_t klen, int R) {
-  const int64_t padded = (klen + 1023) / 1024 * 1024;
-  return m * padded * 2 + m * (klen / 16) * 4 + 2 * 8 * (int64_t)R * gemv_mt(m) * 4;
-}
+inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// Bytes of one row of E4M3 scales in a ring stage of `slab` chunks: the copied superset starts
+// up to 14 bytes before the row's first scale and is rounded to 16 bytes at both ends.
+inline int64_t gemv_scales_stride(int64_t slab) { return round_up(slab * 2 + 28, 16); }
+
+// Launch geometry of the GEMV for one shape and tactic (computed on the host).
+struct GemvGeometry {
+  int S, R, KW, TR, slab, stages, ctas_per_sm, grid_x;
+  int64_t stage_bytes, off_as, off_comb, off_bar, off_ring, smem_bytes;
+};
+// Returns FI_OK and fills g, or FI_ERR_UNSUPPORTED_SHAPE when the activations of m rows over
+// a split do not leave room for two ring stages in shared memory.
+int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int R, int ctas_per_sm, int sms, GemvGeometry* g);
 
 struct GemvArgs {
   const uint16_t* A;
@@ -51,16 +58,19 @@ struct GemvArgs {
   uint16_t* out;       // used when splits == 1
   float* partials;     // [splits, m, n] when splits > 1
   int64_t m, n, k;
-  int splits;         // S: global K splits (grid.y)
-  int kw;             // KW: warps sharing one row group inside a CTA (1, 2, 4, 8)
-  int rows_per_warp;  // R
-  int grid_x;         // CTAs per split wanted by the tactic (capped by occupancy at launch)
-  int ctas_per_sm;
-  int num_sms;
-  int smem_bytes;
-  int pdl;            // launch with programmatic stream serialization
+  int splits;          // S: global K splits (grid.y)
+  int kw;              // KW: consumer warps sharing one row's k range
+  int rows_per_warp;   // R
+  int slab;            // SL: 32-k chunks per ring stage
+  int stages;          // NST: ring stages
+  int grid_x;          // CTAs per split
+  int pdl;             // launch with programmatic stream serialization
+  int debug_stall;     // test hook: the producer issues nothing (consumer waits time out)
+  int64_t stage_bytes, off_as, off_comb, off_bar, off_ring, smem_bytes;
+  uint64_t timeout_ns; // limit of every mbarrier wait
 };
 int launch_gemv(const GemvArgs& a, cudaStream_t stream);
+int gemv_read_error(unsigned* bits);
 
 // ---------------------------------------------------------------------- reduce
 int launch_splitk_reduce(const float* partials, int splits, int64_t m, int64_t n,

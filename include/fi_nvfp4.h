@@ -66,7 +66,7 @@ typedef enum {
  *                (PR #4038, "Sizes GEMV split-K from the device");
  *   ctas_per_sm  co-resident CTAs per SM used to size the grid (1..15); 0 = automatic
  *                (PR #4038, "Adds occupancy tactics");
- *   variant      GEMV: weight rows per warp (1, 2 or 4; 0 = automatic). MMA: 0.
+ *   variant      GEMV: weight rows per consumer warp (1, 2 or 4; 0 = automatic). MMA: 0.
  * Only `kind` and the resolved S change the arithmetic: two tactics with the same kind
  * and S give bitwise identical outputs, and for a fixed tactic every output row is
  * bitwise independent of m. FI_TACTIC_DEFAULT (-1) selects from the built-in per-shape
@@ -104,7 +104,7 @@ typedef struct {
  * Quantise fp32 weights to NVFP4 (the weight-preparation step; not on the timed path).
  *   W       device fp32 [n, k], row-major, 16-byte aligned.
  *   Wq      device uint8 [n, k/2] (output), 16-byte aligned.
- *   Wscale  device uint8 [n, k/16] (output), 8-byte aligned.
+ *   Wscale  device uint8 [n, k/16] (output), 16-byte aligned.
  *   gscale  device fp32 [1] (output); also used as scratch by the call.
  * Recipe: gscale = amax(|W|) / (448*6) (one fp32 division); for each 16-block
  * sf = E4M3_rn_satfinite((amax_block / 6) / gscale); denom = sf * gscale;
@@ -120,8 +120,11 @@ FI_API int fi_nvfp4_pack_weights(const float* W, int64_t n, int64_t k, uint8_t* 
  * out[m, n] = bf16_rn(gscale * sum_k A[m, k] * e2m1(Wq) * e4m3(Wscale)), fp32 accumulate
  * (PR #4038, Description).
  *   A       device bf16 bits [m, k], 16-byte aligned.
- *   Wq, Wscale, gscale  NVFP4 weights as produced by fi_nvfp4_pack_weights; Wq 16-byte
- *           aligned, Wscale 2-byte aligned.
+ *   Wq, Wscale, gscale  NVFP4 weights as produced by fi_nvfp4_pack_weights; Wq and Wscale
+ *           16-byte aligned. The weights are read with bulk asynchronous copies that may
+ *           start before the kernel that precedes this call on `stream` has finished
+ *           (programmatic dependent launch): Wq, Wscale must not be written by that kernel.
+ *           A and gscale are read, and out written, only after it has completed.
  *   out     device bf16 bits [m, n], 2-byte aligned; must not overlap the inputs.
  *   tactic  FI_TACTIC_DEFAULT or an FI_TACTIC(...) code (see above).
  * Preconditions: m >= 0, n >= 0, k >= 0, k % 32 == 0; m <= 32 for GEMV tactics and
@@ -189,6 +192,26 @@ FI_API size_t fi_mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int64_t tac
  * allocated itself for that device. The caller keeps ownership of `ptr` and must keep it
  * alive while calls that use it may run. */
 FI_API int fi_set_workspace(void* ptr, size_t bytes);
+
+/* ------------------------------------------------------------ failure detection
+ * Every wait inside the kernels (on the shared-memory pipeline's mbarriers) is bounded in
+ * time: when a wait runs out, the kernel records a bit in a sticky per-device error word,
+ * stops computing, lets its in-flight copies land and returns; the outputs of that call are
+ * then undefined. The library has no counterpart on the pages; it exists so that a stuck
+ * pipeline ends with an error instead of a hung GPU.
+ */
+
+/* Read and clear the current device's sticky kernel error word (0 = no error; bit 0: a
+ * consumer wait ran out, bit 1: a producer wait ran out, bit 2: the final drain ran out).
+ * Synchronizes the device. */
+FI_API int fi_get_device_error(unsigned* code);
+
+/* Test hooks. FI_DEBUG_STALL_PRODUCER: the producer warp of the next `value` GEMV launches
+ * issues no copies, so their waits run out (exercises the path above without a GPU fault).
+ * FI_DEBUG_WAIT_TIMEOUT_NS: limit of every kernel wait in ns (default 1e9). */
+#define FI_DEBUG_STALL_PRODUCER 1
+#define FI_DEBUG_WAIT_TIMEOUT_NS 2
+FI_API int fi_debug_set(int key, int64_t value);
 
 /* Message describing the last error on this host thread ("" if none). */
 FI_API const char* fi_last_error(void);

