@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
   uint64_t* empty = full + NST;
   uint8_t* ring = smem + p.off_ring;
   const int codes_stride = SL * 16;           // bytes per row of codes in a stage
-  const int scales_stride = SL * 2 + 32;      // bytes per row of scales (+ alignment slack)
+  const int scales_stride = (int)gemv_scales_stride(SL);  // bytes per row of scales (16-byte multiple)
   const int scales_off = TR * codes_stride;   // start of the scale rows in a stage
 
   if (tid == 0) {

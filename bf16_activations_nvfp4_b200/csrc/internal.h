@@ -35,11 +35,12 @@ inline int gemv_mt(int64_t m) {
   return mt;
 }
 
-inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+__host__ __device__ inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 // Bytes of one row of E4M3 scales in a ring stage of `slab` chunks: the copied superset starts
-// up to 14 bytes before the row's first scale and is rounded to 16 bytes at both ends.
-inline int64_t gemv_scales_stride(int64_t slab) { return round_up(slab * 2 + 28, 16); }
+// up to 14 bytes before the row's first scale and is rounded to 16 bytes at both ends. Shared
+// by the host's shared-memory layout and the kernel, so both always agree.
+__host__ __device__ inline int64_t gemv_scales_stride(int64_t slab) { return round_up(slab * 2 + 28, 16); }
 
 // Launch geometry of the GEMV for one shape and tactic (computed on the host).
 struct GemvGeometry {
