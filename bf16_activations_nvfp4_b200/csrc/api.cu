@@ -93,28 +93,23 @@ constexpr int kGemvDefaultRows = 2;
 int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int R, int ctas_per_sm, int sms, GemvGeometry* g) {
   const int64_t C = k / kChunkK;
   const int64_t nch = (C + S - 1) / S;  // chunks of the largest split
-  // KW: the largest power of two <= min(8, warp steps of a split)
-  const int64_t steps = (nch + 31) / 32;
-  int KW = 1;
-  while (KW * 2 <= kGemvConsumerWarps && KW * 2 <= steps) KW *= 2;
-  const int TR = (kGemvConsumerWarps / KW) * R;
+  const int TR = kGemvConsumerWarps * R;
   const int ctas = ctas_per_sm > 0 ? ctas_per_sm : 1;
   const int64_t per_cta = std::min<int64_t>(kSmemBudget, (228 * 1024) / ctas - 2048);
   const int64_t a_bytes = round_up(m * ((nch + 31) / 32) * 2048, 128);
   const int64_t as_bytes = round_up(m * nch * 8, 128);
-  const int64_t comb_bytes = round_up(2 * kGemvConsumerWarps * (int64_t)R * gemv_mt(m) * 4, 128);
   const int64_t bar_bytes = round_up(2 * kGemvMaxStages * 8, 128);
-  const int64_t fixed = a_bytes + as_bytes + comb_bytes + bar_bytes;
+  const int64_t fixed = a_bytes + as_bytes + bar_bytes;
   const int64_t avail = per_cta - fixed;
   auto stage_of = [&](int64_t sl) { return round_up(TR * (sl * 16 + gemv_scales_stride(sl)), 128); };
-  int64_t target = std::min<int64_t>(kGemvStageTarget, avail / 4);
+  // slab: whole split rows when a stage of them is small enough, else whole warp steps
+  const int64_t target = std::min<int64_t>(kGemvStageTarget, avail / 4);
   int64_t slab;
   if (stage_of(nch) <= target) {
     slab = nch;
   } else {
-    const int64_t unit = 32 * KW;
-    slab = unit;
-    while (slab + unit < nch && stage_of(slab + unit) <= target) slab += unit;
+    slab = 32;
+    while (slab + 32 < nch && stage_of(slab + 32) <= target) slab += 32;
   }
   const int64_t stage_bytes = stage_of(slab);
   const int64_t stages = std::min<int64_t>(kGemvMaxStages, avail > 0 ? avail / stage_bytes : 0);
@@ -123,21 +118,18 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int R, int ctas_per_sm
                      "GEMV: m=%lld over %lld k per split leaves no room for the weight ring in shared "
                      "memory; use more splits",
                      (long long)m, (long long)(nch * kChunkK));
-  const int64_t tiles = (n + TR - 1) / TR;
   int64_t gx = std::max<int64_t>(1, (int64_t)sms * ctas / S);
-  if (gx > tiles) gx = tiles;
+  if (gx > n) gx = std::max<int64_t>(1, n);
   g->S = S;
   g->R = R;
-  g->KW = KW;
   g->TR = TR;
   g->slab = (int)slab;
   g->stages = (int)stages;
   g->ctas_per_sm = ctas;
-  g->grid_x = (int)std::max<int64_t>(1, gx);
+  g->grid_x = (int)gx;
   g->stage_bytes = stage_bytes;
   g->off_as = a_bytes;
-  g->off_comb = a_bytes + as_bytes;
-  g->off_bar = a_bytes + as_bytes + comb_bytes;
+  g->off_bar = a_bytes + as_bytes;
   g->off_ring = fixed;
   g->smem_bytes = fixed + stages * stage_bytes;
   return FI_OK;
@@ -145,15 +137,14 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int R, int ctas_per_sm
 
 // Device-sized split (PR #4038, "Sizes GEMV split-K from the device"): the fewest splits S
 // that give every SM a CTA with rows to stream while `m_fit` activation rows of a split fit
-// the shared-memory staging. Depends on (n, k, SMs, R, m_fit) only.
+// the shared-memory staging next to the weight ring. Depends on (n, k, SMs, R, m_fit) only.
 static int gemv_knee(int64_t n, int64_t k, int sms, int64_t m_fit, int R, int ctas, int* S_out) {
   const int64_t C = k / kChunkK;
   const int64_t maxS = std::max<int64_t>(1, std::min<int64_t>(C, 4095));
   for (int64_t S = 1; S <= maxS; ++S) {
     GemvGeometry g;
     if (gemv_geometry(m_fit, n, k, (int)S, R, ctas, sms, &g) != FI_OK) continue;
-    const int64_t tiles = (n + g.TR - 1) / g.TR;
-    const bool enough = tiles * S >= (int64_t)sms * g.ctas_per_sm;
+    const bool enough = (int64_t)g.grid_x * S >= (int64_t)sms * g.ctas_per_sm;
     const bool last = S == maxS || (C / (S + 1)) < 32;  // a split keeps at least one warp step
     if (enough || last) {
       *S_out = (int)S;
@@ -171,9 +162,10 @@ static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms,
 static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms) {
   if (m <= kDefaultGemvMaxM) {
     const int64_t m_fit = m <= 1 ? 1 : (m <= 8 ? 8 : kGemvMaxM);
+    const int R = m_fit <= 4 ? kGemvDefaultRows : 1;  // keep register use within budget for larger m
     int S = 1;
-    if (gemv_knee(n, k, num_sms, m_fit, kGemvDefaultRows, 1, &S) != FI_OK) S = 1;
-    return FI_TACTIC(FI_KIND_GEMV, S, 0, kGemvDefaultRows);
+    if (gemv_knee(n, k, num_sms, m_fit, R, 1, &S) != FI_OK) S = 1;
+    return FI_TACTIC(FI_KIND_GEMV, S, 0, R);
   }
   return FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
 }
@@ -205,7 +197,6 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
     memset(&g, 0, sizeof(g));
     g.S = 1;
     g.R = R;
-    g.KW = 1;
     g.ctas_per_sm = ctas;
     g.grid_x = 1;
   } else {
@@ -364,7 +355,6 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.n = n;
     a.k = k;
     a.splits = g.S;
-    a.kw = g.KW;
     a.rows_per_warp = g.R;
     a.slab = g.slab;
     a.stages = g.stages;
@@ -374,7 +364,6 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     if (g_debug_stall_launches > 0) --g_debug_stall_launches;
     a.stage_bytes = g.stage_bytes;
     a.off_as = g.off_as;
-    a.off_comb = g.off_comb;
     a.off_bar = g.off_bar;
     a.off_ring = g.off_ring;
     a.smem_bytes = g.smem_bytes;

@@ -7,28 +7,27 @@
 //
 //  * Warp specialisation. One producer warp per CTA streams weight tiles HBM -> shared memory
 //    with bulk asynchronous copies (cp.async.bulk, completion counted on an mbarrier) into an
-//    NST-stage ring; 8 consumer warps decode from shared memory. In-flight bytes live in
-//    shared memory, not registers, and cost the producer one instruction per copy.
+//    NST-stage ring; 16 consumer warps decode from shared memory. In-flight bytes live in
+//    shared memory, not registers; the producer's 32 lanes issue the copies of up to 32 rows
+//    at once.
 //  * Programmatic dependent launch. The producer issues the first NST stages before the
 //    grid-dependency wait (weights are never written by the preceding kernel); the consumers
 //    wait, then stage the activations, so the weight stream overlaps the previous kernel's
 //    tail and the activation staging.
-//  * Tiles. Grid (G, S): blockIdx.y is the K split s. The split's weight rows are cut into
-//    tiles of TR = NS * R rows; the G CTAs of a split own balanced contiguous tile ranges. A
-//    tile's rows are fetched in slabs of SL 32-k chunks (one ring stage per slab): one bulk
-//    copy per row for the codes and one per row for the E4M3 scales (a 16-byte-aligned
-//    superset of the scale bytes, indexed from the remainder; the bytes past the end of the
-//    scale tensor, where a superset would overrun it, are copied with plain loads).
-//  * Work split. The 8 consumer warps form NS = 8 / KW slots of KW warps, KW = the largest
-//    power of two <= min(8, ceil(chunks / 32)). Slot `slot` computes rows slot*R .. slot*R+R-1
-//    of the tile; inside a slot, lane L of warp kw takes chunks c = 32*KW*t + 32*kw + L.
-//  * Arithmetic (fixed by k and S alone, hence bitwise identical for every m, R, TR, SL,
-//    NST, G and CTAs per SM): A is staged as f16 with one power-of-two scale per 16-block
-//    (exact for every element within 2^28 of its block maximum); codes are decoded by
+//  * Work. Grid (G, S): blockIdx.y is the K split s; the G CTAs of a split own balanced,
+//    contiguous ranges of weight rows (so every SM streams the same number of bytes, +-1 row)
+//    and walk them in tiles of TR = 16 * R rows; consumer warp w owns rows w*R .. w*R+R-1 of a
+//    tile. A tile's rows are fetched in slabs of SL 32-k chunks (one ring stage per slab): one
+//    bulk copy per row for the codes and one per row for the E4M3 scales (a 16-byte-aligned
+//    superset of the row's scale bytes, indexed from the remainder; a superset that would
+//    overrun the scale tensor is copied with plain loads instead).
+//  * Arithmetic (fixed by k and S alone, hence bitwise identical for every m, R, SL, NST, G
+//    and CTAs per SM): A is staged as f16 with one power-of-two scale per 16-block (exact for
+//    every element within 2^28 of its block maximum); codes are decoded by
 //    cvt.rn.f16x2.e2m1x2 (exact) and multiplied by the mixed-precision fma.rn.f32.f16 (exact
-//    product, fp32 accumulate); per 16-block p = sum_i a_i * e2m1_i in element order, then
-//    acc = fma(p, sf_w * sf_a, acc) over the lane's chunks in order; lanes combine through a
-//    fixed xor butterfly (all lanes end with the same bits), the KW warps in order kw = 0..KW-1.
+//    product, fp32 accumulate). Lane L takes chunks L, L+32, L+64, ... of the split: per
+//    16-block p = sum_i a_i * e2m1_i in element order, then acc = fma(p, sf_w * sf_a, acc);
+//    the lanes combine through a fixed xor butterfly (all lanes end with the same bits).
 //    S == 1 writes bf16_rn(acc * gscale); S > 1 writes fp32 partials for the reduce kernel.
 //  * Bounded waits. Every mbarrier wait gives up after a time limit (%globaltimer): it sets a
 //    device error flag and a CTA-wide abort flag, the CTA finishes its control flow without
@@ -184,16 +183,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ volatile int abort_flag;
 
+  constexpr int NC = kGemvConsumerWarps;
+  constexpr int TR = NC * R;  // rows per tile
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const bool producer = warp == kGemvConsumerWarps;
+  const bool producer = warp == NC;
   const int m = (int)p.m;
   const int64_t n = p.n, k = p.k;
   const int S = p.splits;
   const int s = blockIdx.y;
-  const int KW = p.kw, NS = kGemvConsumerWarps / KW;
-  const int TR = NS * R;
   const int SL = p.slab, NST = p.stages;
 
   // K range of this split, in 32-k chunks
@@ -202,28 +201,27 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
   const int nch = (int)((int64_t)(s + 1) * C / S - c0);
   const int nslab = (nch + SL - 1) / SL;
 
-  // tiles (TR rows) of this CTA
-  const int64_t tiles = (n + TR - 1) / TR;
-  const int64_t t_lo = (int64_t)blockIdx.x * tiles / gridDim.x;
-  const int64_t t_hi = (int64_t)(blockIdx.x + 1) * tiles / gridDim.x;
-  const int64_t Q = (t_hi - t_lo) * nslab;  // ring stages this CTA consumes
+  // rows of this CTA, walked in tiles of TR rows
+  const int64_t r_lo = (int64_t)blockIdx.x * n / gridDim.x;
+  const int64_t r_hi = (int64_t)(blockIdx.x + 1) * n / gridDim.x;
+  const int64_t ntile = (r_hi - r_lo + TR - 1) / TR;
+  const int64_t Q = ntile * nslab;  // ring stages this CTA consumes
 
   // shared memory carve-up (offsets computed on the host, 128-byte aligned)
   uint4* Ah4 = reinterpret_cast<uint4*>(smem);
   float* As = reinterpret_cast<float*>(smem + p.off_as);
-  float* comb = reinterpret_cast<float*>(smem + p.off_comb);  // [2][8 warps][R * MT]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   uint64_t* empty = full + NST;
   uint8_t* ring = smem + p.off_ring;
-  const int codes_stride = SL * 16;           // bytes per row of codes in a stage
+  const int codes_stride = SL * 16;                        // bytes per row of codes in a stage
   const int scales_stride = (int)gemv_scales_stride(SL);  // bytes per row of scales (16-byte multiple)
-  const int scales_off = TR * codes_stride;   // start of the scale rows in a stage
+  const int scales_off = TR * codes_stride;                // start of the scale rows in a stage
 
   if (tid == 0) {
     abort_flag = 0;
     for (int i = 0; i < NST; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kGemvConsumerWarps);
+      mbar_init(&empty[i], NC);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -237,22 +235,21 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
   if (producer) {
     // ------------------------------------------------------------------ producer warp
     int64_t issued = 0;
-    if (lane == 0 && !p.debug_stall) {
+    if (!p.debug_stall) {
       for (int64_t q = 0; q < Q; ++q) {
         const int slot = (int)(q % NST);
-        if (q >= NST && !mbar_wait_bounded(&empty[slot], (uint32_t)((q / NST - 1) & 1), &abort_flag,
-                                           p.timeout_ns, 2u))
-          break;
-        const int64_t tile = t_lo + q / nslab;
-        const int sb = (int)(q % nslab);
-        const int a = sb * SL;
+        bool ok = true;
+        if (lane == 0 && q >= NST)
+          ok = mbar_wait_bounded(&empty[slot], (uint32_t)((q / NST - 1) & 1), &abort_flag, p.timeout_ns, 2u);
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+        const int64_t j0 = r_lo + (q / nslab) * TR;
+        const int rows = (int)min((int64_t)TR, r_hi - j0);
+        const int a = (int)(q % nslab) * SL;
         const int len = min(SL, nch - a);
         uint8_t* stage = ring + (int64_t)slot * p.stage_bytes;
+        // each lane prepares its rows: bytes to expect, and the plain-copied scale tails
         uint32_t bytes = 0;
-        const int64_t j0 = tile * TR;
-        const int rows = (int)min((int64_t)TR, n - j0);
-        // plain-load tail first (only a scale superset that would overrun the tensor)
-        for (int r = 0; r < rows; ++r) {
+        for (int r = lane; r < rows; r += 32) {
           const int64_t st = (j0 + r) * rs_s + (c0 + a) * 2;
           const int64_t al = st & ~(int64_t)15;
           const int64_t ae = (st + (int64_t)len * 2 + 15) & ~(int64_t)15;
@@ -264,8 +261,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
           }
           bytes += (uint32_t)len * 16;
         }
-        mbar_arrive_expect_tx(&full[slot], bytes);
-        for (int r = 0; r < rows; ++r) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
+        __syncwarp();
+        for (int r = lane; r < rows; r += 32) {
           const int64_t j = j0 + r;
           bulk_g2s(stage + r * codes_stride, p.Wq + j * rs_q + (c0 + a) * 16, (uint32_t)len * 16, &full[slot]);
           const int64_t st = j * rs_s + (c0 + a) * 2;
@@ -277,43 +278,45 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
         issued = q + 1;
       }
       // drain: every copy this CTA issued must have landed before the CTA exits
-      const int64_t first = issued > NST ? issued - NST : 0;
-      for (int64_t q = first; q < issued; ++q)
-        mbar_wait_bounded(&full[q % NST], (uint32_t)((q / NST) & 1), &abort_flag, p.timeout_ns, 4u);
+      if (lane == 0) {
+        const int64_t first = issued > NST ? issued - NST : 0;
+        for (int64_t q = first; q < issued; ++q)
+          mbar_wait_bounded(&full[q % NST], (uint32_t)((q / NST) & 1), &abort_flag, p.timeout_ns, 4u);
+      }
     }
     return;
   }
 
   // -------------------------------------------------------------------- consumer warps
-  const int slot_id = warp / KW;
-  const int kw = warp - slot_id * KW;
   pdl_wait();
   const int GA = (nch + 31) / 32;
-  stage_activations(p.A, k, m, c0 * kChunkK, nch, Ah4, As, tid, kGemvConsumerWarps * 32);
-  named_barrier(1, kGemvConsumerWarps * 32);
+  stage_activations(p.A, k, m, c0 * kChunkK, nch, Ah4, As, tid, NC * 32);
+  named_barrier(1, NC * 32);
   const float g = (S == 1) ? *p.gscale : 1.0f;
 
   float acc[R][MT];
   int64_t q = 0;
-  for (int64_t tile = t_lo; tile < t_hi; ++tile) {
+  for (int64_t tile = 0; tile < ntile; ++tile) {
 #pragma unroll
     for (int i = 0; i < R; ++i)
 #pragma unroll
       for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
-    const int64_t j0 = tile * TR + slot_id * R;  // first row of this warp's slot
-    const int rows = (int)max((int64_t)0, min((int64_t)R, n - j0));
+    const int64_t j0 = r_lo + tile * TR + warp * R;  // first row of this warp
+    const int rows = (int)max((int64_t)0, min((int64_t)R, r_hi - j0));
     for (int sb = 0; sb < nslab; ++sb, ++q) {
       const int slot = (int)(q % NST);
       const bool ok = mbar_wait_bounded(&full[slot], (uint32_t)((q / NST) & 1), &abort_flag, p.timeout_ns, 1u);
       const int a = sb * SL;
       const int len = min(SL, nch - a);
-      if (ok) {
+      if (ok && rows > 0) {
         const uint8_t* stage = ring + (int64_t)slot * p.stage_bytes;
+        const uint8_t* crow = stage + warp * R * codes_stride;
+        const uint8_t* srow = stage + scales_off + warp * R * scales_stride;
         // scale superset offset of each of this warp's rows
         int soff[R];
 #pragma unroll
         for (int i = 0; i < R; ++i) soff[i] = (int)((((j0 + i) * rs_s) + (c0 + a) * 2) & 15);
-        for (int lc = 32 * kw + lane; lc < len; lc += 32 * KW) {
+        for (int lc = lane; lc < len; lc += 32) {
           const int c = a + lc;  // chunk inside the split
           // activations: 4 quads per activation row, and the two block scales
           const uint4* ap = Ah4 + ((int64_t)(c / 32) * 4) * 32 + (c % 32);
@@ -326,10 +329,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
 #pragma unroll
             for (int i = 0; i < R; ++i) {
               if (i < rows) {
-                const int rr = slot_id * R + i;
-                const uint4 cq = *reinterpret_cast<const uint4*>(stage + rr * codes_stride + lc * 16);
-                const uint32_t sc = *reinterpret_cast<const uint16_t*>(stage + scales_off + rr * scales_stride +
-                                                                       soff[i] + lc * 2);
+                const uint4 cq = *reinterpret_cast<const uint4*>(crow + i * codes_stride + lc * 16);
+                const uint32_t sc =
+                    *reinterpret_cast<const uint16_t*>(srow + i * scales_stride + soff[i] + lc * 2);
                 uint32_t wf[16];
                 decode32(cq, wf);
                 const float p0 = dot16(av, wf, 0.0f);
@@ -344,12 +346,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
             float sw[R][2];
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-              const int rr = slot_id * R + i;
               uint4 cq = make_uint4(0, 0, 0, 0);
               uint32_t sc = 0;
               if (i < rows) {
-                cq = *reinterpret_cast<const uint4*>(stage + rr * codes_stride + lc * 16);
-                sc = *reinterpret_cast<const uint16_t*>(stage + scales_off + rr * scales_stride + soff[i] + lc * 2);
+                cq = *reinterpret_cast<const uint4*>(crow + i * codes_stride + lc * 16);
+                sc = *reinterpret_cast<const uint16_t*>(srow + i * scales_stride + soff[i] + lc * 2);
               }
               decode32(cq, wf[i]);
               const uint32_t sh = e4m3x2_to_f16x2(sc);
@@ -379,7 +380,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
-    // the tile is done: lanes, then the slot's KW warps in order
+    // the rows are done: combine the lanes and write
 #pragma unroll
     for (int i = 0; i < R; ++i)
 #pragma unroll
@@ -389,28 +390,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         acc[i][r] = v;
       }
-    const int par = (int)((tile - t_lo) & 1);
-    if (KW > 1) {
-      float* mine = comb + ((par * kGemvConsumerWarps) + warp) * (R * MT);
-#pragma unroll
-      for (int i = 0; i < R; ++i)
-#pragma unroll
-        for (int r = 0; r < MT; ++r)
-          if (lane == ((i * MT + r) & 31)) mine[i * MT + r] = acc[i][r];
-      named_barrier(2 + slot_id, KW * 32);
-      if (kw == 0) {
-        const float* all = comb + (par * kGemvConsumerWarps + warp) * (R * MT);
-#pragma unroll
-        for (int i = 0; i < R; ++i)
-#pragma unroll
-          for (int r = 0; r < MT; ++r) {
-            float v = acc[i][r];
-            for (int w = 1; w < KW; ++w) v += all[w * (R * MT) + i * MT + r];
-            acc[i][r] = v;
-          }
-      }
-    }
-    if (kw == 0 && !abort_flag) {
+    if (!abort_flag) {
 #pragma unroll
       for (int i = 0; i < R; ++i)
 #pragma unroll

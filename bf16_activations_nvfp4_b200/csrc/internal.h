@@ -20,13 +20,13 @@ void clear_error();
 int device_sm_count();
 
 // ------------------------------------------------------------------------ GEMV
-constexpr int kGemvConsumerWarps = 8;                     // warps that decode and multiply
+constexpr int kGemvConsumerWarps = 16;                    // warps that decode and multiply
 constexpr int kGemvThreads = (kGemvConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kChunkK = 32;                                // k per lane per step (16 code bytes)
 constexpr int kGemvMaxM = 32;
 constexpr int kSmemBudget = 227 * 1024 - 1024;             // dynamic shared memory per CTA we allow
 constexpr int kGemvMaxStages = 8;
-constexpr int kGemvStageTarget = 32 * 1024;                // preferred bytes per ring stage
+constexpr int kGemvStageTarget = 24 * 1024;                // preferred bytes per ring stage
 
 // Activation rows the GEMV kernel instance for m is compiled for (1, 2, 4, ..., 32).
 inline int gemv_mt(int64_t m) {
@@ -44,8 +44,8 @@ __host__ __device__ inline int64_t gemv_scales_stride(int64_t slab) { return rou
 
 // Launch geometry of the GEMV for one shape and tactic (computed on the host).
 struct GemvGeometry {
-  int S, R, KW, TR, slab, stages, ctas_per_sm, grid_x;
-  int64_t stage_bytes, off_as, off_comb, off_bar, off_ring, smem_bytes;
+  int S, R, TR, slab, stages, ctas_per_sm, grid_x;
+  int64_t stage_bytes, off_as, off_bar, off_ring, smem_bytes;
 };
 // Returns FI_OK and fills g, or FI_ERR_UNSUPPORTED_SHAPE when the activations of m rows over
 // a split do not leave room for two ring stages in shared memory.
@@ -60,14 +60,13 @@ struct GemvArgs {
   float* partials;     // [splits, m, n] when splits > 1
   int64_t m, n, k;
   int splits;          // S: global K splits (grid.y)
-  int kw;              // KW: consumer warps sharing one row's k range
   int rows_per_warp;   // R
   int slab;            // SL: 32-k chunks per ring stage
   int stages;          // NST: ring stages
   int grid_x;          // CTAs per split
   int pdl;             // launch with programmatic stream serialization
   int debug_stall;     // test hook: the producer issues nothing (consumer waits time out)
-  int64_t stage_bytes, off_as, off_comb, off_bar, off_ring, smem_bytes;
+  int64_t stage_bytes, off_as, off_bar, off_ring, smem_bytes;
   uint64_t timeout_ns; // limit of every mbarrier wait
 };
 int launch_gemv(const GemvArgs& a, cudaStream_t stream);
