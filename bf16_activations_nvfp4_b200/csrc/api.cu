@@ -87,13 +87,10 @@ static int check_arch() {
 
 // Largest m the default table sends to the GEMV.
 constexpr int64_t kDefaultGemvMaxM = 32;
-// Rows per consumer warp when the tactic leaves it open.
-constexpr int kGemvDefaultRows = 2;
 
-int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int R, int ctas_per_sm, int sms, GemvGeometry* g) {
+int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_per_sm, int sms, GemvGeometry* g) {
   const int64_t C = k / kChunkK;
   const int64_t nch = (C + S - 1) / S;  // chunks of the largest split
-  const int TR = kGemvConsumerWarps * R;
   const int ctas = ctas_per_sm > 0 ? ctas_per_sm : 1;
   const int64_t per_cta = std::min<int64_t>(kSmemBudget, (228 * 1024) / ctas - 2048);
   const int64_t a_bytes = round_up(m * ((nch + 31) / 32) * 2048, 128);
@@ -101,17 +98,21 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int R, int ctas_per_sm
   const int64_t bar_bytes = round_up(2 * kGemvMaxStages * 8, 128);
   const int64_t fixed = a_bytes + as_bytes + bar_bytes;
   const int64_t avail = per_cta - fixed;
-  auto stage_of = [&](int64_t sl) { return round_up(TR * (sl * 16 + gemv_scales_stride(sl)), 128); };
-  // slab: whole split rows when a stage of them is small enough, else whole warp steps
-  const int64_t target = std::min<int64_t>(kGemvStageTarget, avail / 4);
-  int64_t slab;
-  if (stage_of(nch) <= target) {
-    slab = nch;
-  } else {
-    slab = 32;
-    while (slab + 32 < nch && stage_of(slab + 32) <= target) slab += 32;
+  // a stage: rs rows of codes, then their scales (one contiguous superset when S == 1, one
+  // superset per row otherwise), as the kernel lays them out
+  auto stage_of = [&](int64_t rs) {
+    const int64_t scales = S == 1 ? round_up(rs * nch * 2 + 30, 16) : rs * gemv_scales_stride(nch);
+    return round_up(rs * nch * 16 + scales, 128);
+  };
+  const int rmax = gemv_rows_per_stage_max(m);
+  int64_t rs = rs_req;
+  if (rs == 0) {
+    rs = 1;
+    while (rs < rmax && stage_of(rs + 1) <= kGemvStageTarget) ++rs;
   }
-  const int64_t stage_bytes = stage_of(slab);
+  if (rs < 1 || rs > rmax)
+    return set_error(FI_ERR_INVALID_ARG, "GEMV rows per stage must be 1..%d for m=%lld", rmax, (long long)m);
+  const int64_t stage_bytes = stage_of(rs);
   const int64_t stages = std::min<int64_t>(kGemvMaxStages, avail > 0 ? avail / stage_bytes : 0);
   if (stages < 2)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE,
@@ -121,9 +122,7 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int R, int ctas_per_sm
   int64_t gx = std::max<int64_t>(1, (int64_t)sms * ctas / S);
   if (gx > n) gx = std::max<int64_t>(1, n);
   g->S = S;
-  g->R = R;
-  g->TR = TR;
-  g->slab = (int)slab;
+  g->RS = (int)rs;
   g->stages = (int)stages;
   g->ctas_per_sm = ctas;
   g->grid_x = (int)gx;
@@ -138,12 +137,12 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int R, int ctas_per_sm
 // Device-sized split (PR #4038, "Sizes GEMV split-K from the device"): the fewest splits S
 // that give every SM a CTA with rows to stream while `m_fit` activation rows of a split fit
 // the shared-memory staging next to the weight ring. Depends on (n, k, SMs, R, m_fit) only.
-static int gemv_knee(int64_t n, int64_t k, int sms, int64_t m_fit, int R, int ctas, int* S_out) {
+static int gemv_knee(int64_t n, int64_t k, int sms, int64_t m_fit, int rs, int ctas, int* S_out) {
   const int64_t C = k / kChunkK;
   const int64_t maxS = std::max<int64_t>(1, std::min<int64_t>(C, 4095));
   for (int64_t S = 1; S <= maxS; ++S) {
     GemvGeometry g;
-    if (gemv_geometry(m_fit, n, k, (int)S, R, ctas, sms, &g) != FI_OK) continue;
+    if (gemv_geometry(m_fit, n, k, (int)S, rs, ctas, sms, &g) != FI_OK) continue;
     const bool enough = (int64_t)g.grid_x * S >= (int64_t)sms * g.ctas_per_sm;
     const bool last = S == maxS || (C / (S + 1)) < 32;  // a split keeps at least one warp step
     if (enough || last) {
@@ -162,32 +161,27 @@ static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms,
 static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms) {
   if (m <= kDefaultGemvMaxM) {
     const int64_t m_fit = m <= 1 ? 1 : (m <= 8 ? 8 : kGemvMaxM);
-    const int R = m_fit <= 4 ? kGemvDefaultRows : 1;  // keep register use within budget for larger m
     int S = 1;
-    if (gemv_knee(n, k, num_sms, m_fit, R, 1, &S) != FI_OK) S = 1;
-    return FI_TACTIC(FI_KIND_GEMV, S, 0, R);
+    if (gemv_knee(n, k, num_sms, m_fit, 0, 1, &S) != FI_OK) S = 1;
+    return FI_TACTIC(FI_KIND_GEMV, S, 0, 0);
   }
   return FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
 }
 
-// GEMV variant byte: R, the weight rows per consumer warp (1, 2 or 4; 0 = automatic).
-// Splits 0 = device-sized, resolved for m <= 32 so that the resolved S (and the bits) never
-// depend on m.
+// GEMV variant byte: rows per ring stage (consecutive weight rows one consumer warp
+// computes together; 0 = as many as fit the stage target). Splits 0 = device-sized, resolved
+// for m <= 32 so that the resolved S (and the bits) never depend on m.
 static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var,
                         int sms, fi_tactic_info* out) {
   if (m > kGemvMaxM)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV tactics support m <= %d (got m=%lld)",
                      kGemvMaxM, (long long)m);
-  const int R = var ? var : kGemvDefaultRows;
-  if (R != 1 && R != 2 && R != 4)
-    return set_error(FI_ERR_INVALID_ARG, "GEMV rows per warp must be 0 (auto), 1, 2 or 4");
-  if (R == 4 && m > 16)
-    return set_error(FI_ERR_INVALID_ARG, "GEMV with 4 rows per warp supports m <= 16");
   const int64_t C = k / kChunkK;
   const int ctas = ctas_req ? ctas_req : 1;
+  if (var < 0 || var > 8) return set_error(FI_ERR_INVALID_ARG, "GEMV rows per stage must be 0..8");
   int S = S_req;
   if (S == 0) {
-    const int rc = gemv_knee(n, k, sms, kGemvMaxM, R, ctas, &S);
+    const int rc = gemv_knee(n, k, sms, kGemvMaxM, 0, ctas, &S);
     if (rc != FI_OK) return rc;
   } else if (C > 0 && S > C) {
     return set_error(FI_ERR_INVALID_ARG, "splits=%lld exceeds k/32=%lld", (long long)S, (long long)C);
@@ -196,17 +190,17 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
   if (C == 0) {  // k == 0: nothing to stream; the caller writes zeros
     memset(&g, 0, sizeof(g));
     g.S = 1;
-    g.R = R;
+    g.RS = 1;
     g.ctas_per_sm = ctas;
     g.grid_x = 1;
   } else {
-    const int rc = gemv_geometry(m, n, k, S, R, ctas, sms, &g);
+    const int rc = gemv_geometry(m, n, k, S, var, ctas, sms, &g);
     if (rc != FI_OK) return rc;
   }
   out->kind = FI_KIND_GEMV;
   out->splits = g.S;
   out->ctas_per_sm = g.ctas_per_sm;
-  out->variant = R;
+  out->variant = g.RS;
   out->grid_x = g.grid_x;
   out->grid_y = g.S;
   out->threads = kGemvThreads;
@@ -355,8 +349,7 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.n = n;
     a.k = k;
     a.splits = g.S;
-    a.rows_per_warp = g.R;
-    a.slab = g.slab;
+    a.rows_per_stage = g.RS;
     a.stages = g.stages;
     a.grid_x = g.grid_x;
     a.pdl = 1;
@@ -444,12 +437,12 @@ int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, 
   clear_error();
   const int sms = sms_or_device(num_sms);
   if (sms <= 0) return set_error(FI_ERR_CUDA, "no device to query the SM count from");
-  // the split menu {1, 2, 4, 8, device-sized} for each rows-per-warp choice; entries
-  // resolving to the same launch are listed once
+  // the split menu {1, 2, 4, 8, device-sized}, each with the automatic stage size and with one
+  // and two rows per stage; entries resolving to the same launch are listed once
   int64_t cand[32];
   int nc = 0;
   const int splits[] = {1, 2, 4, 8, 0};
-  for (int R : {1, 2, 4})
+  for (int R : {0, 1, 2})
     for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, R);
   fi_tactic_info seen[32];
   int nseen = 0, count = 0;

@@ -5,24 +5,26 @@
 // "A-in-SMEM staging"), re-designed for B200, where an m=1 GEMV has to keep ~100 KB of
 // weights in flight per SM to run at HBM speed:
 //
-//  * Warp specialisation. One producer warp per CTA streams weight tiles HBM -> shared memory
+//  * Warp specialisation. One producer warp per CTA streams weight rows HBM -> shared memory
 //    with bulk asynchronous copies (cp.async.bulk, completion counted on an mbarrier) into an
 //    NST-stage ring; 16 consumer warps decode from shared memory. In-flight bytes live in
-//    shared memory, not registers; the producer's 32 lanes issue the copies of up to 32 rows
-//    at once.
+//    shared memory, not registers, and few large copies (a stage is ~16 KB) keep the copy
+//    engine's per-copy cost out of the way.
 //  * Programmatic dependent launch. The producer issues the first NST stages before the
 //    grid-dependency wait (weights are never written by the preceding kernel); the consumers
 //    wait, then stage the activations, so the weight stream overlaps the previous kernel's
 //    tail and the activation staging.
 //  * Work. Grid (G, S): blockIdx.y is the K split s; the G CTAs of a split own balanced,
-//    contiguous ranges of weight rows (so every SM streams the same number of bytes, +-1 row)
-//    and walk them in tiles of TR = 16 * R rows; consumer warp w owns rows w*R .. w*R+R-1 of a
-//    tile. A tile's rows are fetched in slabs of SL 32-k chunks (one ring stage per slab): one
-//    bulk copy per row for the codes and one per row for the E4M3 scales (a 16-byte-aligned
-//    superset of the row's scale bytes, indexed from the remainder; a superset that would
-//    overrun the scale tensor is copied with plain loads instead).
-//  * Arithmetic (fixed by k and S alone, hence bitwise identical for every m, R, SL, NST, G
-//    and CTAs per SM): A is staged as f16 with one power-of-two scale per 16-block (exact for
+//    contiguous ranges of weight rows (every SM streams the same bytes, +-1 row). A ring stage
+//    holds RS consecutive rows over the split's whole k range, and consumer warp w processes
+//    stages w, w+16, w+32, ... of its CTA, so a row is always computed by one warp and the
+//    activations it loads once per step serve all RS rows. With one split a stage is two bulk
+//    copies: the rows' contiguous codes and a 16-byte-aligned superset of their contiguous
+//    E4M3 scales (indexed from the remainder; where the superset would overrun the scale
+//    tensor the producer copies the scales with plain loads). With S > 1 each row's slice is
+//    copied on its own.
+//  * Arithmetic (fixed by k and S alone, hence bitwise identical for every m, RS, NST, G and
+//    CTAs per SM): A is staged as f16 with one power-of-two scale per 16-block (exact for
 //    every element within 2^28 of its block maximum); codes are decoded by
 //    cvt.rn.f16x2.e2m1x2 (exact) and multiplied by the mixed-precision fma.rn.f32.f16 (exact
 //    product, fp32 accumulate). Lane L takes chunks L, L+32, L+64, ... of the split: per
@@ -178,13 +180,12 @@ __device__ __forceinline__ void decode32(const uint4 q, uint32_t* wf) {
 
 }  // namespace
 
-template <int MT, int R>
+template <int MT, int RMAX>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ volatile int abort_flag;
 
   constexpr int NC = kGemvConsumerWarps;
-  constexpr int TR = NC * R;  // rows per tile
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
@@ -193,19 +194,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
   const int64_t n = p.n, k = p.k;
   const int S = p.splits;
   const int s = blockIdx.y;
-  const int SL = p.slab, NST = p.stages;
+  const int RS = p.rows_per_stage, NST = p.stages;
 
   // K range of this split, in 32-k chunks
   const int64_t C = k / kChunkK;
   const int64_t c0 = (int64_t)s * C / S;
   const int nch = (int)((int64_t)(s + 1) * C / S - c0);
-  const int nslab = (nch + SL - 1) / SL;
 
-  // rows of this CTA, walked in tiles of TR rows
+  // rows of this CTA, RS per ring stage
   const int64_t r_lo = (int64_t)blockIdx.x * n / gridDim.x;
   const int64_t r_hi = (int64_t)(blockIdx.x + 1) * n / gridDim.x;
-  const int64_t ntile = (r_hi - r_lo + TR - 1) / TR;
-  const int64_t Q = ntile * nslab;  // ring stages this CTA consumes
+  const int64_t Q = (r_hi - r_lo + RS - 1) / RS;  // ring stages of this CTA
 
   // shared memory carve-up (offsets computed on the host, 128-byte aligned)
   uint4* Ah4 = reinterpret_cast<uint4*>(smem);
@@ -213,15 +212,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   uint64_t* empty = full + NST;
   uint8_t* ring = smem + p.off_ring;
-  const int codes_stride = SL * 16;                        // bytes per row of codes in a stage
-  const int scales_stride = (int)gemv_scales_stride(SL);  // bytes per row of scales (16-byte multiple)
-  const int scales_off = TR * codes_stride;                // start of the scale rows in a stage
+  const int codes_stride = nch * 16;  // bytes per row of codes in a stage (rows are adjacent)
+  const int scales_off = RS * codes_stride;
+  // S == 1: one contiguous superset of the rows' scales; S > 1: one superset per row
+  const int scales_stride = (int)gemv_scales_stride(nch);
 
   if (tid == 0) {
     abort_flag = 0;
     for (int i = 0; i < NST; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], NC);
+      mbar_init(&empty[i], 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -234,55 +234,59 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
 
   if (producer) {
     // ------------------------------------------------------------------ producer warp
-    int64_t issued = 0;
-    if (!p.debug_stall) {
+    if (lane == 0 && !p.debug_stall) {
+      int64_t issued = 0;
       for (int64_t q = 0; q < Q; ++q) {
         const int slot = (int)(q % NST);
-        bool ok = true;
-        if (lane == 0 && q >= NST)
-          ok = mbar_wait_bounded(&empty[slot], (uint32_t)((q / NST - 1) & 1), &abort_flag, p.timeout_ns, 2u);
-        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-        const int64_t j0 = r_lo + (q / nslab) * TR;
-        const int rows = (int)min((int64_t)TR, r_hi - j0);
-        const int a = (int)(q % nslab) * SL;
-        const int len = min(SL, nch - a);
+        if (q >= NST && !mbar_wait_bounded(&empty[slot], (uint32_t)((q / NST - 1) & 1), &abort_flag,
+                                           p.timeout_ns, 2u))
+          break;
+        const int64_t j0 = r_lo + q * RS;
+        const int rows = (int)min((int64_t)RS, r_hi - j0);
         uint8_t* stage = ring + (int64_t)slot * p.stage_bytes;
-        // each lane prepares its rows: bytes to expect, and the plain-copied scale tails
-        uint32_t bytes = 0;
-        for (int r = lane; r < rows; r += 32) {
-          const int64_t st = (j0 + r) * rs_s + (c0 + a) * 2;
-          const int64_t al = st & ~(int64_t)15;
-          const int64_t ae = (st + (int64_t)len * 2 + 15) & ~(int64_t)15;
-          if (ae > scale_bytes_total) {
-            uint8_t* dst = stage + scales_off + r * scales_stride;
-            for (int64_t b = al; b < st + (int64_t)len * 2; ++b) dst[b - al] = p.Ws[b];
+        uint8_t* sdst = stage + scales_off;
+        if (S == 1) {
+          const int64_t st = j0 * rs_s, en = (j0 + rows) * rs_s;
+          const int64_t al = st & ~(int64_t)15, ae = (en + 15) & ~(int64_t)15;
+          uint32_t bytes = (uint32_t)(rows * rs_q);
+          const bool plain = ae > scale_bytes_total;
+          if (plain) {
+            for (int64_t b = al; b < en; ++b) sdst[b - al] = p.Ws[b];
           } else {
             bytes += (uint32_t)(ae - al);
           }
-          bytes += (uint32_t)len * 16;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-        __syncwarp();
-        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
-        __syncwarp();
-        for (int r = lane; r < rows; r += 32) {
-          const int64_t j = j0 + r;
-          bulk_g2s(stage + r * codes_stride, p.Wq + j * rs_q + (c0 + a) * 16, (uint32_t)len * 16, &full[slot]);
-          const int64_t st = j * rs_s + (c0 + a) * 2;
-          const int64_t al = st & ~(int64_t)15;
-          const int64_t ae = (st + (int64_t)len * 2 + 15) & ~(int64_t)15;
-          if (ae <= scale_bytes_total)
-            bulk_g2s(stage + scales_off + r * scales_stride, p.Ws + al, (uint32_t)(ae - al), &full[slot]);
+          mbar_arrive_expect_tx(&full[slot], bytes);
+          bulk_g2s(stage, p.Wq + j0 * rs_q, (uint32_t)(rows * rs_q), &full[slot]);
+          if (!plain) bulk_g2s(sdst, p.Ws + al, (uint32_t)(ae - al), &full[slot]);
+        } else {
+          uint32_t bytes = 0;
+          for (int r = 0; r < rows; ++r) {
+            const int64_t st = (j0 + r) * rs_s + c0 * 2;
+            const int64_t al = st & ~(int64_t)15, ae = (st + (int64_t)nch * 2 + 15) & ~(int64_t)15;
+            if (ae > scale_bytes_total) {
+              uint8_t* dst = sdst + r * scales_stride;
+              for (int64_t b = al; b < st + (int64_t)nch * 2; ++b) dst[b - al] = p.Ws[b];
+            } else {
+              bytes += (uint32_t)(ae - al);
+            }
+            bytes += (uint32_t)nch * 16;
+          }
+          mbar_arrive_expect_tx(&full[slot], bytes);
+          for (int r = 0; r < rows; ++r) {
+            const int64_t j = j0 + r;
+            bulk_g2s(stage + r * codes_stride, p.Wq + j * rs_q + c0 * 16, (uint32_t)nch * 16, &full[slot]);
+            const int64_t st = j * rs_s + c0 * 2;
+            const int64_t al = st & ~(int64_t)15, ae = (st + (int64_t)nch * 2 + 15) & ~(int64_t)15;
+            if (ae <= scale_bytes_total)
+              bulk_g2s(sdst + r * scales_stride, p.Ws + al, (uint32_t)(ae - al), &full[slot]);
+          }
         }
         issued = q + 1;
       }
       // drain: every copy this CTA issued must have landed before the CTA exits
-      if (lane == 0) {
-        const int64_t first = issued > NST ? issued - NST : 0;
-        for (int64_t q = first; q < issued; ++q)
-          mbar_wait_bounded(&full[q % NST], (uint32_t)((q / NST) & 1), &abort_flag, p.timeout_ns, 4u);
-      }
+      const int64_t first = issued > NST ? issued - NST : 0;
+      for (int64_t q = first; q < issued; ++q)
+        mbar_wait_bounded(&full[q % NST], (uint32_t)((q / NST) & 1), &abort_flag, p.timeout_ns, 4u);
     }
     return;
   }
@@ -294,95 +298,83 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
   named_barrier(1, NC * 32);
   const float g = (S == 1) ? *p.gscale : 1.0f;
 
-  float acc[R][MT];
-  int64_t q = 0;
-  for (int64_t tile = 0; tile < ntile; ++tile) {
+  for (int64_t q = warp; q < Q; q += NC) {
+    const int slot = (int)(q % NST);
+    const bool ok = mbar_wait_bounded(&full[slot], (uint32_t)((q / NST) & 1), &abort_flag, p.timeout_ns, 1u);
+    const int64_t j0 = r_lo + q * RS;
+    const int rows = (int)min((int64_t)RS, r_hi - j0);
+    float acc[RMAX][MT];
 #pragma unroll
-    for (int i = 0; i < R; ++i)
+    for (int i = 0; i < RMAX; ++i)
 #pragma unroll
       for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
-    const int64_t j0 = r_lo + tile * TR + warp * R;  // first row of this warp
-    const int rows = (int)max((int64_t)0, min((int64_t)R, r_hi - j0));
-    for (int sb = 0; sb < nslab; ++sb, ++q) {
-      const int slot = (int)(q % NST);
-      const bool ok = mbar_wait_bounded(&full[slot], (uint32_t)((q / NST) & 1), &abort_flag, p.timeout_ns, 1u);
-      const int a = sb * SL;
-      const int len = min(SL, nch - a);
-      if (ok && rows > 0) {
-        const uint8_t* stage = ring + (int64_t)slot * p.stage_bytes;
-        const uint8_t* crow = stage + warp * R * codes_stride;
-        const uint8_t* srow = stage + scales_off + warp * R * scales_stride;
-        // scale superset offset of each of this warp's rows
-        int soff[R];
+    if (ok) {
+      const uint8_t* stage = ring + (int64_t)slot * p.stage_bytes;
+      // where row i's scales start in the stage
+      int sbase[RMAX];
 #pragma unroll
-        for (int i = 0; i < R; ++i) soff[i] = (int)((((j0 + i) * rs_s) + (c0 + a) * 2) & 15);
-        for (int lc = lane; lc < len; lc += 32) {
-          const int c = a + lc;  // chunk inside the split
-          // activations: 4 quads per activation row, and the two block scales
-          const uint4* ap = Ah4 + ((int64_t)(c / 32) * 4) * 32 + (c % 32);
-          const float2* sp = reinterpret_cast<const float2*>(As) + c;
-          if (MT == 1) {
-            const uint4 a0 = ap[0], a1 = ap[32], a2 = ap[64], a3 = ap[96];
-            const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
-                                     a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-            const float2 sa = sp[0];
+      for (int i = 0; i < RMAX; ++i) {
+        if (S == 1)
+          sbase[i] = scales_off + (int)((j0 * rs_s) & 15) + i * (int)rs_s;
+        else
+          sbase[i] = scales_off + i * scales_stride + (int)(((j0 + i) * rs_s + c0 * 2) & 15);
+      }
+      for (int c = lane; c < nch; c += 32) {
+        const uint4* ap = Ah4 + ((int64_t)(c / 32) * 4) * 32 + (c % 32);
+        const float2* sp = reinterpret_cast<const float2*>(As) + c;
+        if (MT == 1) {
+          const uint4 a0 = ap[0], a1 = ap[32], a2 = ap[64], a3 = ap[96];
+          const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                                   a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+          const float2 sa = sp[0];
 #pragma unroll
-            for (int i = 0; i < R; ++i) {
-              if (i < rows) {
-                const uint4 cq = *reinterpret_cast<const uint4*>(crow + i * codes_stride + lc * 16);
-                const uint32_t sc =
-                    *reinterpret_cast<const uint16_t*>(srow + i * scales_stride + soff[i] + lc * 2);
-                uint32_t wf[16];
-                decode32(cq, wf);
-                const float p0 = dot16(av, wf, 0.0f);
-                const float p1 = dot16(av + 8, wf + 8, 0.0f);
-                const uint32_t sh = e4m3x2_to_f16x2(sc);
-                acc[i][0] = fmaf(p0, f16_lo_to_f32(sh) * sa.x, acc[i][0]);
-                acc[i][0] = fmaf(p1, f16_hi_to_f32(sh) * sa.y, acc[i][0]);
-              }
-            }
-          } else {
-            uint32_t wf[R][16];
-            float sw[R][2];
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
-              uint4 cq = make_uint4(0, 0, 0, 0);
-              uint32_t sc = 0;
-              if (i < rows) {
-                cq = *reinterpret_cast<const uint4*>(crow + i * codes_stride + lc * 16);
-                sc = *reinterpret_cast<const uint16_t*>(srow + i * scales_stride + soff[i] + lc * 2);
-              }
-              decode32(cq, wf[i]);
+          for (int i = 0; i < RMAX; ++i) {
+            if (i < rows) {
+              const uint4 cq = *reinterpret_cast<const uint4*>(stage + i * codes_stride + c * 16);
+              const uint32_t sc = *reinterpret_cast<const uint16_t*>(stage + sbase[i] + c * 2);
+              uint32_t wf[16];
+              decode32(cq, wf);
+              const float p0 = dot16(av, wf, 0.0f);
+              const float p1 = dot16(av + 8, wf + 8, 0.0f);
               const uint32_t sh = e4m3x2_to_f16x2(sc);
-              sw[i][0] = f16_lo_to_f32(sh);
-              sw[i][1] = f16_hi_to_f32(sh);
+              acc[i][0] = fmaf(p0, f16_lo_to_f32(sh) * sa.x, acc[i][0]);
+              acc[i][0] = fmaf(p1, f16_hi_to_f32(sh) * sa.y, acc[i][0]);
             }
+          }
+        } else {
 #pragma unroll
-            for (int r = 0; r < MT; ++r) {
-              if (r < m) {
-                const uint4* apr = ap + (int64_t)r * GA * 4 * 32;
-                const uint4 a0 = apr[0], a1 = apr[32], a2 = apr[64], a3 = apr[96];
-                const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
-                                         a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-                const float2 sa = sp[(int64_t)r * nch];
+          for (int i = 0; i < RMAX; ++i) {
+            if (i < rows) {
+              const uint4 cq = *reinterpret_cast<const uint4*>(stage + i * codes_stride + c * 16);
+              const uint32_t sc = *reinterpret_cast<const uint16_t*>(stage + sbase[i] + c * 2);
+              uint32_t wf[16];
+              decode32(cq, wf);
+              const uint32_t sh = e4m3x2_to_f16x2(sc);
+              const float sw0 = f16_lo_to_f32(sh), sw1 = f16_hi_to_f32(sh);
 #pragma unroll
-                for (int i = 0; i < R; ++i) {
-                  const float p0 = dot16(av, wf[i], 0.0f);
-                  const float p1 = dot16(av + 8, wf[i] + 8, 0.0f);
-                  acc[i][r] = fmaf(p0, sw[i][0] * sa.x, acc[i][r]);
-                  acc[i][r] = fmaf(p1, sw[i][1] * sa.y, acc[i][r]);
+              for (int r = 0; r < MT; ++r) {
+                if (r < m) {
+                  const uint4* apr = ap + (int64_t)r * GA * 4 * 32;
+                  const uint4 a0 = apr[0], a1 = apr[32], a2 = apr[64], a3 = apr[96];
+                  const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                                           a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+                  const float2 sa = sp[(int64_t)r * nch];
+                  const float p0 = dot16(av, wf, 0.0f);
+                  const float p1 = dot16(av + 8, wf + 8, 0.0f);
+                  acc[i][r] = fmaf(p0, sw0 * sa.x, acc[i][r]);
+                  acc[i][r] = fmaf(p1, sw1 * sa.y, acc[i][r]);
                 }
               }
             }
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
     }
-    // the rows are done: combine the lanes and write
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+    // the stage's rows are done: combine the lanes and write
 #pragma unroll
-    for (int i = 0; i < R; ++i)
+    for (int i = 0; i < RMAX; ++i)
 #pragma unroll
       for (int r = 0; r < MT; ++r) {
         float v = acc[i][r];
@@ -390,9 +382,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         acc[i][r] = v;
       }
-    if (!abort_flag) {
+    if (ok && !abort_flag) {
 #pragma unroll
-      for (int i = 0; i < R; ++i)
+      for (int i = 0; i < RMAX; ++i)
 #pragma unroll
         for (int r = 0; r < MT; ++r)
           if (i < rows && r < m && lane == ((i * MT + r) & 31)) {
@@ -408,9 +400,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
 
 namespace {
 
-template <int MT, int R>
+template <int MT, int RMAX>
 int launch_one(const GemvArgs& a, cudaStream_t stream) {
-  auto kern = gemv_nvfp4_kernel<MT, R>;
+  auto kern = gemv_nvfp4_kernel<MT, RMAX>;
   // the opt-in shared memory limit is a per-device function attribute; raise it once
   static int configured[kMaxDevices] = {};
   int dev = 0;
@@ -435,27 +427,19 @@ int launch_one(const GemvArgs& a, cudaStream_t stream) {
   return FI_OK;
 }
 
-template <int MT>
-int launch_rows(const GemvArgs& a, cudaStream_t stream) {
-  switch (a.rows_per_warp) {
-    case 1: return launch_one<MT, 1>(a, stream);
-    case 2: return launch_one<MT, 2>(a, stream);
-    case 4:
-      if constexpr (MT <= 16) return launch_one<MT, 4>(a, stream);
-      return set_error(FI_ERR_INVALID_ARG, "GEMV with 4 rows per warp supports m <= 16");
-    default: return set_error(FI_ERR_INVALID_ARG, "GEMV rows per warp must be 1, 2 or 4");
-  }
-}
-
 }  // namespace
 
+int gemv_rows_per_stage_max(int64_t m) { return gemv_rmax(gemv_mt(m)); }
+
 int launch_gemv(const GemvArgs& a, cudaStream_t stream) {
-  if (a.m <= 1) return launch_rows<1>(a, stream);
-  if (a.m <= 2) return launch_rows<2>(a, stream);
-  if (a.m <= 4) return launch_rows<4>(a, stream);
-  if (a.m <= 8) return launch_rows<8>(a, stream);
-  if (a.m <= 16) return launch_rows<16>(a, stream);
-  if (a.m <= 32) return launch_rows<32>(a, stream);
+  if (a.rows_per_stage < 1 || a.rows_per_stage > gemv_rows_per_stage_max(a.m))
+    return set_error(FI_ERR_INVALID_ARG, "GEMV rows per stage out of range");
+  if (a.m <= 1) return launch_one<1, gemv_rmax(1)>(a, stream);
+  if (a.m <= 2) return launch_one<2, gemv_rmax(2)>(a, stream);
+  if (a.m <= 4) return launch_one<4, gemv_rmax(4)>(a, stream);
+  if (a.m <= 8) return launch_one<8, gemv_rmax(8)>(a, stream);
+  if (a.m <= 16) return launch_one<16, gemv_rmax(16)>(a, stream);
+  if (a.m <= 32) return launch_one<32, gemv_rmax(32)>(a, stream);
   return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV supports m <= %d", kGemvMaxM);
 }
 

@@ -25,8 +25,8 @@ constexpr int kGemvThreads = (kGemvConsumerWarps + 1) * 32;  // + one producer w
 constexpr int kChunkK = 32;                                // k per lane per step (16 code bytes)
 constexpr int kGemvMaxM = 32;
 constexpr int kSmemBudget = 227 * 1024 - 1024;             // dynamic shared memory per CTA we allow
-constexpr int kGemvMaxStages = 8;
-constexpr int kGemvStageTarget = 24 * 1024;                // preferred bytes per ring stage
+constexpr int kGemvMaxStages = 16;
+constexpr int kGemvStageTarget = 16 * 1024;                // preferred bytes per ring stage
 
 // Activation rows the GEMV kernel instance for m is compiled for (1, 2, 4, ..., 32).
 inline int gemv_mt(int64_t m) {
@@ -42,14 +42,20 @@ __host__ __device__ inline int64_t round_up(int64_t x, int64_t a) { return (x + 
 // by the host's shared-memory layout and the kernel, so both always agree.
 __host__ __device__ inline int64_t gemv_scales_stride(int64_t slab) { return round_up(slab * 2 + 28, 16); }
 
+// Most weight rows a ring stage holds for the kernel instance of MT activation rows (bounded
+// by the accumulator registers, RMAX * MT <= 16).
+__host__ __device__ constexpr int gemv_rmax(int mt) { return mt >= 16 ? 1 : (16 / mt > 8 ? 8 : 16 / mt); }
+int gemv_rows_per_stage_max(int64_t m);
+
 // Launch geometry of the GEMV for one shape and tactic (computed on the host).
 struct GemvGeometry {
-  int S, R, TR, slab, stages, ctas_per_sm, grid_x;
+  int S, RS, stages, ctas_per_sm, grid_x;
   int64_t stage_bytes, off_as, off_bar, off_ring, smem_bytes;
 };
 // Returns FI_OK and fills g, or FI_ERR_UNSUPPORTED_SHAPE when the activations of m rows over
-// a split do not leave room for two ring stages in shared memory.
-int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int R, int ctas_per_sm, int sms, GemvGeometry* g);
+// a split leave no room for two ring stages of one weight row in shared memory. rs_req is
+// the requested rows per stage (0 = as many as fit the stage target).
+int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_per_sm, int sms, GemvGeometry* g);
 
 struct GemvArgs {
   const uint16_t* A;
@@ -60,8 +66,7 @@ struct GemvArgs {
   float* partials;     // [splits, m, n] when splits > 1
   int64_t m, n, k;
   int splits;          // S: global K splits (grid.y)
-  int rows_per_warp;   // R
-  int slab;            // SL: 32-k chunks per ring stage
+  int rows_per_stage;  // RS: consecutive weight rows per ring stage (one consumer warp each)
   int stages;          // NST: ring stages
   int grid_x;          // CTAs per split
   int pdl;             // launch with programmatic stream serialization

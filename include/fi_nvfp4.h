@@ -66,7 +66,8 @@ typedef enum {
  *                (PR #4038, "Sizes GEMV split-K from the device");
  *   ctas_per_sm  co-resident CTAs per SM used to size the grid (1..15); 0 = automatic
  *                (PR #4038, "Adds occupancy tactics");
- *   variant      GEMV: weight rows per consumer warp (1, 2 or 4; 0 = automatic). MMA: 0.
+ *   variant      GEMV: weight rows per pipeline stage, computed together by one warp
+ *                (1..8, at most 16 / m rounded to a power of two; 0 = automatic). MMA: 0.
  * Only `kind` and the resolved S change the arithmetic: two tactics with the same kind
  * and S give bitwise identical outputs, and for a fixed tactic every output row is
  * bitwise independent of m. FI_TACTIC_DEFAULT (-1) selects from the built-in per-shape

@@ -49,7 +49,7 @@ def test_default_gemv_tactic_resolves_for_decode_shapes(n, k):
     assert 1 <= info["splits"] <= k // 32
     # one persistent wave: the grid never asks for more CTAs than the SMs hold
     assert info["grid_x"] * info["grid_y"] <= B200_SMS * info["ctas_per_sm"]
-    assert info["threads"] == 9 * 32 and 0 < info["smem_bytes"] <= 227 * 1024
+    assert info["threads"] == 17 * 32 and 0 < info["smem_bytes"] <= 227 * 1024
     assert info["workspace_bytes"] == (info["splits"] * n * 4 if info["splits"] > 1 else 0)
 
 
@@ -57,7 +57,7 @@ def test_device_sized_split_is_m_independent():
     """The device-sized tactic (splits=0) resolves to the same S for every m the GEMV takes,
     and gives every SM a CTA unless the k range cannot be divided further."""
     for n, k in [(512, 2048), (1024, 4096), (4096, 14336), (14336, 4096), (2048, 7168), (10304, 2688)]:
-        for R in (1, 2):
+        for R in (0, 1):
             t = fi.make_tactic(fi.KIND_GEMV, 0, 0, R)
             got = {fi.resolve_tactic(m, n, k, t, B200_SMS)["splits"] for m in (1, 2, 3, 8, 16, 32)}
             assert len(got) == 1, (n, k, R, got)
@@ -102,14 +102,15 @@ def test_workspace_bytes():
 @pytest.mark.parametrize("m,n,k,tactic,status", [
     (1, 64, 48, -1, -2),                                  # k % 32 != 0
     (33, 64, 64, fi.make_tactic(0, 1, 0, 1), -2),         # GEMV beyond m = 32
-    (1, 64, 64, fi.make_tactic(0, 1, 0, 3), -1),          # rows per warp 3
+    (1, 64, 64, fi.make_tactic(0, 1, 0, 9), -1),          # rows per stage 9
     (1, 64, 64, fi.make_tactic(0, 3, 0, 1), -1),          # splits > k/32
     (1, 64, 64, fi.make_tactic(7, 1, 0, 1), -1),          # unknown kind
     (1, 64, 64, 1 << 30, -1),                             # out-of-range code
     (-1, 64, 64, -1, -1),                                 # negative size
     (32, 64, 14336, fi.make_tactic(0, 1, 0, 1), -2),      # A slice does not fit shared memory
-    (32, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),       # 4 rows per warp only up to m = 16
-    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x12), -1),     # rows per warp 18
+    (32, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),       # one row per stage above m = 8
+    (5, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),        # two rows per stage above m = 4
+    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x12), -1),     # rows per stage 18
 ])
 def test_resolve_rejects(m, n, k, tactic, status):
     with pytest.raises(fi.FiError) as e:
