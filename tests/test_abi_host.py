@@ -111,6 +111,7 @@ def test_workspace_bytes():
     (32, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),       # one row per stage above m = 8
     (5, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),        # two rows per stage above m = 4
     (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x12), -1),     # rows per stage 18
+    (1, 8, 65536, fi.make_tactic(0, 1, 0, 2), -2),        # two 36 KB rows per stage do not fit twice
 ])
 def test_resolve_rejects(m, n, k, tactic, status):
     with pytest.raises(fi.FiError) as e:

@@ -153,7 +153,7 @@ def test_multi_slab_rows_and_many_splits():
         W, (Wq, Ws, g) = _gpu.weights(n, k, 3)
         ref = oracle.mm(A, Wq, Ws, g)
         dw = _gpu.device_weights(n, k, 3)
-        for R in (1, 2):
+        for R in (0, 1):  # one 32 KB row per stage is what fits next to A at k = 65536
             _gpu.assert_within_tolerance(_mm(A, dw, fi.make_tactic(GEMV, S, 0, R)), ref, f"{m}x{n}x{k} S={S} R={R}")
 
 
