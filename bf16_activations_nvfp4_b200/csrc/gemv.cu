@@ -16,9 +16,10 @@
 //    tail and the activation staging.
 //  * Work. Grid (G, S): blockIdx.y is the K split s; the G CTAs of a split own balanced,
 //    contiguous ranges of weight rows (every SM streams the same bytes, +-1 row). A ring stage
-//    holds RS consecutive rows over the split's whole k range, and consumer warp w processes
-//    stages w, w+16, w+32, ... of its CTA, so a row is always computed by one warp and the
-//    activations it loads once per step serve all RS rows. With one split a stage is two bulk
+//    holds RS consecutive rows over the split's whole k range, and consumer warp w computes
+//    stages w, w+16, w+32, ... of its CTA (every warp waits on and releases every stage, so a
+//    slot never runs more than one mbarrier phase ahead of a waiter), so a row is always
+//    computed by one warp and the activations it loads once per step serve all RS rows. With one split a stage is two bulk
 //    copies: the rows' contiguous codes and a 16-byte-aligned superset of their contiguous
 //    E4M3 scales (indexed from the remainder; where the superset would overrun the scale
 //    tensor the producer copies the scales with plain loads). With S > 1 each row's slice is
@@ -221,7 +222,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
     abort_flag = 0;
     for (int i = 0; i < NST; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], NC);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -298,9 +299,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
   named_barrier(1, NC * 32);
   const float g = (S == 1) ? *p.gscale : 1.0f;
 
-  for (int64_t q = warp; q < Q; q += NC) {
+  // Every consumer warp passes every stage in order and releases it (the empty barrier counts
+  // all NC warps), but only warp q % NC computes stage q. A slot therefore never runs more than
+  // one phase ahead of any warp waiting on it, which the parity-based waits require.
+  for (int64_t q = 0; q < Q; ++q) {
     const int slot = (int)(q % NST);
     const bool ok = mbar_wait_bounded(&full[slot], (uint32_t)((q / NST) & 1), &abort_flag, p.timeout_ns, 1u);
+    if (q % NC != warp) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      continue;
+    }
     const int64_t j0 = r_lo + q * RS;
     const int rows = (int)min((int64_t)RS, r_hi - j0);
     float acc[RMAX][MT];
