@@ -108,10 +108,11 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_p
   int64_t rs = rs_req;
   if (rs == 0) {
     rs = 1;
-    while (rs < rmax && stage_of(rs + 1) <= kGemvStageTarget) ++rs;
+    while (rs * 2 <= rmax && stage_of(rs * 2) <= kGemvStageTarget) rs *= 2;
   }
-  if (rs < 1 || rs > rmax)
-    return set_error(FI_ERR_INVALID_ARG, "GEMV rows per stage must be 1..%d for m=%lld", rmax, (long long)m);
+  if (rs < 1 || rs > rmax || (rs & (rs - 1)) != 0)
+    return set_error(FI_ERR_INVALID_ARG, "GEMV rows per stage must be a power of two in 1..%d for m=%lld", rmax,
+                     (long long)m);
   const int64_t stage_bytes = stage_of(rs);
   const int64_t stages = std::min<int64_t>(kGemvMaxStages, avail > 0 ? avail / stage_bytes : 0);
   if (stages < 2)
@@ -178,7 +179,7 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
                      kGemvMaxM, (long long)m);
   const int64_t C = k / kChunkK;
   const int ctas = ctas_req ? ctas_req : 1;
-  if (var < 0 || var > 8) return set_error(FI_ERR_INVALID_ARG, "GEMV rows per stage must be 0..8");
+  if (var < 0 || var > 8) return set_error(FI_ERR_INVALID_ARG, "GEMV rows per stage must be 0, 1, 2, 4 or 8");
   int S = S_req;
   if (S == 0) {
     const int rc = gemv_knee(n, k, sms, kGemvMaxM, 0, ctas, &S);

@@ -179,9 +179,92 @@ __device__ __forceinline__ void decode32(const uint4 q, uint32_t* wf) {
   }
 }
 
+// NR weight rows of a ring stage against MT activation rows: lane L takes chunks L, L+32, ...
+// of the split; the activations loaded for a chunk serve all NR rows. codes[i] / scales[i]
+// point at row i's codes and E4M3 scales in shared memory; acc[i][r] accumulates in fp32.
+template <int MT, int NR>
+__device__ __forceinline__ void stage_rows(const uint8_t* const* codes, const uint8_t* const* scales,
+                                           const uint4* __restrict__ Ah4, const float* __restrict__ As,
+                                           int m, int nch, int GA, int lane, float (&acc)[NR][MT]) {
+  for (int c = lane; c < nch; c += 32) {
+    const uint4* ap = Ah4 + ((int64_t)(c / 32) * 4) * 32 + (c % 32);
+    const float2* sp = reinterpret_cast<const float2*>(As) + c;
+    if (MT == 1) {
+      const uint4 a0 = ap[0], a1 = ap[32], a2 = ap[64], a3 = ap[96];
+      const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                               a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+      const float2 sa = sp[0];
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        const uint4 cq = *reinterpret_cast<const uint4*>(codes[i] + c * 16);
+        const uint32_t sc = *reinterpret_cast<const uint16_t*>(scales[i] + c * 2);
+        uint32_t wf[16];
+        decode32(cq, wf);
+        const float p0 = dot16(av, wf, 0.0f);
+        const float p1 = dot16(av + 8, wf + 8, 0.0f);
+        const uint32_t sh = e4m3x2_to_f16x2(sc);
+        acc[i][0] = fmaf(p0, f16_lo_to_f32(sh) * sa.x, acc[i][0]);
+        acc[i][0] = fmaf(p1, f16_hi_to_f32(sh) * sa.y, acc[i][0]);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        const uint4 cq = *reinterpret_cast<const uint4*>(codes[i] + c * 16);
+        const uint32_t sc = *reinterpret_cast<const uint16_t*>(scales[i] + c * 2);
+        uint32_t wf[16];
+        decode32(cq, wf);
+        const uint32_t sh = e4m3x2_to_f16x2(sc);
+        const float sw0 = f16_lo_to_f32(sh), sw1 = f16_hi_to_f32(sh);
+#pragma unroll
+        for (int r = 0; r < MT; ++r) {
+          if (r < m) {
+            const uint4* apr = ap + (int64_t)r * GA * 4 * 32;
+            const uint4 a0 = apr[0], a1 = apr[32], a2 = apr[64], a3 = apr[96];
+            const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                                     a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+            const float2 sa = sp[(int64_t)r * nch];
+            const float p0 = dot16(av, wf, 0.0f);
+            const float p1 = dot16(av + 8, wf + 8, 0.0f);
+            acc[i][r] = fmaf(p0, sw0 * sa.x, acc[i][r]);
+            acc[i][r] = fmaf(p1, sw1 * sa.y, acc[i][r]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// Combine the lanes of acc (fixed xor butterfly: every lane ends with the same bits) and
+// write rows j0 .. j0+NR-1: bf16_rn(acc * g) when S == 1, else the fp32 partial of split s.
+template <int MT, int NR>
+__device__ __forceinline__ void finish_rows(float (&acc)[NR][MT], const GemvArgs& p, int64_t j0, int m, int S,
+                                            int s, float g, int lane, bool write) {
+#pragma unroll
+  for (int i = 0; i < NR; ++i)
+#pragma unroll
+    for (int r = 0; r < MT; ++r) {
+      float v = acc[i][r];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      acc[i][r] = v;
+    }
+  if (!write) return;
+#pragma unroll
+  for (int i = 0; i < NR; ++i)
+#pragma unroll
+    for (int r = 0; r < MT; ++r)
+      if (r < m && lane == ((i * MT + r) & 31)) {
+        const int64_t j = j0 + i;
+        if (S == 1)
+          p.out[(int64_t)r * p.n + j] = f32_to_bf16_rn(acc[i][r] * g);
+        else
+          p.partials[((int64_t)s * m + r) * p.n + j] = acc[i][r];
+      }
+}
+
 }  // namespace
 
-template <int MT, int RMAX>
+template <int MT, int RS>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ volatile int abort_flag;
@@ -195,7 +278,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
   const int64_t n = p.n, k = p.k;
   const int S = p.splits;
   const int s = blockIdx.y;
-  const int RS = p.rows_per_stage, NST = p.stages;
+  const int NST = p.stages;
 
   // K range of this split, in 32-k chunks
   const int64_t C = k / kChunkK;
@@ -312,106 +395,45 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
     }
     const int64_t j0 = r_lo + q * RS;
     const int rows = (int)min((int64_t)RS, r_hi - j0);
-    float acc[RMAX][MT];
+    const uint8_t* stage = ring + (int64_t)slot * p.stage_bytes;
+    // where row i's codes and scales start in the stage
+    const uint8_t* cptr[RS];
+    const uint8_t* sptr[RS];
 #pragma unroll
-    for (int i = 0; i < RMAX; ++i)
+    for (int i = 0; i < RS; ++i) {
+      cptr[i] = stage + i * codes_stride;
+      sptr[i] = S == 1 ? stage + scales_off + (int)((j0 * rs_s) & 15) + i * (int)rs_s
+                       : stage + scales_off + i * scales_stride + (int)(((j0 + i) * rs_s + c0 * 2) & 15);
+    }
+    const bool write = ok && !abort_flag;
+    if (rows == RS) {
+      float acc[RS][MT];
 #pragma unroll
-      for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
-    if (ok) {
-      const uint8_t* stage = ring + (int64_t)slot * p.stage_bytes;
-      // where row i's scales start in the stage
-      int sbase[RMAX];
+      for (int i = 0; i < RS; ++i)
 #pragma unroll
-      for (int i = 0; i < RMAX; ++i) {
-        if (S == 1)
-          sbase[i] = scales_off + (int)((j0 * rs_s) & 15) + i * (int)rs_s;
-        else
-          sbase[i] = scales_off + i * scales_stride + (int)(((j0 + i) * rs_s + c0 * 2) & 15);
-      }
-      for (int c = lane; c < nch; c += 32) {
-        const uint4* ap = Ah4 + ((int64_t)(c / 32) * 4) * 32 + (c % 32);
-        const float2* sp = reinterpret_cast<const float2*>(As) + c;
-        if (MT == 1) {
-          const uint4 a0 = ap[0], a1 = ap[32], a2 = ap[64], a3 = ap[96];
-          const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
-                                   a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-          const float2 sa = sp[0];
+        for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
+      if (ok) stage_rows<MT, RS>(cptr, sptr, Ah4, As, m, nch, GA, lane, acc);
+      finish_rows<MT, RS>(acc, p, j0, m, S, s, g, lane, write);
+    } else {
+      // the CTA's last, partial stage: one row at a time
+      for (int i = 0; i < rows; ++i) {
+        float acc[1][MT];
 #pragma unroll
-          for (int i = 0; i < RMAX; ++i) {
-            if (i < rows) {
-              const uint4 cq = *reinterpret_cast<const uint4*>(stage + i * codes_stride + c * 16);
-              const uint32_t sc = *reinterpret_cast<const uint16_t*>(stage + sbase[i] + c * 2);
-              uint32_t wf[16];
-              decode32(cq, wf);
-              const float p0 = dot16(av, wf, 0.0f);
-              const float p1 = dot16(av + 8, wf + 8, 0.0f);
-              const uint32_t sh = e4m3x2_to_f16x2(sc);
-              acc[i][0] = fmaf(p0, f16_lo_to_f32(sh) * sa.x, acc[i][0]);
-              acc[i][0] = fmaf(p1, f16_hi_to_f32(sh) * sa.y, acc[i][0]);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < RMAX; ++i) {
-            if (i < rows) {
-              const uint4 cq = *reinterpret_cast<const uint4*>(stage + i * codes_stride + c * 16);
-              const uint32_t sc = *reinterpret_cast<const uint16_t*>(stage + sbase[i] + c * 2);
-              uint32_t wf[16];
-              decode32(cq, wf);
-              const uint32_t sh = e4m3x2_to_f16x2(sc);
-              const float sw0 = f16_lo_to_f32(sh), sw1 = f16_hi_to_f32(sh);
-#pragma unroll
-              for (int r = 0; r < MT; ++r) {
-                if (r < m) {
-                  const uint4* apr = ap + (int64_t)r * GA * 4 * 32;
-                  const uint4 a0 = apr[0], a1 = apr[32], a2 = apr[64], a3 = apr[96];
-                  const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
-                                           a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-                  const float2 sa = sp[(int64_t)r * nch];
-                  const float p0 = dot16(av, wf, 0.0f);
-                  const float p1 = dot16(av + 8, wf + 8, 0.0f);
-                  acc[i][r] = fmaf(p0, sw0 * sa.x, acc[i][r]);
-                  acc[i][r] = fmaf(p1, sw1 * sa.y, acc[i][r]);
-                }
-              }
-            }
-          }
-        }
+        for (int r = 0; r < MT; ++r) acc[0][r] = 0.0f;
+        if (ok) stage_rows<MT, 1>(cptr + i, sptr + i, Ah4, As, m, nch, GA, lane, acc);
+        finish_rows<MT, 1>(acc, p, j0 + i, m, S, s, g, lane, write);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
-    // the stage's rows are done: combine the lanes and write
-#pragma unroll
-    for (int i = 0; i < RMAX; ++i)
-#pragma unroll
-      for (int r = 0; r < MT; ++r) {
-        float v = acc[i][r];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        acc[i][r] = v;
-      }
-    if (ok && !abort_flag) {
-#pragma unroll
-      for (int i = 0; i < RMAX; ++i)
-#pragma unroll
-        for (int r = 0; r < MT; ++r)
-          if (i < rows && r < m && lane == ((i * MT + r) & 31)) {
-            const int64_t j = j0 + i;
-            if (S == 1)
-              p.out[(int64_t)r * n + j] = f32_to_bf16_rn(acc[i][r] * g);
-            else
-              p.partials[((int64_t)s * m + r) * n + j] = acc[i][r];
-          }
-    }
   }
 }
 
 namespace {
 
-template <int MT, int RMAX>
+template <int MT, int RS>
 int launch_one(const GemvArgs& a, cudaStream_t stream) {
-  auto kern = gemv_nvfp4_kernel<MT, RMAX>;
+  auto kern = gemv_nvfp4_kernel<MT, RS>;
   // the opt-in shared memory limit is a per-device function attribute; raise it once
   static int configured[kMaxDevices] = {};
   int dev = 0;
@@ -436,19 +458,36 @@ int launch_one(const GemvArgs& a, cudaStream_t stream) {
   return FI_OK;
 }
 
+template <int MT>
+int launch_rs(const GemvArgs& a, cudaStream_t stream) {
+  switch (a.rows_per_stage) {
+    case 1: return launch_one<MT, 1>(a, stream);
+    case 2:
+      if constexpr (gemv_rmax(MT) >= 2) return launch_one<MT, 2>(a, stream);
+      break;
+    case 4:
+      if constexpr (gemv_rmax(MT) >= 4) return launch_one<MT, 4>(a, stream);
+      break;
+    case 8:
+      if constexpr (gemv_rmax(MT) >= 8) return launch_one<MT, 8>(a, stream);
+      break;
+    default: break;
+  }
+  return set_error(FI_ERR_INVALID_ARG, "GEMV rows per stage %d is not available for m=%lld", a.rows_per_stage,
+                   (long long)a.m);
+}
+
 }  // namespace
 
 int gemv_rows_per_stage_max(int64_t m) { return gemv_rmax(gemv_mt(m)); }
 
 int launch_gemv(const GemvArgs& a, cudaStream_t stream) {
-  if (a.rows_per_stage < 1 || a.rows_per_stage > gemv_rows_per_stage_max(a.m))
-    return set_error(FI_ERR_INVALID_ARG, "GEMV rows per stage out of range");
-  if (a.m <= 1) return launch_one<1, gemv_rmax(1)>(a, stream);
-  if (a.m <= 2) return launch_one<2, gemv_rmax(2)>(a, stream);
-  if (a.m <= 4) return launch_one<4, gemv_rmax(4)>(a, stream);
-  if (a.m <= 8) return launch_one<8, gemv_rmax(8)>(a, stream);
-  if (a.m <= 16) return launch_one<16, gemv_rmax(16)>(a, stream);
-  if (a.m <= 32) return launch_one<32, gemv_rmax(32)>(a, stream);
+  if (a.m <= 1) return launch_rs<1>(a, stream);
+  if (a.m <= 2) return launch_rs<2>(a, stream);
+  if (a.m <= 4) return launch_rs<4>(a, stream);
+  if (a.m <= 8) return launch_rs<8>(a, stream);
+  if (a.m <= 16) return launch_rs<16>(a, stream);
+  if (a.m <= 32) return launch_rs<32>(a, stream);
   return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV supports m <= %d", kGemvMaxM);
 }
 

@@ -67,7 +67,8 @@ typedef enum {
  *   ctas_per_sm  co-resident CTAs per SM used to size the grid (1..15); 0 = automatic
  *                (PR #4038, "Adds occupancy tactics");
  *   variant      GEMV: weight rows per pipeline stage, computed together by one warp
- *                (1..8, at most 16 / m rounded to a power of two; 0 = automatic). MMA: 0.
+ *                (1, 2, 4 or 8, at most 16 / m rounded to a power of two; 0 = automatic).
+ *                MMA: 0.
  * Only `kind` and the resolved S change the arithmetic: two tactics with the same kind
  * and S give bitwise identical outputs, and for a fixed tactic every output row is
  * bitwise independent of m. FI_TACTIC_DEFAULT (-1) selects from the built-in per-shape

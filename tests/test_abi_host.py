@@ -103,6 +103,7 @@ def test_workspace_bytes():
     (1, 64, 48, -1, -2),                                  # k % 32 != 0
     (33, 64, 64, fi.make_tactic(0, 1, 0, 1), -2),         # GEMV beyond m = 32
     (1, 64, 64, fi.make_tactic(0, 1, 0, 9), -1),          # rows per stage 9
+    (1, 64, 64, fi.make_tactic(0, 1, 0, 3), -1),          # rows per stage not a power of two
     (1, 64, 64, fi.make_tactic(0, 3, 0, 1), -1),          # splits > k/32
     (1, 64, 64, fi.make_tactic(7, 1, 0, 1), -1),          # unknown kind
     (1, 64, 64, 1 << 30, -1),                             # out-of-range code
