@@ -71,12 +71,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// One bounded, suspending test of the phase: the thread sleeps in hardware until the phase
+// completes or kWaitSliceNs pass, so waiting warps do not spin on the issue slots the
+// computing warps need.
+constexpr uint32_t kWaitSliceNs = 20000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
       : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(kWaitSliceNs)
       : "memory");
   return done != 0;
 }
@@ -85,19 +89,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // the device error bit) if it has not after timeout_ns, or at once if the CTA has aborted.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                   uint64_t timeout_ns, unsigned err_bit) {
-  uint64_t t0 = 0;
-  for (uint32_t it = 0;; ++it) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if ((it & 63) == 63) {
-      const uint64_t now = globaltimer_ns();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > timeout_ns) {
-        *abort_flag = 1;
-        atomicOr(&g_gemv_error, err_bit);
-        return false;
-      }
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      *abort_flag = 1;
+      atomicOr(&g_gemv_error, err_bit);
+      return false;
     }
   }
 }
