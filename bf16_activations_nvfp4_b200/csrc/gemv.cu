@@ -110,6 +110,24 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -180,24 +198,32 @@ __device__ __forceinline__ void decode32(const uint4 q, uint32_t* wf) {
 }
 
 // NR weight rows of a ring stage against MT activation rows: lane L takes chunks L, L+32, ...
-// of the split; the activations loaded for a chunk serve all NR rows. codes[i] / scales[i]
-// point at row i's codes and E4M3 scales in shared memory; acc[i][r] accumulates in fp32.
+// of the split; the activations loaded for a chunk serve all NR rows. Row i's codes start at
+// shared address code0 + i * cstride and its E4M3 scales at sbase + i * sstride + ((off0 + i *
+// doff) & 15) (the scales sit at their source offset within 16-byte aligned copies); a_s / as_s
+// are the shared addresses of the staged activations and their scales; acc[i][r] accumulates
+// in fp32.
 template <int MT, int NR>
-__device__ __forceinline__ void stage_rows(const uint8_t* const* codes, const uint8_t* const* scales,
-                                           const uint4* __restrict__ Ah4, const float* __restrict__ As,
-                                           int m, int nch, int GA, int lane, float (&acc)[NR][MT]) {
+__device__ __forceinline__ void stage_rows(uint32_t code0, int cstride, uint32_t sbase, int sstride, uint32_t off0,
+                                           uint32_t doff, uint32_t a_s, uint32_t as_s, int m, int nch, int GA,
+                                           int lane, float (&acc)[NR][MT]) {
+  const uint32_t a_row = (uint32_t)GA * 4 * 32 * 16;  // bytes per activation row
+  const uint32_t as_row = (uint32_t)nch * 8;
+  uint32_t scale0[NR];
+#pragma unroll
+  for (int i = 0; i < NR; ++i) scale0[i] = sbase + (uint32_t)(i * sstride) + ((off0 + (uint32_t)i * doff) & 15u);
   for (int c = lane; c < nch; c += 32) {
-    const uint4* ap = Ah4 + ((int64_t)(c / 32) * 4) * 32 + (c % 32);
-    const float2* sp = reinterpret_cast<const float2*>(As) + c;
+    const uint32_t ap = a_s + (uint32_t)(((c >> 5) * 4 * 32 + (c & 31)) * 16);
+    const uint32_t sp = as_s + (uint32_t)c * 8;
     if (MT == 1) {
-      const uint4 a0 = ap[0], a1 = ap[32], a2 = ap[64], a3 = ap[96];
+      const uint4 a0 = lds_v4(ap), a1 = lds_v4(ap + 512), a2 = lds_v4(ap + 1024), a3 = lds_v4(ap + 1536);
       const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
                                a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-      const float2 sa = sp[0];
+      const float2 sa = lds_f2(sp);
 #pragma unroll
       for (int i = 0; i < NR; ++i) {
-        const uint4 cq = *reinterpret_cast<const uint4*>(codes[i] + c * 16);
-        const uint32_t sc = *reinterpret_cast<const uint16_t*>(scales[i] + c * 2);
+        const uint4 cq = lds_v4(code0 + (uint32_t)(i * cstride + c * 16));
+        const uint32_t sc = lds_u16(scale0[i] + (uint32_t)(c * 2));
         uint32_t wf[16];
         decode32(cq, wf);
         const float p0 = dot16(av, wf, 0.0f);
@@ -209,8 +235,8 @@ __device__ __forceinline__ void stage_rows(const uint8_t* const* codes, const ui
     } else {
 #pragma unroll
       for (int i = 0; i < NR; ++i) {
-        const uint4 cq = *reinterpret_cast<const uint4*>(codes[i] + c * 16);
-        const uint32_t sc = *reinterpret_cast<const uint16_t*>(scales[i] + c * 2);
+        const uint4 cq = lds_v4(code0 + (uint32_t)(i * cstride + c * 16));
+        const uint32_t sc = lds_u16(scale0[i] + (uint32_t)(c * 2));
         uint32_t wf[16];
         decode32(cq, wf);
         const uint32_t sh = e4m3x2_to_f16x2(sc);
@@ -218,11 +244,11 @@ __device__ __forceinline__ void stage_rows(const uint8_t* const* codes, const ui
 #pragma unroll
         for (int r = 0; r < MT; ++r) {
           if (r < m) {
-            const uint4* apr = ap + (int64_t)r * GA * 4 * 32;
-            const uint4 a0 = apr[0], a1 = apr[32], a2 = apr[64], a3 = apr[96];
+            const uint32_t apr = ap + (uint32_t)r * a_row;
+            const uint4 a0 = lds_v4(apr), a1 = lds_v4(apr + 512), a2 = lds_v4(apr + 1024), a3 = lds_v4(apr + 1536);
             const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
                                      a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-            const float2 sa = sp[(int64_t)r * nch];
+            const float2 sa = lds_f2(sp + (uint32_t)r * as_row);
             const float p0 = dot16(av, wf, 0.0f);
             const float p1 = dot16(av + 8, wf + 8, 0.0f);
             acc[i][r] = fmaf(p0, sw0 * sa.x, acc[i][r]);
@@ -296,6 +322,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   uint64_t* empty = full + NST;
   uint8_t* ring = smem + p.off_ring;
+  const uint32_t ring_s = smem_addr(ring), a_s = smem_addr(Ah4), as_s = smem_addr(As);
   const int codes_stride = nch * 16;  // bytes per row of codes in a stage (rows are adjacent)
   const int scales_off = RS * codes_stride;
   // S == 1: one contiguous superset of the rows' scales; S > 1: one superset per row
@@ -395,16 +422,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
     }
     const int64_t j0 = r_lo + q * RS;
     const int rows = (int)min((int64_t)RS, r_hi - j0);
-    const uint8_t* stage = ring + (int64_t)slot * p.stage_bytes;
-    // where row i's codes and scales start in the stage
-    const uint8_t* cptr[RS];
-    const uint8_t* sptr[RS];
-#pragma unroll
-    for (int i = 0; i < RS; ++i) {
-      cptr[i] = stage + i * codes_stride;
-      sptr[i] = S == 1 ? stage + scales_off + (int)((j0 * rs_s) & 15) + i * (int)rs_s
-                       : stage + scales_off + i * scales_stride + (int)(((j0 + i) * rs_s + c0 * 2) & 15);
-    }
+    const uint32_t stage_s = ring_s + (uint32_t)slot * (uint32_t)p.stage_bytes;
+    // row i's scales: S == 1 copies the rows' contiguous scales as one aligned superset (stride
+    // k/16); S > 1 copies an aligned superset per row (stride scales_stride). Either way row i's
+    // scales sit at offset ((j0 + i) * k/16 + c0 * 2) & 15 within its part of the stage.
+    const uint32_t sbase = stage_s + (uint32_t)scales_off;
+    const int sstride = S == 1 ? (int)rs_s : scales_stride;
+    const uint32_t off0 = (uint32_t)((j0 * rs_s + c0 * 2) & 15);
+    const uint32_t doff = S == 1 ? 0u : (uint32_t)(rs_s & 15);
     const bool write = ok && !abort_flag;
     if (rows == RS) {
       float acc[RS][MT];
@@ -412,7 +437,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
       for (int i = 0; i < RS; ++i)
 #pragma unroll
         for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
-      if (ok) stage_rows<MT, RS>(cptr, sptr, Ah4, As, m, nch, GA, lane, acc);
+      if (ok)
+        stage_rows<MT, RS>(stage_s, codes_stride, sbase, sstride, off0, doff, a_s, as_s, m, nch, GA, lane, acc);
       finish_rows<MT, RS>(acc, p, j0, m, S, s, g, lane, write);
     } else {
       // the CTA's last, partial stage: one row at a time
@@ -420,7 +446,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
         float acc[1][MT];
 #pragma unroll
         for (int r = 0; r < MT; ++r) acc[0][r] = 0.0f;
-        if (ok) stage_rows<MT, 1>(cptr + i, sptr + i, Ah4, As, m, nch, GA, lane, acc);
+        if (ok)
+          stage_rows<MT, 1>(stage_s + (uint32_t)(i * codes_stride), codes_stride,
+                            sbase + (uint32_t)(i * sstride) + ((off0 + (uint32_t)i * doff) & 15u), 0, 0u, 0u,
+                            a_s, as_s, m, nch, GA, lane, acc);
         finish_rows<MT, 1>(acc, p, j0 + i, m, S, s, g, lane, write);
       }
     }
