@@ -135,7 +135,7 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_p
   return FI_OK;
 }
 
-// Device-sized split (PR #4038, "Sizes GEMV split-K from the device"): the fewest splits S
+// Device-sized split (PR #4038, Description, "What it does": the device-sized GEMV split): the fewest splits S
 // that give every SM a CTA with rows to stream while `m_fit` activation rows of a split fit
 // the shared-memory staging next to the weight ring. Depends on (n, k, SMs, R, m_fit) only.
 static int gemv_knee(int64_t n, int64_t k, int sms, int64_t m_fit, int rs, int ctas, int* S_out) {

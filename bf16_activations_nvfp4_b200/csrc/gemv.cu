@@ -1,9 +1,10 @@
 // Streaming GEMV for bf16 activations x NVFP4 weights, m <= 32 (sm_100a).
 //
-// After PR #4038's streaming GEMV ("weights stream from global memory ... latency hidden by
-// warp count", "one output row per warp, warp-shuffle reduction", the v2 commit's
-// "A-in-SMEM staging"), re-designed for B200, where an m=1 GEMV has to keep ~100 KB of
-// weights in flight per SM to run at HBM speed:
+// After the streaming GEMV of PR #4038 (Description, "What it does", and its GEMV commit
+// messages: weights go from global memory straight to registers with many warps covering
+// the latency, each output row is reduced across a warp with shuffles, and a later commit
+// stages the activations in shared memory), re-designed for B200, where an m=1 GEMV has to
+// keep ~100 KB of weights in flight per SM to run at HBM speed:
 //
 //  * Warp specialisation. One producer warp per CTA streams weight rows HBM -> shared memory
 //    with bulk asynchronous copies (cp.async.bulk, completion counted on an mbarrier) into an

@@ -1,5 +1,6 @@
-// Fixed-order split-K reduction (PR #4038: "Splits write fp32 partials, and a PDL-chained
-// reduce kernel sums them in fixed order, so results are deterministic run to run").
+// Fixed-order split-K reduction (PR #4038, Description, "What it does": the split-K item;
+// each split leaves an fp32 partial and a second, PDL-chained kernel adds the partials in
+// one fixed order, which makes the result repeat bit for bit from run to run).
 //
 //   out[e] = bf16_rn( (((p[0][e] + p[1][e]) + p[2][e]) + ...) * gscale )   all fp32
 //

@@ -11,18 +11,18 @@
  * Split-K tactics write fp32 partials that a second kernel sums in a fixed order, so
  * results are bitwise deterministic run to run (PR #4038, "What it does"); within one
  * tactic a row's bits do not depend on m (the batch-invariant property of the FlashInfer
- * v0.7.4 article, "Why identical bits matter").
+ * v0.7.4 article, in its section on why identical bits matter).
  *
  * Conventions for every entry point
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library never frees
  *    or retains them beyond the call. Calls are asynchronous on `stream` (NULL = legacy
  *    default stream) and never synchronise the host.
  *  - bf16 tensors are passed as uint16_t bit patterns; layouts are row-major, dense.
- *  - NVFP4 layout ("canonical", PR #4038 GEMV commit: "(N, K/2) packed layout + linear
- *    E4M3 scales"): Wq is uint8 [n, k/2], byte j of a row holds code 2j in bits 0-3 and
- *    code 2j+1 in bits 4-7; Wscale is uint8 [n, k/16] of E4M3 codes, row-major (linear,
- *    unswizzled); gscale points to one fp32 in device memory (so calls can be captured in
- *    a CUDA graph without a host read).
+ *  - NVFP4 layout (the canonical one of PR #4038's GEMV commit message: packed
+ *    [N, K/2] codes with linear E4M3 scales): Wq is uint8 [n, k/2], byte j of a row holds
+ *    code 2j in bits 0-3 and code 2j+1 in bits 4-7; Wscale is uint8 [n, k/16] of E4M3
+ *    codes, row-major (linear, unswizzled); gscale points to one fp32 in device memory (so
+ *    calls can be captured in a CUDA graph without a host read).
  *  - Return value: FI_OK (0) or a negative fi_status. On error nothing was launched and a
  *    message is available from fi_last_error() (thread-local). A CUDA launch failure
  *    returns FI_ERR_CUDA after other work of the same call may already be queued.
@@ -63,18 +63,18 @@ typedef enum {
  *                tensor-core GEMM, 1 <= m <= 256);
  *   splits       number of K partitions S (1..4095); 0 = device-sized ("knee") split:
  *                the smallest S that gives the device enough concurrent weight streams
- *                (PR #4038, "Sizes GEMV split-K from the device");
+ *                (PR #4038, Description, "What it does": the device-sized GEMV split);
  *   ctas_per_sm  co-resident CTAs per SM used to size the grid (1..15); 0 = automatic
- *                (PR #4038, "Adds occupancy tactics");
+ *                (PR #4038, Description, "What it does": occupancy tactics);
  *   variant      GEMV: weight rows per pipeline stage, computed together by one warp
  *                (1, 2, 4 or 8, at most 16 / m rounded to a power of two; 0 = automatic).
  *                MMA: 0.
  * Only `kind` and the resolved S change the arithmetic: two tactics with the same kind
  * and S give bitwise identical outputs, and for a fixed tactic every output row is
  * bitwise independent of m. FI_TACTIC_DEFAULT (-1) selects from the built-in per-shape
- * table (PR #4038, "Routes the no-autotune m=1 fallback onto the GEMV"); the table's
- * choice of kind and S depends on m, so the default is batch-invariant only within the
- * m range of one table entry.
+ * table (PR #4038, Description, "What it does": the untuned m=1 route to the GEMV); the
+ * table's choice of kind and S depends on m, so the default is batch-invariant only
+ * within the m range of one table entry.
  */
 #define FI_KIND_GEMV 0
 #define FI_KIND_MMA 1
@@ -155,8 +155,8 @@ FI_API int fi_mm_bf16_fp4_ex(const uint16_t* A, const uint8_t* Wq, const uint8_t
                       fi_stream_t stream);
 
 /*
- * Fixed-order split-K reduction (PR #4038, "a PDL-chained reduce kernel sums them in
- * fixed order"): for every element e of [m, n],
+ * Fixed-order split-K reduction (PR #4038, Description, "What it does": the split-K item):
+ * for every element e of [m, n],
  *     s = ((p[0][e] + p[1][e]) + p[2][e]) + ...   (fp32, s = 0 .. splits-1 in order)
  *     out[e] = bf16_rn(s * gscale[0])             (fp32 product)
  *   partials  device fp32 [splits, m, n], 16-byte aligned.

@@ -9,7 +9,7 @@
  *  - "perf(gemm): split-K, occupancy, and m=1 stream-GEMV decode tactics for mm_bf16_fp4"
  *    (flashinfer PR #4038), Description: the op multiplies bf16 activations by nvfp4
  *    weights; the GEMV commit message: weights come in the canonical (N, K/2) packed layout
- *    with "linear" (row-major, unswizzled) E4M3 scales, one per 16 k.
+ *    with linear (row-major, unswizzled) E4M3 scales, one per 16 k.
  *  - The NVFP4 quantisation recipe this library targets: per 16-k block scale = block
  *    amax / 6 rounded to E4M3, global scale = tensor amax / (448 * 6), E2M1 codes packed two
  *    per byte. The pages name the format but not the recipe.
