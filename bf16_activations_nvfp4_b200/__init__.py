@@ -78,6 +78,7 @@ def library() -> ctypes.CDLL:
         lib.fi_nvfp4_pack_weights.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         lib.fi_mm_bf16_fp4.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
         lib.fi_mm_bf16_fp4_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp]
+        lib.fi_mm_bf16_fp4_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
         lib.fi_splitk_reduce.argtypes = [vp, i64, i64, i64, vp, vp, vp]
         lib.fi_resolve_tactic.argtypes = [i64, i64, i64, i64, ctypes.c_int, ctypes.POINTER(TacticInfo)]
         lib.fi_default_tactic.argtypes = [i64, i64, i64, ctypes.c_int]
@@ -91,7 +92,8 @@ def library() -> ctypes.CDLL:
         lib.fi_version.argtypes = []
         lib.fi_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         lib.fi_debug_set.argtypes = [ctypes.c_int, i64]
-        for name in ("fi_nvfp4_pack_weights", "fi_mm_bf16_fp4", "fi_mm_bf16_fp4_ex", "fi_splitk_reduce",
+        for name in ("fi_nvfp4_pack_weights", "fi_mm_bf16_fp4", "fi_mm_bf16_fp4_ex", "fi_mm_bf16_fp4_noalloc",
+                     "fi_splitk_reduce",
                      "fi_resolve_tactic", "fi_list_tactics", "fi_set_workspace", "fi_version",
                      "fi_get_device_error", "fi_debug_set"):
             getattr(lib, name).restype = ctypes.c_int

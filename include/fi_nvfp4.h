@@ -155,6 +155,33 @@ FI_API int fi_mm_bf16_fp4_ex(const uint16_t* A, const uint8_t* Wq, const uint8_t
                       fi_stream_t stream);
 
 /*
+ * fi_mm_bf16_fp4 without any device allocation. The paper has no counterpart: this entry
+ * point exists for users of this library who may not allocate GPU memory at call time, such
+ * as an operator plugin inside a serving engine that has already reserved the device's memory
+ * for weights and the KV cache, or a component whose memory plan is fixed at start-up and
+ * that owns no buffer it could pass to fi_mm_bf16_fp4_ex. fi_mm_bf16_fp4 would cudaMalloc its
+ * split-K workspace on first use; this variant keeps the fp32 partials in a static device
+ * array compiled into the library instead: FI_NOALLOC_SCRATCH_BYTES (4 MiB) on every GPU that
+ * loads the library, held until the process exits.
+ * Arguments, tactics, preconditions and results are those of fi_mm_bf16_fp4.
+ * Limit: the resolved tactic's fi_mm_workspace_bytes() (4 * splits * m * n) must not exceed
+ * FI_NOALLOC_SCRATCH_BYTES; a larger call returns FI_ERR_WORKSPACE and launches nothing.
+ * Single-split tactics use no scratch.
+ * Set-up: the first call on a device that reaches a launch looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first call before any
+ * stream capture begins.
+ * Sharing: all calls on a device use the same array, and it keeps the last call's partials.
+ * Nothing in it needs to start at zero (each split writes all of its partials before the
+ * reduce reads them), but calls whose kernels can overlap on the GPU (different streams,
+ * parallel graph branches) race on it and must be serialised by the caller.
+ * Never calls cudaMalloc, cudaFree or any other allocating routine.
+ */
+#define FI_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+FI_API int fi_mm_bf16_fp4_noalloc(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale,
+                           const float* gscale, uint16_t* out, int64_t m, int64_t n, int64_t k,
+                           int64_t tactic, fi_stream_t stream);
+
+/*
  * Fixed-order split-K reduction (PR #4038, Description, "What it does": the split-K item):
  * for every element e of [m, n],
  *     s = ((p[0][e] + p[1][e]) + p[2][e]) + ...   (fp32, s = 0 .. splits-1 in order)

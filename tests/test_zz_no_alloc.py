@@ -1,0 +1,88 @@
+"""fi_mm_bf16_fp4_noalloc, the entry point for callers that may not allocate GPU memory.
+
+An operator plugin running inside an engine that has already reserved the device's memory
+(or any caller with a memory plan fixed at start-up) cannot let the library cudaMalloc a
+split-K workspace, and may own no buffer to lend it either. fi_mm_bf16_fp4_noalloc keeps the
+split-K partials in a static device array of the library instead. These tests call it
+through the C ABI and hold it to the allocating entry point, fi_mm_bf16_fp4: two split-K
+calls in a row (the second with another shape, over the partials the first one left
+behind) must both agree within the parity tolerance used by the other GPU tests, and a call
+whose partials would not fit the array must be refused before anything is launched.
+
+This file sorts last so that a run which stops at the first failure has run every other
+test first; it passes on its own in a fresh process as well.
+"""
+import numpy as np
+import pytest
+import torch
+
+import bf16_activations_nvfp4_b200 as fi
+from bf16_activations_nvfp4_b200 import inputs
+from tests import _gpu
+
+pytestmark = pytest.mark.gpu
+
+SCRATCH_BYTES = 4 << 20  # FI_NOALLOC_SCRATCH_BYTES
+
+
+def _noalloc(A, Wq, Ws, g, out, tactic):
+    m, k = A.shape
+    n = Wq.shape[0]
+    lib = fi.library()
+    return lib.fi_mm_bf16_fp4_noalloc(A.data_ptr(), Wq.data_ptr(), Ws.data_ptr(), g.data_ptr(), out.data_ptr(),
+                                      m, n, k, tactic, torch.cuda.current_stream().cuda_stream)
+
+
+def _allocating(A, Wq, Ws, g, tactic):
+    m, k = A.shape
+    n = Wq.shape[0]
+    out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    st = fi.library().fi_mm_bf16_fp4(A.data_ptr(), Wq.data_ptr(), Ws.data_ptr(), g.data_ptr(), out.data_ptr(),
+                                     m, n, k, tactic, torch.cuda.current_stream().cuda_stream)
+    assert st == 0, fi.last_error()
+    return out
+
+
+@pytest.mark.parametrize("splits", [4, 8])
+def test_two_calls_in_a_row_match_the_allocating_entry_point(splits):
+    tactic = fi.make_tactic(fi.KIND_GEMV, splits, 0, 0)
+    calls = [(3, 1000, 4096, 11), (2, 600, 2048, 12)]  # ragged n; the second reuses dirty scratch
+    for m, n, k, seed in calls:
+        assert 0 < fi.workspace_bytes(m, n, k, tactic) <= SCRATCH_BYTES
+        A = _gpu.dev_bf16(inputs.activations(m, k, seed=seed))
+        Wq, Ws, g = _gpu.device_weights(n, k, seed)
+        out = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = _noalloc(A, Wq, Ws, g, out, tactic)
+        assert st == 0, fi.last_error()
+        ref = _allocating(A, Wq, Ws, g, tactic)
+        torch.cuda.synchronize()
+        _gpu.assert_within_tolerance(_gpu.host_bits(out), _gpu.bits_to_f64(_gpu.host_bits(ref)),
+                                     f"no-alloc vs allocating, m={m} n={n} k={k} S={splits}")
+
+
+def test_single_split_needs_no_scratch():
+    m, n, k = 1, 512, 2048
+    tactic = fi.make_tactic(fi.KIND_GEMV, 1, 0, 0)
+    A = _gpu.dev_bf16(inputs.activations(m, k, seed=3))
+    Wq, Ws, g = _gpu.device_weights(n, k, 0)
+    out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    assert _noalloc(A, Wq, Ws, g, out, tactic) == 0, fi.last_error()
+    ref = _allocating(A, Wq, Ws, g, tactic)
+    torch.cuda.synchronize()
+    _gpu.assert_within_tolerance(_gpu.host_bits(out), _gpu.bits_to_f64(_gpu.host_bits(ref)), "single split")
+
+
+def test_partials_beyond_the_static_scratch_are_refused():
+    m, n, k = 32, 8192, 4096
+    tactic = fi.make_tactic(fi.KIND_GEMV, 8, 0, 0)
+    assert fi.workspace_bytes(m, n, k, tactic) > SCRATCH_BYTES
+    A = _gpu.dev_bf16(inputs.activations(m, k, seed=5))
+    Wq = torch.zeros((n, k // 2), dtype=torch.uint8, device="cuda")
+    Ws = torch.zeros((n, k // 16), dtype=torch.uint8, device="cuda")
+    g = torch.ones(1, dtype=torch.float32, device="cuda")
+    out = torch.full((m, n), 7.0, dtype=torch.bfloat16, device="cuda")
+    st = _noalloc(A, Wq, Ws, g, out, tactic)
+    assert st == -4  # FI_ERR_WORKSPACE
+    assert "scratch" in fi.last_error()
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())  # nothing was launched
