@@ -122,6 +122,8 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_p
                      (long long)m, (long long)(nch * kChunkK));
   int64_t gx = std::max<int64_t>(1, (int64_t)sms * ctas / S);
   if (gx > n) gx = std::max<int64_t>(1, n);
+  g->pipeline = kPipeRing;
+  g->threads = kGemvThreads;
   g->S = S;
   g->RS = (int)rs;
   g->stages = (int)stages;
@@ -135,15 +137,68 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_p
   return FI_OK;
 }
 
+// Per-warp async-copy pipeline: a CTA of kStreamWarps warps holds the split's activations and,
+// per warp, NS slots of R rows x 32 lanes x (16 code bytes + a 4-byte scale word). Every CTA
+// stays within half an SM, so two fit side by side (this call's and the next call's). The grid
+// has ctas_per_sm CTAs per SM (1 or 2; 0 = 1), never more warps than rows.
+int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int ctas_per_sm, int sms,
+                         GemvGeometry* g) {
+  const int64_t C = k / kChunkK;
+  const int64_t nch = (C + S - 1) / S;  // chunks of the largest split
+  const int ctas = ctas_per_sm > 0 ? ctas_per_sm : 1;
+  if (ctas > 2) return set_error(FI_ERR_INVALID_ARG, "GEMV stream pipeline: at most 2 CTAs per SM");
+  const int64_t a_bytes = round_up(m * ((nch + 31) / 32) * 2048, 128);
+  const int64_t as_bytes = round_up(m * nch * 8, 128);
+  const int rmax = std::min(4, gemv_rows_per_stage_max(m));  // registers: at most 4 rows per item
+  int64_t r = r_req;
+  if (r == 0) {  // up to 4 rows per item, fewer when the grid's warps would otherwise run out of rows
+    r = std::min(4, rmax);
+    while (r > 1 && (n + r - 1) / r < (int64_t)sms * ctas * kStreamWarps) r /= 2;
+  }
+  if (r < 1 || r > rmax || (r & (r - 1)) != 0)
+    return set_error(FI_ERR_INVALID_ARG, "GEMV rows per item must be a power of two in 1..%d for m=%lld", rmax,
+                     (long long)m);
+  const int64_t slot = r * kStreamSlotBytesPerRow;
+  const int64_t fixed = a_bytes + as_bytes;
+  int ns = 4;
+  if (fixed + (int64_t)kStreamWarps * ns * slot > kStreamSmemBudget) ns = 2;
+  if (fixed + (int64_t)kStreamWarps * ns * slot > kStreamSmemBudget)
+    return set_error(FI_ERR_UNSUPPORTED_SHAPE,
+                     "GEMV: m=%lld over %lld k per split leaves no room for the weight slots in shared memory; "
+                     "use more splits",
+                     (long long)m, (long long)(nch * kChunkK));
+  const int64_t warps_wanted = (n + r - 1) / r;  // at least one row group per warp
+  int64_t gx = std::max<int64_t>(1, (int64_t)sms * ctas / S);
+  gx = std::max<int64_t>(1, std::min<int64_t>(gx, (warps_wanted + kStreamWarps - 1) / kStreamWarps));
+  g->pipeline = kPipeStream;
+  g->threads = kStreamThreads;
+  g->S = S;
+  g->RS = (int)r;
+  g->stages = ns;
+  g->ctas_per_sm = ctas;
+  g->grid_x = (int)gx;
+  g->stage_bytes = slot;
+  g->off_as = a_bytes;
+  g->off_bar = fixed;
+  g->off_ring = fixed;
+  g->smem_bytes = fixed + (int64_t)kStreamWarps * ns * slot;
+  return FI_OK;
+}
+
+static int geometry_for(int pipe, int64_t m, int64_t n, int64_t k, int S, int r, int ctas, int sms, GemvGeometry* g) {
+  return pipe == kPipeRing ? gemv_geometry(m, n, k, S, r, ctas, sms, g)
+                           : gemv_stream_geometry(m, n, k, S, r, ctas, sms, g);
+}
+
 // Device-sized split (PR #4038, Description, "What it does": the device-sized GEMV split): the fewest splits S
 // that give every SM a CTA with rows to stream while `m_fit` activation rows of a split fit
 // the shared-memory staging next to the weight ring. Depends on (n, k, SMs, R, m_fit) only.
-static int gemv_knee(int64_t n, int64_t k, int sms, int64_t m_fit, int rs, int ctas, int* S_out) {
+static int gemv_knee(int pipe, int64_t n, int64_t k, int sms, int64_t m_fit, int rs, int ctas, int* S_out) {
   const int64_t C = k / kChunkK;
   const int64_t maxS = std::max<int64_t>(1, std::min<int64_t>(C, 4095));
   for (int64_t S = 1; S <= maxS; ++S) {
     GemvGeometry g;
-    if (gemv_geometry(m_fit, n, k, (int)S, rs, ctas, sms, &g) != FI_OK) continue;
+    if (geometry_for(pipe, m_fit, n, k, (int)S, rs, ctas, sms, &g) != FI_OK) continue;
     const bool enough = (int64_t)g.grid_x * S >= (int64_t)sms * g.ctas_per_sm;
     const bool last = S == maxS || (C / (S + 1)) < 32;  // a split keeps at least one warp step
     if (enough || last) {
@@ -163,15 +218,17 @@ static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms)
   if (m <= kDefaultGemvMaxM) {
     const int64_t m_fit = m <= 1 ? 1 : (m <= 8 ? 8 : kGemvMaxM);
     int S = 1;
-    if (gemv_knee(n, k, num_sms, m_fit, 0, 1, &S) != FI_OK) S = 1;
-    return FI_TACTIC(FI_KIND_GEMV, S, 0, 0);
+    if (gemv_knee(kPipeStream, n, k, num_sms, m_fit, 0, 1, &S) != FI_OK) S = 1;
+    return FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeStream << 4);
   }
   return FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
 }
 
-// GEMV variant byte: rows per ring stage (consecutive weight rows one consumer warp
-// computes together; 0 = as many as fit the stage target). Splits 0 = device-sized, resolved
-// for m <= 32 so that the resolved S (and the bits) never depend on m.
+// GEMV variant byte: low nibble = weight rows computed together by one warp (ring pipeline:
+// rows per ring stage; stream pipeline: rows per work item; 0 = automatic); high nibble = the
+// pipeline (0 = automatic = stream, 1 = stream, 2 = ring). Both pipelines give the same bits
+// for the same S. Splits 0 = device-sized, resolved for m <= 32 so that the resolved S (and
+// the bits) never depend on m.
 static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var,
                         int sms, fi_tactic_info* out) {
   if (m > kGemvMaxM)
@@ -179,10 +236,15 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
                      kGemvMaxM, (long long)m);
   const int64_t C = k / kChunkK;
   const int ctas = ctas_req ? ctas_req : 1;
-  if (var < 0 || var > 8) return set_error(FI_ERR_INVALID_ARG, "GEMV rows per stage must be 0, 1, 2, 4 or 8");
+  const int rsel = var & 0xF;
+  const bool pipe_auto = (var >> 4) == kPipeAuto;
+  int pipe = pipe_auto ? kPipeStream : var >> 4;
+  if (var < 0 || pipe > kPipeRing || rsel > 8)
+    return set_error(FI_ERR_INVALID_ARG, "GEMV variant 0x%x: rows must be 0, 1, 2, 4 or 8 and the pipeline 0, 1 or 2",
+                     var);
   int S = S_req;
   if (S == 0) {
-    const int rc = gemv_knee(n, k, sms, kGemvMaxM, 0, ctas, &S);
+    const int rc = gemv_knee(pipe, n, k, sms, kGemvMaxM, 0, ctas, &S);
     if (rc != FI_OK) return rc;
   } else if (C > 0 && S > C) {
     return set_error(FI_ERR_INVALID_ARG, "splits=%lld exceeds k/32=%lld", (long long)S, (long long)C);
@@ -190,21 +252,29 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
   GemvGeometry g;
   if (C == 0) {  // k == 0: nothing to stream; the caller writes zeros
     memset(&g, 0, sizeof(g));
+    g.pipeline = pipe;
     g.S = 1;
     g.RS = 1;
     g.ctas_per_sm = ctas;
     g.grid_x = 1;
+    g.threads = pipe == kPipeRing ? kGemvThreads : kStreamThreads;
   } else {
-    const int rc = gemv_geometry(m, n, k, S, var, ctas, sms, &g);
+    int rc = geometry_for(pipe, m, n, k, S, rsel, ctas, sms, &g);
+    // the automatic pipeline takes the ring (a whole SM's shared memory) when the activations
+    // do not fit the stream pipeline's half SM; both give the same bits for the same S
+    if (rc == FI_ERR_UNSUPPORTED_SHAPE && pipe_auto) {
+      rc = geometry_for(kPipeRing, m, n, k, S, rsel, ctas, sms, &g);
+      if (rc == FI_OK) clear_error();
+    }
     if (rc != FI_OK) return rc;
   }
   out->kind = FI_KIND_GEMV;
   out->splits = g.S;
   out->ctas_per_sm = g.ctas_per_sm;
-  out->variant = g.RS;
+  out->variant = g.RS | (g.pipeline << 4);
   out->grid_x = g.grid_x;
   out->grid_y = g.S;
-  out->threads = kGemvThreads;
+  out->threads = g.threads;
   out->smem_bytes = (int32_t)g.smem_bytes;
   out->workspace_bytes = g.S > 1 ? (int64_t)g.S * m * n * (int64_t)sizeof(float) : 0;
   return FI_OK;
@@ -336,7 +406,7 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
   }
   if (info.kind == FI_KIND_GEMV) {
     GemvGeometry g;
-    rc = gemv_geometry(m, n, k, info.splits, info.variant, info.ctas_per_sm, sms, &g);
+    rc = geometry_for(info.variant >> 4, m, n, k, info.splits, info.variant & 0xF, info.ctas_per_sm, sms, &g);
     if (rc != FI_OK) return rc;
     GemvArgs a;
     memset(&a, 0, sizeof(a));
@@ -349,6 +419,7 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.m = m;
     a.n = n;
     a.k = k;
+    a.pipeline = g.pipeline;
     a.splits = g.S;
     a.rows_per_stage = g.RS;
     a.stages = g.stages;
@@ -438,14 +509,17 @@ int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, 
   clear_error();
   const int sms = sms_or_device(num_sms);
   if (sms <= 0) return set_error(FI_ERR_CUDA, "no device to query the SM count from");
-  // the split menu {1, 2, 4, 8, device-sized}, each with the automatic stage size and with one
-  // and two rows per stage; entries resolving to the same launch are listed once
-  int64_t cand[32];
+  // the split menu {1, 2, 4, 8, device-sized} on both pipelines, each with the automatic row
+  // count and with one and two rows per warp, the stream pipeline also with two CTAs per SM;
+  // entries resolving to the same launch are listed once
+  int64_t cand[64];
   int nc = 0;
   const int splits[] = {1, 2, 4, 8, 0};
-  for (int R : {0, 1, 2})
-    for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, R);
-  fi_tactic_info seen[32];
+  for (int pipe : {kPipeStream, kPipeRing})
+    for (int R : {0, 1, 2})
+      for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, R | (pipe << 4));
+  for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 2, kPipeStream << 4);
+  fi_tactic_info seen[64];
   int nseen = 0, count = 0;
   for (int c = 0; c < nc; ++c) {
     fi_tactic_info info;

@@ -262,10 +262,10 @@ __device__ __forceinline__ void stage_rows(uint32_t code0, int cstride, uint32_t
 }
 
 // Combine the lanes of acc (fixed xor butterfly: every lane ends with the same bits) and
-// write rows j0 .. j0+NR-1: bf16_rn(acc * g) when S == 1, else the fp32 partial of split s.
+// write rows j0 .. j0+rows-1: bf16_rn(acc * g) when S == 1, else the fp32 partial of split s.
 template <int MT, int NR>
-__device__ __forceinline__ void finish_rows(float (&acc)[NR][MT], const GemvArgs& p, int64_t j0, int m, int S,
-                                            int s, float g, int lane, bool write) {
+__device__ __forceinline__ void finish_rows(float (&acc)[NR][MT], const GemvArgs& p, int64_t j0, int rows, int m,
+                                            int S, int s, float g, int lane, bool write) {
 #pragma unroll
   for (int i = 0; i < NR; ++i)
 #pragma unroll
@@ -280,7 +280,7 @@ __device__ __forceinline__ void finish_rows(float (&acc)[NR][MT], const GemvArgs
   for (int i = 0; i < NR; ++i)
 #pragma unroll
     for (int r = 0; r < MT; ++r)
-      if (r < m && lane == ((i * MT + r) & 31)) {
+      if (i < rows && r < m && lane == ((i * MT + r) & 31)) {
         const int64_t j = j0 + i;
         if (S == 1)
           p.out[(int64_t)r * p.n + j] = f32_to_bf16_rn(acc[i][r] * g);
@@ -440,7 +440,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
         for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
       if (ok)
         stage_rows<MT, RS>(stage_s, codes_stride, sbase, sstride, off0, doff, a_s, as_s, m, nch, GA, lane, acc);
-      finish_rows<MT, RS>(acc, p, j0, m, S, s, g, lane, write);
+      finish_rows<MT, RS>(acc, p, j0, RS, m, S, s, g, lane, write);
     } else {
       // the CTA's last, partial stage: one row at a time
       for (int i = 0; i < rows; ++i) {
@@ -451,12 +451,251 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
           stage_rows<MT, 1>(stage_s + (uint32_t)(i * codes_stride), codes_stride,
                             sbase + (uint32_t)(i * sstride) + ((off0 + (uint32_t)i * doff) & 15u), 0, 0u, 0u,
                             a_s, as_s, m, nch, GA, lane, acc);
-        finish_rows<MT, 1>(acc, p, j0 + i, m, S, s, g, lane, write);
+        finish_rows<MT, 1>(acc, p, j0 + i, 1, m, S, s, g, lane, write);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
   }
+}
+
+// ============================================================ per-warp async-copy pipeline
+//
+// The second GEMV pipeline. Every warp streams its own weight rows with per-thread
+// asynchronous copies (cp.async, the load/store-unit path of ordinary loads) into its own ring
+// of NS shared-memory slots, and computes from there. There is no producer warp and no barrier
+// between warps: lane L copies exactly the 16-byte code cells (and the scale bytes) of the
+// chunks it computes, so each thread waits only for its own copies (cp.async.wait_group, a
+// hardware wait that costs no issue slots and cannot outlive the copies). A slot holds R
+// weight rows at one chunk iteration: row i's cell of lane L at i*512 + L*16, and the 4-byte
+// aligned word holding the lane's two E4M3 scale bytes at R*512 + i*128 + L*4.
+//
+// The work item of a warp is (row group, chunk iteration t): chunk c = 32 t + L of the split
+// for R consecutive rows. Items run in order, each lane taking chunks L, L+32, ... of every
+// row in increasing order with the same per-chunk arithmetic as the ring pipeline, so the
+// two pipelines give bitwise identical results for the same S.
+//
+// A CTA is 8 warps and at most about half of an SM's shared memory and registers, so the
+// CTAs of the next programmatically dependent launch can become resident beside it and start
+// their weight stream while this one finishes.
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void sts_u16(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"((unsigned short)v) : "memory");
+}
+
+// One chunk c of the split for R weight rows against MT activation rows. code_s is the lane's
+// cell of row 0 in the slot, scale_s the lane's scale word of row 0; soff[i] is the offset (0
+// or 2) of the lane's two scale bytes within row i's word. Every weight row is computed
+// without a branch, so the compiler can interleave the rows' independent FMA chains; rows of a
+// partial group compute on stale cells and are never written. Same arithmetic per chunk as
+// stage_rows.
+template <int MT, int R>
+__device__ __forceinline__ void item_rows(uint32_t code_s, uint32_t scale_s, const uint32_t (&soff)[R], uint32_t a_s,
+                                          uint32_t as_s, int m, int nch, int GA, int c, float (&acc)[R][MT]) {
+  const uint32_t a_row = (uint32_t)GA * 4 * 32 * 16;
+  const uint32_t as_row = (uint32_t)nch * 8;
+  const uint32_t ap = a_s + (uint32_t)(((c >> 5) * 4 * 32 + (c & 31)) * 16);
+  const uint32_t sp = as_s + (uint32_t)c * 8;
+  if (MT == 1) {
+    const uint4 a0 = lds_v4(ap), a1 = lds_v4(ap + 512), a2 = lds_v4(ap + 1024), a3 = lds_v4(ap + 1536);
+    const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                             a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+    const float2 sa = lds_f2(sp);
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const uint4 cq = lds_v4(code_s + (uint32_t)(i * 512));
+      const uint32_t sc = lds_u16(scale_s + (uint32_t)(i * 128) + soff[i]);
+      uint32_t wf[16];
+      decode32(cq, wf);
+      const float p0 = dot16(av, wf, 0.0f);
+      const float p1 = dot16(av + 8, wf + 8, 0.0f);
+      const uint32_t sh = e4m3x2_to_f16x2(sc);
+      acc[i][0] = fmaf(p0, f16_lo_to_f32(sh) * sa.x, acc[i][0]);
+      acc[i][0] = fmaf(p1, f16_hi_to_f32(sh) * sa.y, acc[i][0]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const uint4 cq = lds_v4(code_s + (uint32_t)(i * 512));
+      const uint32_t sc = lds_u16(scale_s + (uint32_t)(i * 128) + soff[i]);
+      uint32_t wf[16];
+      decode32(cq, wf);
+      const uint32_t sh = e4m3x2_to_f16x2(sc);
+      const float sw0 = f16_lo_to_f32(sh), sw1 = f16_hi_to_f32(sh);
+#pragma unroll
+      for (int r = 0; r < MT; ++r) {
+        if (r < m) {
+          const uint32_t apr = ap + (uint32_t)r * a_row;
+          const uint4 a0 = lds_v4(apr), a1 = lds_v4(apr + 512), a2 = lds_v4(apr + 1024), a3 = lds_v4(apr + 1536);
+          const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                                   a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+          const float2 sa = lds_f2(sp + (uint32_t)r * as_row);
+          const float p0 = dot16(av, wf, 0.0f);
+          const float p1 = dot16(av + 8, wf + 8, 0.0f);
+          acc[i][r] = fmaf(p0, sw0 * sa.x, acc[i][r]);
+          acc[i][r] = fmaf(p1, sw1 * sa.y, acc[i][r]);
+        }
+      }
+    }
+  }
+}
+
+template <int MT, int R, int NS>
+__global__ void __launch_bounds__(kStreamThreads, 2) gemv_stream_kernel(GemvArgs p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr uint32_t kSlot = (uint32_t)R * kStreamSlotBytesPerRow;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int m = (int)p.m;
+  const int64_t n = p.n, k = p.k;
+  const int S = p.splits;
+  const int s = blockIdx.y;
+
+  // K range of this split, in 32-k chunks, and the chunk iterations of a row
+  const int64_t C = k / kChunkK;
+  const int64_t c0 = (int64_t)s * C / S;
+  const int nch = (int)((int64_t)(s + 1) * C / S - c0);
+  const int T = (nch + 31) / 32;
+
+  // rows of this warp (balanced over all warps of the split), R per group
+  const int64_t GW = (int64_t)gridDim.x * kStreamWarps;
+  const int64_t gw = (int64_t)blockIdx.x * kStreamWarps + warp;
+  const int64_t r_lo = gw * n / GW, r_hi = (gw + 1) * n / GW;
+  const int64_t Q = (r_hi - r_lo + R - 1) / R * T;  // items of this warp
+
+  const int64_t rs_q = k / 2, rs_s = k / 16;
+  const uint8_t* const ws_end = p.Ws + n * rs_s;
+  const uint32_t a_s = smem_addr(smem), as_s = smem_addr(smem + p.off_as);
+  const uint32_t ring = smem_addr(smem + p.off_ring) + (uint32_t)warp * NS * kSlot;
+  const uint32_t my_code = ring + (uint32_t)lane * 16;
+  const uint32_t my_scale = ring + (uint32_t)R * 512 + (uint32_t)lane * 4;
+  const int64_t lane_k = (c0 + lane) * 2;  // the lane's first scale byte within a row's split
+
+  pdl_launch_dependents();
+
+  // ---- issue cursor: item iq = (group ig, iteration it); row pointers advance per item
+  int64_t ig = 0, iq = 0;
+  int it = 0;
+  const uint8_t* qsrc[R];  // row i's code cell for this lane at iteration it
+  const uint8_t* ssrc[R];  // the 4-byte aligned word holding the lane's two scale bytes
+  int irows = 0;
+  bool ifast = true;  // a full group that cannot reach the tensor's last scale bytes
+  auto issue_group = [&]() {
+    const int64_t j0 = r_lo + ig * R;
+    irows = (int)max((int64_t)0, min((int64_t)R, r_hi - j0));
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int64_t j = j0 + i;
+      qsrc[i] = p.Wq + j * rs_q + (c0 + lane) * 16;
+      ssrc[i] = p.Ws + ((j * rs_s + lane_k) & ~(int64_t)3);
+    }
+    ifast = irows == R && !((n * rs_s) % 4 != 0 && j0 + R >= n);
+  };
+  // copy item iq into slot u; always commits one group (empty past the warp's last item) so
+  // that wait_group counts stay uniform
+  auto issue = [&](int u) {
+    if (iq < Q) {
+      if (it * 32 + lane < nch) {
+        const uint32_t cdst = my_code + (uint32_t)u * kSlot;
+        const uint32_t sdst = my_scale + (uint32_t)u * kSlot;
+        if (ifast) {
+#pragma unroll
+          for (int i = 0; i < R; ++i) {
+            cp_async_16(cdst + (uint32_t)(i * 512), qsrc[i]);
+            cp_async_4(sdst + (uint32_t)(i * 128), ssrc[i]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < R; ++i) {
+            if (i < irows) {
+              cp_async_16(cdst + (uint32_t)(i * 512), qsrc[i]);
+              if (ssrc[i] + 4 <= ws_end) {
+                cp_async_4(sdst + (uint32_t)(i * 128), ssrc[i]);
+              } else {  // the tensor's last scale pair when its size is 2 mod 4: plain load
+                const uint32_t off = (uint32_t)(((r_lo + ig * R + i) * rs_s + lane_k) & 2);
+                sts_u16(sdst + (uint32_t)(i * 128) + off, ldg_stream_u16(ssrc[i] + off));
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        qsrc[i] += 512;
+        ssrc[i] += 64;
+      }
+      ++iq;
+      if (++it == T) {
+        it = 0;
+        ++ig;
+        issue_group();
+      }
+    }
+    cp_async_commit();
+  };
+
+  // prologue: the first NS items (weights only: they do not depend on the preceding kernel)
+  issue_group();
+#pragma unroll
+  for (int u = 0; u < NS; ++u) issue(u);
+
+  pdl_wait();
+  const int GA = (nch + 31) / 32;
+  stage_activations(p.A, k, m, c0 * kChunkK, nch, reinterpret_cast<uint4*>(smem),
+                    reinterpret_cast<float*>(smem + p.off_as), tid, kStreamThreads);
+  __syncthreads();
+  const float g = (S == 1) ? *p.gscale : 1.0f;
+
+  // ---- compute cursor
+  float acc[R][MT];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
+  int64_t j0 = r_lo;
+  int ct = 0, u = 0;
+  uint32_t soff[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) soff[i] = (uint32_t)(((j0 + i) * rs_s + lane_k) & 2);
+  for (int64_t q = 0; q < Q; ++q) {
+    const int c = ct * 32 + lane;
+    cp_async_wait<NS - 1>();  // this lane's copies of item q have landed
+    if (c < nch)
+      item_rows<MT, R>(my_code + (uint32_t)u * kSlot, my_scale + (uint32_t)u * kSlot, soff, a_s, as_s, m, nch, GA, c,
+                       acc);
+    // refill the slot just read with item q + NS (the reads above are complete: their
+    // results have been consumed)
+    issue(u);
+    if (++ct == T) {
+      finish_rows<MT, R>(acc, p, j0, (int)min((int64_t)R, r_hi - j0), m, S, s, g, lane, true);
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
+      ct = 0;
+      j0 += R;
+#pragma unroll
+      for (int i = 0; i < R; ++i) soff[i] = (uint32_t)(((j0 + i) * rs_s + lane_k) & 2);
+    }
+    u = (u + 1 == NS) ? 0 : u + 1;
+  }
+  cp_async_wait<0>();
 }
 
 namespace {
@@ -488,6 +727,55 @@ int launch_one(const GemvArgs& a, cudaStream_t stream) {
   return FI_OK;
 }
 
+template <int MT, int R, int NS>
+int launch_stream_one(const GemvArgs& a, cudaStream_t stream) {
+  auto kern = gemv_stream_kernel<MT, R, NS>;
+  static int configured[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return set_cuda_error("cudaGetDevice");
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget) != cudaSuccess)
+      return set_cuda_error("cudaFuncSetAttribute(gemv stream smem)");
+    configured[dev] = 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.grid_x, (unsigned)a.splits);
+  cfg.blockDim = dim3(kStreamThreads);
+  cfg.dynamicSmemBytes = (size_t)a.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return set_cuda_error("gemv stream kernel launch");
+  return FI_OK;
+}
+
+template <int MT, int R>
+int launch_stream_ns(const GemvArgs& a, cudaStream_t stream) {
+  if (a.stages == 4) return launch_stream_one<MT, R, 4>(a, stream);
+  if (a.stages == 2) return launch_stream_one<MT, R, 2>(a, stream);
+  return set_error(FI_ERR_INVALID_ARG, "GEMV stream pipeline: %d slots per warp is not available", a.stages);
+}
+
+template <int MT>
+int launch_stream_r(const GemvArgs& a, cudaStream_t stream) {
+  switch (a.rows_per_stage) {
+    case 1: return launch_stream_ns<MT, 1>(a, stream);
+    case 2:
+      if constexpr (gemv_rmax(MT) >= 2) return launch_stream_ns<MT, 2>(a, stream);
+      break;
+    case 4:
+      if constexpr (gemv_rmax(MT) >= 4) return launch_stream_ns<MT, 4>(a, stream);
+      break;
+    default: break;
+  }
+  return set_error(FI_ERR_INVALID_ARG, "GEMV rows per item %d is not available for m=%lld", a.rows_per_stage,
+                   (long long)a.m);
+}
+
 template <int MT>
 int launch_rs(const GemvArgs& a, cudaStream_t stream) {
   switch (a.rows_per_stage) {
@@ -511,13 +799,20 @@ int launch_rs(const GemvArgs& a, cudaStream_t stream) {
 
 int gemv_rows_per_stage_max(int64_t m) { return gemv_rmax(gemv_mt(m)); }
 
+namespace {
+template <int MT>
+int launch_mt(const GemvArgs& a, cudaStream_t stream) {
+  return a.pipeline == kPipeRing ? launch_rs<MT>(a, stream) : launch_stream_r<MT>(a, stream);
+}
+}  // namespace
+
 int launch_gemv(const GemvArgs& a, cudaStream_t stream) {
-  if (a.m <= 1) return launch_rs<1>(a, stream);
-  if (a.m <= 2) return launch_rs<2>(a, stream);
-  if (a.m <= 4) return launch_rs<4>(a, stream);
-  if (a.m <= 8) return launch_rs<8>(a, stream);
-  if (a.m <= 16) return launch_rs<16>(a, stream);
-  if (a.m <= 32) return launch_rs<32>(a, stream);
+  if (a.m <= 1) return launch_mt<1>(a, stream);
+  if (a.m <= 2) return launch_mt<2>(a, stream);
+  if (a.m <= 4) return launch_mt<4>(a, stream);
+  if (a.m <= 8) return launch_mt<8>(a, stream);
+  if (a.m <= 16) return launch_mt<16>(a, stream);
+  if (a.m <= 32) return launch_mt<32>(a, stream);
   return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV supports m <= %d", kGemvMaxM);
 }
 

@@ -28,6 +28,14 @@ constexpr int kSmemBudget = 227 * 1024 - 1024;             // dynamic shared mem
 constexpr int kGemvMaxStages = 16;
 constexpr int kGemvStageTarget = 16 * 1024;                // preferred bytes per ring stage
 
+// The per-warp async-copy pipeline: 8 warps per CTA, every CTA at most half an SM.
+constexpr int kStreamWarps = 8;
+constexpr int kStreamThreads = kStreamWarps * 32;
+constexpr int kStreamSlotBytesPerRow = 32 * 16 + 32 * 4;   // a row's code cells + scale words
+constexpr int kStreamSmemBudget = 228 * 1024 / 2 - 1024;   // two CTAs per SM
+// pipelines (the high nibble of the GEMV tactic variant)
+constexpr int kPipeAuto = 0, kPipeStream = 1, kPipeRing = 2;
+
 // Activation rows the GEMV kernel instance for m is compiled for (1, 2, 4, ..., 32).
 inline int gemv_mt(int64_t m) {
   int mt = 1;
@@ -49,13 +57,18 @@ int gemv_rows_per_stage_max(int64_t m);
 
 // Launch geometry of the GEMV for one shape and tactic (computed on the host).
 struct GemvGeometry {
-  int S, RS, stages, ctas_per_sm, grid_x;
+  int pipeline;  // kPipeStream or kPipeRing
+  int S, RS, stages, ctas_per_sm, grid_x, threads;
   int64_t stage_bytes, off_as, off_bar, off_ring, smem_bytes;
 };
 // Returns FI_OK and fills g, or FI_ERR_UNSUPPORTED_SHAPE when the activations of m rows over
 // a split leave no room for two ring stages of one weight row in shared memory. rs_req is
 // the requested rows per stage (0 = as many as fit the stage target).
 int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_per_sm, int sms, GemvGeometry* g);
+// The same for the per-warp async-copy pipeline: R rows per item (0 = automatic), ring slots
+// per warp (4, else 2 when the activations leave room for only two).
+int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int ctas_per_sm, int sms,
+                         GemvGeometry* g);
 
 struct GemvArgs {
   const uint16_t* A;
@@ -65,9 +78,10 @@ struct GemvArgs {
   uint16_t* out;       // used when splits == 1
   float* partials;     // [splits, m, n] when splits > 1
   int64_t m, n, k;
+  int pipeline;        // kPipeStream or kPipeRing
   int splits;          // S: global K splits (grid.y)
   int rows_per_stage;  // RS: consecutive weight rows per ring stage (one consumer warp each)
-  int stages;          // NST: ring stages
+  int stages;          // NST: ring stages (stream pipeline: slots per warp)
   int grid_x;          // CTAs per split
   int pdl;             // launch with programmatic stream serialization
   int debug_stall;     // test hook: the producer issues nothing (consumer waits time out)

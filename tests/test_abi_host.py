@@ -49,7 +49,9 @@ def test_default_gemv_tactic_resolves_for_decode_shapes(n, k):
     assert 1 <= info["splits"] <= k // 32
     # one persistent wave: the grid never asks for more CTAs than the SMs hold
     assert info["grid_x"] * info["grid_y"] <= B200_SMS * info["ctas_per_sm"]
-    assert info["threads"] == 17 * 32 and 0 < info["smem_bytes"] <= 227 * 1024
+    # the default runs the per-warp async-copy pipeline: 8 warps, at most half an SM
+    assert info["variant"] >> 4 == 1
+    assert info["threads"] == 8 * 32 and 0 < info["smem_bytes"] <= 228 * 1024 // 2 - 1024
     assert info["workspace_bytes"] == (info["splits"] * n * 4 if info["splits"] > 1 else 0)
 
 
@@ -83,7 +85,9 @@ def test_explicit_splits_are_kept():
         info = fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, S, 0, 2), B200_SMS)
         assert info["splits"] == S and info["variant"] & 0xF == 2
     info = fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, 2, 2, 1), B200_SMS)
-    assert (info["splits"], info["ctas_per_sm"], info["variant"]) == (2, 2, 1)
+    assert (info["splits"], info["ctas_per_sm"], info["variant"] & 0xF) == (2, 2, 1)
+    ring = fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, 2, 1, 0x21), B200_SMS)
+    assert (ring["variant"], ring["threads"]) == (0x21, 17 * 32)
 
 
 def test_list_tactics_unique_and_valid():
@@ -111,7 +115,8 @@ def test_workspace_bytes():
     (32, 64, 14336, fi.make_tactic(0, 1, 0, 1), -2),      # A slice does not fit shared memory
     (32, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),       # one row per stage above m = 8
     (5, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),        # two rows per stage above m = 4
-    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x12), -1),     # rows per stage 18
+    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x32), -1),     # pipeline 3
+    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x19), -1),     # rows 9 on the stream pipeline
     (1, 8, 65536, fi.make_tactic(0, 1, 0, 2), -2),        # two 36 KB rows per stage do not fit twice
 ])
 def test_resolve_rejects(m, n, k, tactic, status):

@@ -1,9 +1,10 @@
 """Failure detection on the GPU without a fault: a pipeline wait that runs out.
 
-The test hook stalls the GEMV's producer warp for one launch, so the consumer warps' waits on
-the shared-memory pipeline run out after a short limit. The kernel must then end on its own,
-record the timeout in the device error word that the host reads, and leave the context usable:
-the next call runs normally and is correct.
+The test hook stalls the producer warp of the GEMV's ring pipeline for one launch, so the
+consumer warps' waits on the shared-memory pipeline run out after a short limit. (The stream
+pipeline has no waits between warps: each thread waits only for its own copies.) The kernel
+must then end on its own, record the timeout in the device error word that the host reads,
+and leave the context usable: the next call runs normally and is correct.
 """
 import numpy as np
 import pytest
@@ -15,6 +16,8 @@ from bf16_activations_nvfp4_b200 import inputs
 from tests import _gpu
 
 pytestmark = pytest.mark.gpu
+
+RING = fi.make_tactic(fi.KIND_GEMV, 1, 0, 0x22)  # ring pipeline, two rows per stage
 
 
 def test_stalled_pipeline_reports_timeout_and_recovers():
@@ -28,7 +31,7 @@ def test_stalled_pipeline_reports_timeout_and_recovers():
     fi.debug_set(fi.DEBUG_WAIT_TIMEOUT_NS, 20_000_000)  # 20 ms
     fi.debug_set(fi.DEBUG_STALL_PRODUCER, 1)
     try:
-        fi.mm_bf16_fp4(A, Wq, Ws, g, tactic=fi.make_tactic(fi.KIND_GEMV, 1, 0, 2))
+        fi.mm_bf16_fp4(A, Wq, Ws, g, tactic=RING)
         torch.cuda.synchronize()
         code = fi.get_device_error()
         assert code & 1, code  # a consumer wait ran out
@@ -36,7 +39,7 @@ def test_stalled_pipeline_reports_timeout_and_recovers():
     finally:
         fi.debug_set(fi.DEBUG_STALL_PRODUCER, 0)
         fi.debug_set(fi.DEBUG_WAIT_TIMEOUT_NS, 1_000_000_000)
-    out = fi.mm_bf16_fp4(A, Wq, Ws, g, tactic=fi.make_tactic(fi.KIND_GEMV, 1, 0, 2))
+    out = fi.mm_bf16_fp4(A, Wq, Ws, g, tactic=RING)
     torch.cuda.synchronize()
     _gpu.assert_within_tolerance(_gpu.host_bits(out), ref, "after recovery")
     assert fi.get_device_error() == 0

@@ -135,15 +135,32 @@ def test_batch_invariance_many_rows_per_stage_small_m():
 
 
 def test_rows_per_stage_and_occupancy_do_not_change_bits():
-    """Only the kind and S fix the arithmetic: rows per stage and CTAs per SM only move work
-    between warps and CTAs."""
+    """Only the kind and S fix the arithmetic: the pipeline, rows per warp and CTAs per SM only
+    move work between warps and CTAs."""
     m, n, k = 2, 2048, 7168
     A = inputs.activations(m, k, seed=9)
     dw = _gpu.device_weights(n, k, 0)
     for S in (1, 3):
-        outs = [_mm(A, dw, fi.make_tactic(GEMV, S, c, R)) for R in (0, 1, 2, 8) for c in (1, 2)]
-        for o in outs[1:]:
-            assert np.array_equal(o, outs[0]), S
+        variants = [(0x10 | R, c) for R in (0, 1, 2, 4) for c in (1, 2)] + [(0x20 | R, 1) for R in (0, 1, 8)]
+        outs = [_mm(A, dw, fi.make_tactic(GEMV, S, c, v)) for v, c in variants]
+        for (v, c), o in zip(variants[1:], outs[1:]):
+            assert np.array_equal(o, outs[0]), (S, hex(v), c)
+
+
+def test_pipelines_give_identical_bits():
+    """The per-warp async-copy pipeline and the producer-warp ring run the same per-chunk
+    arithmetic in the same order, so for one S their outputs are bitwise equal."""
+    for m, n, k in [(1, 2048, 7168), (3, 1000, 4096), (8, 515, 2688), (32, 300, 2048)]:
+        A = inputs.activations(m, k, seed=21, outliers=True)
+        dw = _gpu.device_weights(n, k, 2)
+        for S in (1, 2, 5):
+            try:
+                stream = _mm(A, dw, fi.make_tactic(GEMV, S, 0, 0x10))
+            except fi.FiError as e:  # activations of this split do not fit half an SM
+                assert e.status == -2
+                continue
+            ring = _mm(A, dw, fi.make_tactic(GEMV, S, 0, 0x20))
+            assert np.array_equal(stream, ring), (m, n, k, S)
 
 
 def test_multi_slab_rows_and_many_splits():
