@@ -137,41 +137,44 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_p
   return FI_OK;
 }
 
-// Per-warp async-copy pipeline: a CTA of kStreamWarps warps holds the split's activations and,
-// per warp, NS slots of R rows x 32 lanes x (16 code bytes + a 4-byte scale word). Every CTA
-// stays within half an SM, so two fit side by side (this call's and the next call's). The grid
-// has ctas_per_sm CTAs per SM (1 or 2; 0 = 1), never more warps than rows.
+// Per-warp async-copy pipeline. ctas_per_sm 1: one CTA of 16 warps per SM with the whole
+// shared memory; 2: two CTAs of 8 warps per SM with half of it each. A CTA holds the split's
+// activations and, per warp, NS slots of kStreamIters chunk iterations x R rows x 32 lanes x
+// (16 code bytes + a 4-byte scale word). The grid never has more warps than row groups.
+// Automatic choices (measured on B200 at m = 1): from n = 64 rows per SM on, two 8-warp CTAs per
+// SM with four rows per item; below that, one 16-warp CTA per SM with two rows per item.
+static bool stream_wide(int64_t n, int sms) { return n >= (int64_t)sms * 64; }
+
 int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int ctas_per_sm, int sms,
                          GemvGeometry* g) {
   const int64_t C = k / kChunkK;
   const int64_t nch = (C + S - 1) / S;  // chunks of the largest split
-  const int ctas = ctas_per_sm > 0 ? ctas_per_sm : 1;
+  const int ctas = ctas_per_sm > 0 ? ctas_per_sm : (stream_wide(n, sms) ? 2 : 1);
   if (ctas > 2) return set_error(FI_ERR_INVALID_ARG, "GEMV stream pipeline: at most 2 CTAs per SM");
+  const int nw = ctas == 1 ? 16 : 8;
+  const int64_t budget = ctas == 1 ? kSmemBudget : kStreamHalfBudget;
   const int64_t a_bytes = round_up(m * ((nch + 31) / 32) * 2048, 128);
   const int64_t as_bytes = round_up(m * nch * 8, 128);
   const int rmax = std::min(4, gemv_rows_per_stage_max(m));  // registers: at most 4 rows per item
   int64_t r = r_req;
-  if (r == 0) {  // up to 4 rows per item, fewer when the grid's warps would otherwise run out of rows
-    r = std::min(4, rmax);
-    while (r > 1 && (n + r - 1) / r < (int64_t)sms * ctas * kStreamWarps) r /= 2;
-  }
+  if (r == 0) r = std::min(ctas == 2 ? 4 : 2, rmax);
   if (r < 1 || r > rmax || (r & (r - 1)) != 0)
     return set_error(FI_ERR_INVALID_ARG, "GEMV rows per item must be a power of two in 1..%d for m=%lld", rmax,
                      (long long)m);
-  const int64_t slot = r * kStreamSlotBytesPerRow;
+  const int64_t slot = (int64_t)kStreamIters * r * kStreamCellBytes;
   const int64_t fixed = a_bytes + as_bytes;
   int ns = 4;
-  if (fixed + (int64_t)kStreamWarps * ns * slot > kStreamSmemBudget) ns = 2;
-  if (fixed + (int64_t)kStreamWarps * ns * slot > kStreamSmemBudget)
+  if (fixed + (int64_t)nw * ns * slot > budget) ns = 2;
+  if (fixed + (int64_t)nw * ns * slot > budget)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE,
                      "GEMV: m=%lld over %lld k per split leaves no room for the weight slots in shared memory; "
                      "use more splits",
                      (long long)m, (long long)(nch * kChunkK));
-  const int64_t warps_wanted = (n + r - 1) / r;  // at least one row group per warp
+  const int64_t groups = (n + r - 1) / r;
   int64_t gx = std::max<int64_t>(1, (int64_t)sms * ctas / S);
-  gx = std::max<int64_t>(1, std::min<int64_t>(gx, (warps_wanted + kStreamWarps - 1) / kStreamWarps));
+  gx = std::max<int64_t>(1, std::min<int64_t>(gx, (groups + nw - 1) / nw));
   g->pipeline = kPipeStream;
-  g->threads = kStreamThreads;
+  g->threads = nw * 32;
   g->S = S;
   g->RS = (int)r;
   g->stages = ns;
@@ -181,7 +184,7 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
   g->off_as = a_bytes;
   g->off_bar = fixed;
   g->off_ring = fixed;
-  g->smem_bytes = fixed + (int64_t)kStreamWarps * ns * slot;
+  g->smem_bytes = fixed + (int64_t)nw * ns * slot;
   return FI_OK;
 }
 
@@ -199,7 +202,10 @@ static int gemv_knee(int pipe, int64_t n, int64_t k, int sms, int64_t m_fit, int
   for (int64_t S = 1; S <= maxS; ++S) {
     GemvGeometry g;
     if (geometry_for(pipe, m_fit, n, k, (int)S, rs, ctas, sms, &g) != FI_OK) continue;
-    const bool enough = (int64_t)g.grid_x * S >= (int64_t)sms * g.ctas_per_sm;
+    // enough: the split's CTAs cover at least 40% of the SMs' CTA slots. Measured on B200:
+    // idle SMs cost less than a second kernel and the partials' traffic until well below that
+    // (2048 x 7168 at m = 1 runs faster on 64 CTAs than split in two).
+    const bool enough = (int64_t)g.grid_x * S * 5 >= (int64_t)sms * g.ctas_per_sm * 2;
     const bool last = S == maxS || (C / (S + 1)) < 32;  // a split keeps at least one warp step
     if (enough || last) {
       *S_out = (int)S;
@@ -217,8 +223,9 @@ static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms,
 static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms) {
   if (m <= kDefaultGemvMaxM) {
     const int64_t m_fit = m <= 1 ? 1 : (m <= 8 ? 8 : kGemvMaxM);
+    // stream pipeline with its automatic CTA shape and rows per item (see gemv_stream_geometry)
     int S = 1;
-    if (gemv_knee(kPipeStream, n, k, num_sms, m_fit, 0, 1, &S) != FI_OK) S = 1;
+    if (gemv_knee(kPipeStream, n, k, num_sms, m_fit, 0, 0, &S) != FI_OK) S = 1;
     return FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeStream << 4);
   }
   return FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
@@ -235,7 +242,7 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
     return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV tactics support m <= %d (got m=%lld)",
                      kGemvMaxM, (long long)m);
   const int64_t C = k / kChunkK;
-  const int ctas = ctas_req ? ctas_req : 1;
+  const int ctas = ctas_req;  // 0 = the pipeline's automatic choice
   const int rsel = var & 0xF;
   const bool pipe_auto = (var >> 4) == kPipeAuto;
   int pipe = pipe_auto ? kPipeStream : var >> 4;
@@ -255,9 +262,9 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
     g.pipeline = pipe;
     g.S = 1;
     g.RS = 1;
-    g.ctas_per_sm = ctas;
+    g.ctas_per_sm = ctas ? ctas : 1;
     g.grid_x = 1;
-    g.threads = pipe == kPipeRing ? kGemvThreads : kStreamThreads;
+    g.threads = pipe == kPipeRing ? kGemvThreads : kStreamMaxThreads;
   } else {
     int rc = geometry_for(pipe, m, n, k, S, rsel, ctas, sms, &g);
     // the automatic pipeline takes the ring (a whole SM's shared memory) when the activations
@@ -424,6 +431,7 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.rows_per_stage = g.RS;
     a.stages = g.stages;
     a.grid_x = g.grid_x;
+    a.threads = g.threads;
     a.pdl = 1;
     a.debug_stall = g_debug_stall_launches > 0 ? 1 : 0;
     if (g_debug_stall_launches > 0) --g_debug_stall_launches;

@@ -133,46 +133,65 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+__device__ __forceinline__ void stage_block(const uint4 v0, const uint4 v1, int r, int b, int GA, int blocks_per_row,
+                                            uint4* Ah4, float* As) {
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  uint32_t e = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    e = max(e, (w[i] >> 7) & 0xFFu);
+    e = max(e, (w[i] >> 23) & 0xFFu);
+  }
+  int sh = 141 - (int)e;  // biased exponent E -> block maximum in [2^14, 2^15)
+  sh = sh < -126 ? -126 : (sh > 126 ? 126 : sh);
+  const float up = __uint_as_float((uint32_t)(sh + 127) << 23);
+  const float down = __uint_as_float((uint32_t)(127 - sh) << 23);
+  uint32_t h[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float lo = __uint_as_float(w[i] << 16) * up;
+    const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * up;
+    h[i] = f32x2_to_f16x2(lo, hi);
+  }
+  const int c = b >> 1, half = b & 1;
+  uint4* dst = Ah4 + ((int64_t)(r * GA + c / 32) * 4 + 2 * half) * 32 + (c % 32);
+  dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
+  dst[32] = make_uint4(h[4], h[5], h[6], h[7]);
+  As[r * blocks_per_row + b] = down;
+}
+
 // Stage A[0:m, kbase : kbase + 32*nch] for the consumer warps. Layout for conflict-free reads:
 // chunk c (32 k) of row r is 4 16-byte quads at uint4 index ((r * GA + c / 32) * 4 + q) * 32 +
 // c % 32 (GA = ceil(nch / 32)), so a warp reading 32 consecutive chunks touches 512
 // contiguous bytes per quad. Values are f16 scaled by a power of two per 16-block that puts
-// the block maximum in [2^14, 2^15); As[r][b] holds the inverse scale.
+// the block maximum in [2^14, 2^15); As[r][b] holds the inverse scale. A thread loads up to four
+// of its blocks before converting any, so their global-memory latencies overlap.
 __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A, int64_t k, int m,
                                                   int64_t kbase, int nch, uint4* Ah4, float* As, int tid,
                                                   int nthreads) {
   const int GA = (nch + 31) / 32;
   const int blocks_per_row = nch * 2;
   const int nblk = m * blocks_per_row;
-  for (int bi = tid; bi < nblk; bi += nthreads) {
-    const int r = bi / blocks_per_row;
-    const int b = bi - r * blocks_per_row;
-    const uint16_t* src = A + (int64_t)r * k + kbase + (int64_t)b * 16;
-    const uint4 v0 = ldg_v4(src);
-    const uint4 v1 = ldg_v4(src + 8);
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t e = 0;
+  for (int b0 = tid; b0 < nblk; b0 += 4 * nthreads) {
+    uint4 v[4][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      e = max(e, (w[i] >> 7) & 0xFFu);
-      e = max(e, (w[i] >> 23) & 0xFFu);
+    for (int u = 0; u < 4; ++u) {
+      const int bi = b0 + u * nthreads;
+      if (bi < nblk) {
+        const int r = bi / blocks_per_row;
+        const uint16_t* src = A + (int64_t)r * k + kbase + (int64_t)(bi - r * blocks_per_row) * 16;
+        v[u][0] = ldg_v4(src);
+        v[u][1] = ldg_v4(src + 8);
+      }
     }
-    int sh = 141 - (int)e;  // biased exponent E -> block maximum in [2^14, 2^15)
-    sh = sh < -126 ? -126 : (sh > 126 ? 126 : sh);
-    const float up = __uint_as_float((uint32_t)(sh + 127) << 23);
-    const float down = __uint_as_float((uint32_t)(127 - sh) << 23);
-    uint32_t h[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float lo = __uint_as_float(w[i] << 16) * up;
-      const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * up;
-      h[i] = f32x2_to_f16x2(lo, hi);
+    for (int u = 0; u < 4; ++u) {
+      const int bi = b0 + u * nthreads;
+      if (bi < nblk) {
+        const int r = bi / blocks_per_row;
+        stage_block(v[u][0], v[u][1], r, bi - r * blocks_per_row, GA, blocks_per_row, Ah4, As);
+      }
     }
-    const int c = b >> 1, half = b & 1;
-    uint4* dst = Ah4 + ((int64_t)(r * GA + c / 32) * 4 + 2 * half) * 32 + (c % 32);
-    dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
-    dst[32] = make_uint4(h[4], h[5], h[6], h[7]);
-    As[r * blocks_per_row + b] = down;
   }
 }
 
@@ -556,93 +575,106 @@ __device__ __forceinline__ void item_rows(uint32_t code_s, uint32_t scale_s, con
 }
 
 template <int MT, int R, int NS>
-__global__ void __launch_bounds__(kStreamThreads, 2) gemv_stream_kernel(GemvArgs p) {
+__global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_stream_kernel(GemvArgs p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr uint32_t kSlot = (uint32_t)R * kStreamSlotBytesPerRow;
+  constexpr int TI = kStreamIters;  // chunk iterations per work item
+  constexpr uint32_t kSlot = (uint32_t)(TI * R) * kStreamCellBytes;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
+  const int NW = (int)(blockDim.x >> 5);
   const int m = (int)p.m;
   const int64_t n = p.n, k = p.k;
   const int S = p.splits;
   const int s = blockIdx.y;
 
-  // K range of this split, in 32-k chunks, and the chunk iterations of a row
+  // K range of this split, in 32-k chunks; chunk iterations of a row; items of a row group
   const int64_t C = k / kChunkK;
   const int64_t c0 = (int64_t)s * C / S;
   const int nch = (int)((int64_t)(s + 1) * C / S - c0);
   const int T = (nch + 31) / 32;
+  const int TT = (T + TI - 1) / TI;
 
-  // rows of this warp (balanced over all warps of the split), R per group
-  const int64_t GW = (int64_t)gridDim.x * kStreamWarps;
-  const int64_t gw = (int64_t)blockIdx.x * kStreamWarps + warp;
-  const int64_t r_lo = gw * n / GW, r_hi = (gw + 1) * n / GW;
-  const int64_t Q = (r_hi - r_lo + R - 1) / R * T;  // items of this warp
+  // rows of this warp: whole groups of R rows, balanced over all warps of the split (only the
+  // matrix's last group can be partial)
+  const int64_t GW = (int64_t)gridDim.x * NW;
+  const int64_t gw = (int64_t)blockIdx.x * NW + warp;
+  const int64_t ngr = (n + R - 1) / R;
+  const int64_t g_lo = gw * ngr / GW, g_hi = (gw + 1) * ngr / GW;
+  const int64_t r_lo = g_lo * R, r_hi = min(n, g_hi * R);
+  const int Q = (int)(g_hi - g_lo) * TT;  // items of this warp
 
   const int64_t rs_q = k / 2, rs_s = k / 16;
   const uint8_t* const ws_end = p.Ws + n * rs_s;
   const uint32_t a_s = smem_addr(smem), as_s = smem_addr(smem + p.off_as);
+  // this warp's ring: NS slots; in a slot, the cell of (iteration ti, row i) for lane L at
+  // (ti*R + i)*512 + L*16, and its scale word at TI*R*512 + (ti*R + i)*128 + L*4
   const uint32_t ring = smem_addr(smem + p.off_ring) + (uint32_t)warp * NS * kSlot;
   const uint32_t my_code = ring + (uint32_t)lane * 16;
-  const uint32_t my_scale = ring + (uint32_t)R * 512 + (uint32_t)lane * 4;
+  const uint32_t my_scale = ring + (uint32_t)(TI * R) * 512 + (uint32_t)lane * 4;
   const int64_t lane_k = (c0 + lane) * 2;  // the lane's first scale byte within a row's split
 
   pdl_launch_dependents();
 
-  // ---- issue cursor: item iq = (group ig, iteration it); row pointers advance per item
-  int64_t ig = 0, iq = 0;
-  int it = 0;
-  const uint8_t* qsrc[R];  // row i's code cell for this lane at iteration it
-  const uint8_t* ssrc[R];  // the 4-byte aligned word holding the lane's two scale bytes
+  // ---- issue cursor: item iq = (group ig, item itt of the row group). One code pointer and
+  // one scale pointer (row j0 of the group, this lane's cell at the item's first iteration)
+  // advance by TI*512 and TI*64 bytes per item; row i adds i * k/2 to the code pointer and a
+  // per-group offset to the scale pointer (the 4-byte aligned word with the lane's two bytes).
+  const uint32_t rsq = (uint32_t)rs_q;
+  int ig = 0, itt = 0, iq = 0;
+  const uint8_t* qp = nullptr;
+  const uint8_t* sp = nullptr;
+  uint32_t sdel[R];
   int irows = 0;
-  bool ifast = true;  // a full group that cannot reach the tensor's last scale bytes
+  bool iedge = false;  // the group holds the tensor's last scale pair and its size is 2 mod 4
   auto issue_group = [&]() {
-    const int64_t j0 = r_lo + ig * R;
+    const int64_t j0 = r_lo + (int64_t)ig * R;
     irows = (int)max((int64_t)0, min((int64_t)R, r_hi - j0));
+    const int64_t x0 = j0 * rs_s + lane_k;
+    qp = p.Wq + j0 * rs_q + (c0 + lane) * 16;
+    sp = p.Ws + (x0 & ~(int64_t)3);
 #pragma unroll
-    for (int i = 0; i < R; ++i) {
-      const int64_t j = j0 + i;
-      qsrc[i] = p.Wq + j * rs_q + (c0 + lane) * 16;
-      ssrc[i] = p.Ws + ((j * rs_s + lane_k) & ~(int64_t)3);
-    }
-    ifast = irows == R && !((n * rs_s) % 4 != 0 && j0 + R >= n);
+    for (int i = 0; i < R; ++i) sdel[i] = (uint32_t)(((x0 + i * rs_s) & ~(int64_t)3) - (x0 & ~(int64_t)3));
+    iedge = (n * rs_s) % 4 != 0 && j0 + irows >= n;
   };
-  // copy item iq into slot u; always commits one group (empty past the warp's last item) so
-  // that wait_group counts stay uniform
-  auto issue = [&](int u) {
+  // copy item iq into the slot at byte offset uo; always commits one group (empty past the
+  // warp's last item) so that wait_group counts stay uniform
+  auto issue = [&](uint32_t uo) {
     if (iq < Q) {
-      if (it * 32 + lane < nch) {
-        const uint32_t cdst = my_code + (uint32_t)u * kSlot;
-        const uint32_t sdst = my_scale + (uint32_t)u * kSlot;
-        if (ifast) {
+      const int t0 = itt * TI;
 #pragma unroll
-          for (int i = 0; i < R; ++i) {
-            cp_async_16(cdst + (uint32_t)(i * 512), qsrc[i]);
-            cp_async_4(sdst + (uint32_t)(i * 128), ssrc[i]);
-          }
-        } else {
+      for (int ti = 0; ti < TI; ++ti) {
+        if ((t0 + ti) * 32 + lane < nch) {
+          const uint32_t cdst = my_code + uo + (uint32_t)(ti * R * 512);
+          const uint32_t sdst = my_scale + uo + (uint32_t)(ti * R * 128);
+          if (irows == R && !iedge) {
 #pragma unroll
-          for (int i = 0; i < R; ++i) {
-            if (i < irows) {
-              cp_async_16(cdst + (uint32_t)(i * 512), qsrc[i]);
-              if (ssrc[i] + 4 <= ws_end) {
-                cp_async_4(sdst + (uint32_t)(i * 128), ssrc[i]);
-              } else {  // the tensor's last scale pair when its size is 2 mod 4: plain load
-                const uint32_t off = (uint32_t)(((r_lo + ig * R + i) * rs_s + lane_k) & 2);
-                sts_u16(sdst + (uint32_t)(i * 128) + off, ldg_stream_u16(ssrc[i] + off));
+            for (int i = 0; i < R; ++i) {
+              cp_async_16(cdst + (uint32_t)(i * 512), qp + i * rsq + ti * 512);
+              cp_async_4(sdst + (uint32_t)(i * 128), sp + sdel[i] + ti * 64);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+              if (i < irows) {
+                cp_async_16(cdst + (uint32_t)(i * 512), qp + i * rsq + ti * 512);
+                const uint8_t* w = sp + sdel[i] + ti * 64;
+                if (w + 4 <= ws_end) {
+                  cp_async_4(sdst + (uint32_t)(i * 128), w);
+                } else {  // the tensor's last scale pair when its size is 2 mod 4: plain load
+                  const uint32_t off = (uint32_t)(((r_lo + (int64_t)ig * R + i) * rs_s + lane_k) & 2);
+                  sts_u16(sdst + (uint32_t)(i * 128) + off, ldg_stream_u16(w + off));
+                }
               }
             }
           }
         }
       }
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        qsrc[i] += 512;
-        ssrc[i] += 64;
-      }
+      qp += TI * 512;
+      sp += TI * 64;
       ++iq;
-      if (++it == T) {
-        it = 0;
+      if (++itt == TT) {
+        itt = 0;
         ++ig;
         issue_group();
       }
@@ -653,12 +685,12 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_stream_kernel(GemvArgs
   // prologue: the first NS items (weights only: they do not depend on the preceding kernel)
   issue_group();
 #pragma unroll
-  for (int u = 0; u < NS; ++u) issue(u);
+  for (int u = 0; u < NS; ++u) issue((uint32_t)u * kSlot);
 
   pdl_wait();
   const int GA = (nch + 31) / 32;
   stage_activations(p.A, k, m, c0 * kChunkK, nch, reinterpret_cast<uint4*>(smem),
-                    reinterpret_cast<float*>(smem + p.off_as), tid, kStreamThreads);
+                    reinterpret_cast<float*>(smem + p.off_as), tid, (int)blockDim.x);
   __syncthreads();
   const float g = (S == 1) ? *p.gscale : 1.0f;
 
@@ -669,31 +701,36 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_stream_kernel(GemvArgs
 #pragma unroll
     for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
   int64_t j0 = r_lo;
-  int ct = 0, u = 0;
-  uint32_t soff[R];
+  int ctt = 0;
+  uint32_t uo = 0;  // byte offset of the slot being computed
+  uint32_t soff[R];  // 0 or 2: the lane's scale bytes within its word (the same for every chunk of a row)
 #pragma unroll
   for (int i = 0; i < R; ++i) soff[i] = (uint32_t)(((j0 + i) * rs_s + lane_k) & 2);
-  for (int64_t q = 0; q < Q; ++q) {
-    const int c = ct * 32 + lane;
+  for (int q = 0; q < Q; ++q) {
     cp_async_wait<NS - 1>();  // this lane's copies of item q have landed
-    if (c < nch)
-      item_rows<MT, R>(my_code + (uint32_t)u * kSlot, my_scale + (uint32_t)u * kSlot, soff, a_s, as_s, m, nch, GA, c,
-                       acc);
+    const int t0 = ctt * TI;
+#pragma unroll
+    for (int ti = 0; ti < TI; ++ti) {
+      const int c = (t0 + ti) * 32 + lane;
+      if (c < nch)
+        item_rows<MT, R>(my_code + uo + (uint32_t)(ti * R * 512), my_scale + uo + (uint32_t)(ti * R * 128), soff,
+                         a_s, as_s, m, nch, GA, c, acc);
+    }
     // refill the slot just read with item q + NS (the reads above are complete: their
     // results have been consumed)
-    issue(u);
-    if (++ct == T) {
+    issue(uo);
+    if (++ctt == TT) {
       finish_rows<MT, R>(acc, p, j0, (int)min((int64_t)R, r_hi - j0), m, S, s, g, lane, true);
 #pragma unroll
       for (int i = 0; i < R; ++i)
 #pragma unroll
         for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
-      ct = 0;
+      ctt = 0;
       j0 += R;
 #pragma unroll
       for (int i = 0; i < R; ++i) soff[i] = (uint32_t)(((j0 + i) * rs_s + lane_k) & 2);
     }
-    u = (u + 1 == NS) ? 0 : u + 1;
+    uo = (uo == (uint32_t)(NS - 1) * kSlot) ? 0u : uo + kSlot;
   }
   cp_async_wait<0>();
 }
@@ -735,13 +772,13 @@ int launch_stream_one(const GemvArgs& a, cudaStream_t stream) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return set_cuda_error("cudaGetDevice");
   if (!configured[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) != cudaSuccess)
       return set_cuda_error("cudaFuncSetAttribute(gemv stream smem)");
     configured[dev] = 1;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)a.grid_x, (unsigned)a.splits);
-  cfg.blockDim = dim3(kStreamThreads);
+  cfg.blockDim = dim3((unsigned)a.threads);
   cfg.dynamicSmemBytes = (size_t)a.smem_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -28,11 +28,11 @@ constexpr int kSmemBudget = 227 * 1024 - 1024;             // dynamic shared mem
 constexpr int kGemvMaxStages = 16;
 constexpr int kGemvStageTarget = 16 * 1024;                // preferred bytes per ring stage
 
-// The per-warp async-copy pipeline: 8 warps per CTA, every CTA at most half an SM.
-constexpr int kStreamWarps = 8;
-constexpr int kStreamThreads = kStreamWarps * 32;
-constexpr int kStreamSlotBytesPerRow = 32 * 16 + 32 * 4;   // a row's code cells + scale words
-constexpr int kStreamSmemBudget = 228 * 1024 / 2 - 1024;   // two CTAs per SM
+// The per-warp async-copy pipeline: one CTA of 16 warps per SM, or two of 8 warps.
+constexpr int kStreamMaxThreads = 512;
+constexpr int kStreamIters = 2;                            // chunk iterations per work item
+constexpr int kStreamCellBytes = 32 * 16 + 32 * 4;         // one iteration of one row: code cells + scale words
+constexpr int kStreamHalfBudget = 228 * 1024 / 2 - 1024;   // dynamic shared memory per CTA, two CTAs per SM
 // pipelines (the high nibble of the GEMV tactic variant)
 constexpr int kPipeAuto = 0, kPipeStream = 1, kPipeRing = 2;
 
@@ -83,6 +83,7 @@ struct GemvArgs {
   int rows_per_stage;  // RS: consecutive weight rows per ring stage (one consumer warp each)
   int stages;          // NST: ring stages (stream pipeline: slots per warp)
   int grid_x;          // CTAs per split
+  int threads;         // threads per CTA
   int pdl;             // launch with programmatic stream serialization
   int debug_stall;     // test hook: the producer issues nothing (consumer waits time out)
   int64_t stage_bytes, off_as, off_bar, off_ring, smem_bytes;

@@ -49,9 +49,13 @@ def test_default_gemv_tactic_resolves_for_decode_shapes(n, k):
     assert 1 <= info["splits"] <= k // 32
     # one persistent wave: the grid never asks for more CTAs than the SMs hold
     assert info["grid_x"] * info["grid_y"] <= B200_SMS * info["ctas_per_sm"]
-    # the default runs the per-warp async-copy pipeline: 8 warps, at most half an SM
+    # the default runs the per-warp async-copy pipeline: one CTA of 16 warps per SM, or two
+    # of 8 warps within half an SM each
     assert info["variant"] >> 4 == 1
-    assert info["threads"] == 8 * 32 and 0 < info["smem_bytes"] <= 228 * 1024 // 2 - 1024
+    if info["ctas_per_sm"] == 1:
+        assert info["threads"] == 16 * 32 and 0 < info["smem_bytes"] <= 227 * 1024 - 1024
+    else:
+        assert info["threads"] == 8 * 32 and 0 < info["smem_bytes"] <= 228 * 1024 // 2 - 1024
     assert info["workspace_bytes"] == (info["splits"] * n * 4 if info["splits"] > 1 else 0)
 
 
@@ -117,7 +121,8 @@ def test_workspace_bytes():
     (5, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),        # two rows per stage above m = 4
     (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x32), -1),     # pipeline 3
     (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x19), -1),     # rows 9 on the stream pipeline
-    (1, 8, 65536, fi.make_tactic(0, 1, 0, 2), -2),        # two 36 KB rows per stage do not fit twice
+    (1, 8, 65536, fi.make_tactic(0, 1, 0, 0x22), -2),     # ring: two 36 KB rows per stage do not fit twice
+    (1, 8, 65536, fi.make_tactic(0, 1, 2, 0x11), -2),     # stream, half-SM CTAs: 128 KB of activations
 ])
 def test_resolve_rejects(m, n, k, tactic, status):
     with pytest.raises(fi.FiError) as e:
