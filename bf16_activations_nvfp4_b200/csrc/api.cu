@@ -287,6 +287,28 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
   return FI_OK;
 }
 
+// MMA tactic: splits 0 or 1 (one split), CTAs per SM 0 or 1, variant 0. Needs m <= 256 and k a
+// multiple of 64; the workspace holds the f16 activations and their row scales.
+static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var, fi_tactic_info* out) {
+  if (m > kMmaMaxM)
+    return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA tactics support m <= %d (got m=%lld)", kMmaMaxM, (long long)m);
+  if (k % kMmaKStep != 0)
+    return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA tactics need k to be a multiple of %d (got k=%lld)", kMmaKStep,
+                     (long long)k);
+  if (S_req > 1 || ctas_req > 1 || var != 0)
+    return set_error(FI_ERR_INVALID_ARG, "MMA tactics take splits 0/1, CTAs per SM 0/1 and variant 0");
+  out->kind = FI_KIND_MMA;
+  out->splits = 1;
+  out->ctas_per_sm = 1;
+  out->variant = 0;
+  out->grid_x = (int32_t)std::max<int64_t>(1, (n + kMmaTileRows - 1) / kMmaTileRows);
+  out->grid_y = 1;
+  out->threads = kMmaThreads;
+  out->smem_bytes = (int32_t)mma_smem_bytes();
+  out->workspace_bytes = (m > 0 && k > 0) ? mma_workspace_bytes(m, k) : 0;
+  return FI_OK;
+}
+
 static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms, fi_tactic_info* out) {
   if (m < 0 || n < 0 || k < 0) return set_error(FI_ERR_INVALID_ARG, "negative size");
   if (k % 32 != 0) return set_error(FI_ERR_UNSUPPORTED_SHAPE, "k=%lld is not a multiple of 32", (long long)k);
@@ -300,8 +322,7 @@ static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms,
   const int var = FI_TACTIC_VARIANT(tactic);
   memset(out, 0, sizeof(*out));
   if (kind == FI_KIND_GEMV) return resolve_gemv(m, n, k, S, ctas, var, num_sms, out);
-  if (kind == FI_KIND_MMA)
-    return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA tactics are not available in this build");
+  if (kind == FI_KIND_MMA) return resolve_mma(m, n, k, S, ctas, var, out);
   return set_error(FI_ERR_INVALID_ARG, "unknown tactic kind %d", kind);
 }
 
@@ -444,7 +465,28 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     rc = launch_gemv(a, stream);
     if (rc != FI_OK) return rc;
   } else {
-    return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA tactics are not available in this build");
+    MmaArgs a;
+    memset(&a, 0, sizeof(a));
+    a.A = A;
+    a.Wq = Wq;
+    a.Ws = Wscale;
+    a.gscale = gscale;
+    a.out = out;
+    uint8_t* ws = reinterpret_cast<uint8_t*>(partials);
+    a.a16 = reinterpret_cast<uint16_t*>(ws);
+    a.rs = reinterpret_cast<float*>(ws + mma_rs_offset(m, k));
+    a.m = m;
+    a.n = n;
+    a.k = k;
+    a.m_pad = mma_m_pad(m);
+    a.debug_stall = g_debug_stall_launches > 0 ? 1 : 0;
+    if (g_debug_stall_launches > 0) --g_debug_stall_launches;
+    a.err = device_error_word();
+    if (!a.err) return set_cuda_error("cudaGetSymbolAddress(device error word)");
+    a.timeout_ns = g_wait_timeout_ns;
+    rc = launch_mma(a, stream);
+    if (rc != FI_OK) return rc;
+    return FI_OK;
   }
   if (info.splits > 1) return launch_splitk_reduce(partials, info.splits, m, n, gscale, out, true, stream);
   return FI_OK;
@@ -527,6 +569,7 @@ int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, 
     for (int R : {0, 1, 2})
       for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, R | (pipe << 4));
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 2, kPipeStream << 4);
+  cand[nc++] = FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
   fi_tactic_info seen[64];
   int nseen = 0, count = 0;
   for (int c = 0; c < nc; ++c) {

@@ -40,6 +40,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "sync.cuh"
 
 namespace fi {
 
@@ -49,58 +50,10 @@ __device__ unsigned int g_gemv_error = 0;
 
 namespace {
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-               : "memory");
-}
-
-// One bounded, suspending test of the phase: the thread sleeps in hardware until the phase
-// completes or kWaitSliceNs pass, so waiting warps do not spin on the issue slots the
-// computing warps need.
-constexpr uint32_t kWaitSliceNs = 20000;
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(kWaitSliceNs)
-      : "memory");
-  return done != 0;
-}
-
-// Wait for phase `parity` of `bar` to complete. Returns false (and raises the abort flag and
-// the device error bit) if it has not after timeout_ns, or at once if the CTA has aborted.
+// Wait for phase `parity` of `bar` (bounded; see sync.cuh), recording timeouts in g_gemv_error.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                   uint64_t timeout_ns, unsigned err_bit) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > timeout_ns) {
-      *abort_flag = 1;
-      atomicOr(&g_gemv_error, err_bit);
-      return false;
-    }
-  }
+  return fi::mbar_wait_bounded(bar, parity, abort_flag, timeout_ns, &g_gemv_error, err_bit);
 }
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -851,6 +804,21 @@ int launch_gemv(const GemvArgs& a, cudaStream_t stream) {
   if (a.m <= 16) return launch_mt<16>(a, stream);
   if (a.m <= 32) return launch_mt<32>(a, stream);
   return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV supports m <= %d", kGemvMaxM);
+}
+
+unsigned* device_error_word() {
+  static unsigned* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gemv_error) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = static_cast<unsigned*>(p);
+  }
+  return addr[dev];
 }
 
 int gemv_read_error(unsigned* bits) {

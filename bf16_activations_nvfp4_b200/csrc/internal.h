@@ -92,6 +92,37 @@ struct GemvArgs {
 int launch_gemv(const GemvArgs& a, cudaStream_t stream);
 int gemv_read_error(unsigned* bits);
 
+// ------------------------------------------------------------------------- MMA
+// Tensor-core path: one CTA per kMmaTileRows weight rows, 64 k per pipeline step, activations
+// converted to f16 (times a per-row power of two) in the workspace: a16 [m_pad, k] then
+// rs [m_pad] fp32 at the next 256-byte boundary.
+constexpr int kMmaTileRows = 256;
+constexpr int kMmaKStep = 64;
+constexpr int kMmaMaxM = 256;
+constexpr int kMmaThreads = 14 * 32;
+inline int mma_m_pad(int64_t m) { return (int)((m + 15) / 16 * 16); }
+inline int64_t mma_rs_offset(int64_t m, int64_t k) { return round_up((int64_t)mma_m_pad(m) * k * 2, 256); }
+inline int64_t mma_workspace_bytes(int64_t m, int64_t k) { return mma_rs_offset(m, k) + (int64_t)mma_m_pad(m) * 4; }
+int64_t mma_smem_bytes();
+
+struct MmaArgs {
+  const uint16_t* A;
+  const uint8_t* Wq;
+  const uint8_t* Ws;
+  const float* gscale;
+  uint16_t* out;
+  uint16_t* a16;  // workspace: f16 activations [m_pad, k]
+  float* rs;      // workspace: per-row inverse scales [m_pad]
+  int64_t m, n, k;
+  int m_pad;
+  int debug_stall;      // test hook: the producer issues nothing (the waits time out)
+  unsigned* err;        // the device error word
+  uint64_t timeout_ns;  // limit of every mbarrier wait
+};
+int launch_mma(const MmaArgs& a, cudaStream_t stream);
+// Device address of the sticky kernel error word on the current device (looked up once).
+unsigned* device_error_word();
+
 // ---------------------------------------------------------------------- reduce
 int launch_splitk_reduce(const float* partials, int splits, int64_t m, int64_t n,
                          const float* gscale, uint16_t* out, bool pdl, cudaStream_t stream);

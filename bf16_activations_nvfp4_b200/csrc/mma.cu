@@ -1,0 +1,465 @@
+// Tensor-core path for bf16 activations x NVFP4 weights (sm_100a, tcgen05 + TMA + TMEM).
+//
+// After PR #4038's MMA path (Description, "What it does": the GEMV reads the same packed
+// operands as the MMA kernel, so the tactic can pick either per shape), re-designed for B200:
+//
+//  * Operands. tcgen05.mma kind::f16 needs both operands of one 16-bit type. The weights are
+//    decoded to f16 (every E2M1 value times its E4M3 block scale is exact in f16: at most 6
+//    significant bits, magnitudes 2^-10 .. 2688); the activations are converted once per call
+//    by act_to_f16_kernel to f16 times a per-row power of two that puts the row maximum in
+//    [2^14, 2^15) (exact for every element within 2^29 of its row maximum), so the tensor core
+//    accumulates sum_k W'[i][k] * A'[j][k] in fp32 and one per-row factor undoes the scale.
+//  * Roles (one CTA per 256 weight rows, 14 warps):
+//      warp 0      TMA producer: raw codes of the tile (256 rows x 32 bytes per 64-k step) into
+//                  a 4-stage ring, issued before the grid-dependency wait (weights never depend
+//                  on the preceding kernel); f16 activation tiles (m_pad rows x 64 k, 128-byte
+//                  swizzled) into a 2-stage ring;
+//      warps 2-9   decode: one weight row per thread, codes -> f16 (cvt.rn.f16x2.e2m1x2) times
+//                  the block scale (exact f16 multiply), stored in the 128-byte-swizzled
+//                  K-major layout the MMA reads;
+//      warp 1      TMEM allocation and, from one thread, the MMAs: per 64-k step 4 K=16 steps x
+//                  2 M=128 halves, N = m_pad, accumulating in TMEM; tcgen05.commit frees the
+//                  stage;
+//      warps 10-13 epilogue: tcgen05.ld of the accumulator, out[j][i] = bf16_rn(D[i][j] *
+//                  rs[j] * gscale).
+//  * The weight tile is decoded once per call (the activations, m_pad <= 256 rows, are one MMA
+//    N tile), so the decode work is one cvt and one f16 multiply per two codes.
+//  * Every wait is bounded (see sync.cuh); on a timeout the roles stop, the MMA issuer and the
+//    producer drain what they issued, and TMEM is freed before the CTA exits.
+//
+// Arithmetic order: fixed by k (64-k steps in order, K=16 sub-steps in order) and independent
+// of m, so for a fixed tactic a row's bits do not depend on m (an output element depends only
+// on its weight row and activation row); results are deterministic run to run.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sync.cuh"
+
+namespace fi {
+
+namespace {
+
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpDq0 = 2, kDqWarps = 8, kWarpEpi0 = 10, kEpiWarps = 4;
+static_assert((kWarpEpi0 + kEpiWarps) * 32 == kMmaThreads, "warp roles cover the CTA");
+static_assert(kWarpDq0 + kDqWarps == kWarpEpi0 && kDqWarps * 32 == kMmaTileRows, "one decode thread per tile row");
+constexpr int kOpStages = 2, kRawStages = 4;
+constexpr uint32_t kWopBytes = kMmaTileRows * 128;  // 256 rows x 64 f16, 128-byte swizzled
+constexpr uint32_t kActBytes = 256 * 128;           // up to 256 activation rows x 64 f16
+constexpr uint32_t kStageBytes = kWopBytes + kActBytes;
+constexpr uint32_t kRawBytes = kMmaTileRows * 32;   // 256 rows x 32 code bytes
+// barriers: raw_full, raw_empty, act_full, op_full, op_empty, tmem_full, drain
+constexpr int kNumBars = 2 * kRawStages + 3 * kOpStages + 2;
+constexpr uint32_t kBarOff = kOpStages * kStageBytes + kRawStages * kRawBytes;
+
+// Shared-memory matrix descriptor of a K-major tile with 128-byte rows in the 128-byte swizzle
+// (8-row atoms of 1024 bytes): start address >> 4 in bits 0-13, leading-dimension offset 1
+// (unused for swizzled K-major), stride-dimension offset 1024 >> 4 in bits 32-45, descriptor
+// version 1 in bits 46-47, swizzle mode 2 (128 bytes) in bits 61-63.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), f16 A and B (bits 7-9,
+// 10-12 = 0), both K-major, N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+__device__ __forceinline__ uint32_t f16_idesc(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
+      "[%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds_v4m(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Wait that ignores the abort flag (used to drain copies and MMAs in flight before exit).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, unsigned* err) {
+  volatile int never = 0;
+  mbar_wait_bounded(bar, parity, &never, timeout_ns, err, 8u);
+}
+
+}  // namespace
+
+// A[m, k] bf16 -> a16[m_pad, k] f16 scaled by a per-row power of two (row maximum in
+// [2^14, 2^15)); rs[row] = the inverse scale. Rows m .. m_pad-1 are zero.
+__global__ void __launch_bounds__(256) act_to_f16_kernel(const uint16_t* __restrict__ A, int64_t m, int64_t k,
+                                                         uint16_t* __restrict__ a16, float* __restrict__ rs) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t row = blockIdx.x;
+  const int tid = threadIdx.x;
+  uint4* dst = reinterpret_cast<uint4*>(a16 + row * k);
+  const int64_t n8 = k / 8;  // 16-byte groups of the row
+  if (row >= m) {
+    for (int64_t i = tid; i < n8; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
+    if (tid == 0) rs[row] = 0.0f;
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(A + row * k);
+  uint32_t e = 0;
+  for (int64_t i = tid; i < n8; i += blockDim.x) {
+    const uint4 v = ldg_v4(src + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) e = max(e, max((w[q] >> 7) & 0xFFu, (w[q] >> 23) & 0xFFu));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
+  __shared__ uint32_t red[8];
+  if ((tid & 31) == 0) red[tid >> 5] = e;
+  __syncthreads();
+  e = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) e = max(e, red[w]);
+  int sh = 141 - (int)e;  // biased exponent E of the row maximum -> [2^14, 2^15)
+  sh = sh < -126 ? -126 : (sh > 126 ? 126 : sh);
+  const float up = __uint_as_float((uint32_t)(sh + 127) << 23);
+  for (int64_t i = tid; i < n8; i += blockDim.x) {
+    const uint4 v = ldg_v4(src + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t h[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      h[q] = f32x2_to_f16x2(__uint_as_float(w[q] << 16) * up, __uint_as_float(w[q] & 0xFFFF0000u) * up);
+    dst[i] = make_uint4(h[0], h[1], h[2], h[3]);
+  }
+  if (tid == 0) rs[row] = __uint_as_float((uint32_t)(127 - sh) << 23);
+}
+
+__global__ void __launch_bounds__(kMmaThreads, 1)
+    mma_nvfp4_kernel(const MmaArgs p, const __grid_constant__ CUtensorMap tmap_a,
+                     const __grid_constant__ CUtensorMap tmap_w) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ volatile int abort_flag;
+  __shared__ uint32_t tmem_slot;
+  // 1024-byte aligned base for the swizzled tiles
+  const uint32_t raw_s = smem_addr(smem_raw);
+  const uint32_t base = (raw_s + 1023u) & ~1023u;
+  uint8_t* const basep = smem_raw + (base - raw_s);
+  uint64_t* const bars = reinterpret_cast<uint64_t*>(basep + kBarOff);
+  uint64_t* const raw_full = bars;
+  uint64_t* const raw_empty = bars + kRawStages;
+  uint64_t* const act_full = bars + 2 * kRawStages;
+  uint64_t* const op_full = act_full + kOpStages;
+  uint64_t* const op_empty = op_full + kOpStages;
+  uint64_t* const tmem_full = op_empty + kOpStages;
+  uint64_t* const drain = tmem_full + 1;
+  auto wop_addr = [&](int st) { return base + (uint32_t)st * kStageBytes; };
+  auto act_addr = [&](int st) { return base + (uint32_t)st * kStageBytes + kWopBytes; };
+  auto raw_addr = [&](int st) { return base + kOpStages * kStageBytes + (uint32_t)st * kRawBytes; };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t n = p.n, k = p.k;
+  const int m = (int)p.m, N = p.m_pad;
+  const int KS = (int)(k / kMmaKStep);
+  const int64_t w0 = (int64_t)blockIdx.x * kMmaTileRows;
+  const uint32_t ncols = N <= 16 ? 32u : (N <= 64 ? 128u : (N <= 128 ? 256u : 512u));  // >= 2N, a power of two
+
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < kRawStages; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], kDqWarps);
+    }
+    for (int i = 0; i < kOpStages; ++i) {
+      mbar_init(&act_full[i], 1);
+      mbar_init(&op_full[i], kDqWarps);
+      mbar_init(&op_empty[i], 1);
+    }
+    mbar_init(tmem_full, 1);
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kWarpMma) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&tmem_slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = tmem_slot;
+  pdl_launch_dependents();
+
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------------------ producer
+    if (lane == 0 && !p.debug_stall) {
+      int raw_issued = 0, act_issued = 0;
+      const int pro = KS < kRawStages ? KS : kRawStages;
+      for (int s = 0; s < pro; ++s) {
+        mbar_arrive_expect_tx(&raw_full[s], kRawBytes);
+        tma_load_2d(raw_addr(s), &tmap_w, s * 32, (int)w0, smem_addr(&raw_full[s]));
+        ++raw_issued;
+      }
+      pdl_wait();
+      for (int s = 0; s < KS && !abort_flag; ++s) {
+        const int os = s % kOpStages;
+        if (s >= kOpStages &&
+            !mbar_wait_bounded(&op_empty[os], (uint32_t)((s / kOpStages - 1) & 1), &abort_flag, p.timeout_ns, p.err, 2u))
+          break;
+        mbar_arrive_expect_tx(&act_full[os], (uint32_t)N * 128u);
+        tma_load_2d(act_addr(os), &tmap_a, s * kMmaKStep, 0, smem_addr(&act_full[os]));
+        ++act_issued;
+        const int sn = s + kRawStages;
+        if (sn < KS) {
+          const int rs = s % kRawStages;
+          if (!mbar_wait_bounded(&raw_empty[rs], (uint32_t)((s / kRawStages) & 1), &abort_flag, p.timeout_ns, p.err,
+                                 2u))
+            break;
+          mbar_arrive_expect_tx(&raw_full[rs], kRawBytes);
+          tma_load_2d(raw_addr(rs), &tmap_w, sn * 32, (int)w0, smem_addr(&raw_full[rs]));
+          ++raw_issued;
+        }
+      }
+      // drain: every copy issued must have landed before the CTA exits
+      for (int s = raw_issued - kRawStages < 0 ? 0 : raw_issued - kRawStages; s < raw_issued; ++s)
+        drain_wait(&raw_full[s % kRawStages], (uint32_t)((s / kRawStages) & 1), p.timeout_ns, p.err);
+      for (int s = act_issued - kOpStages < 0 ? 0 : act_issued - kOpStages; s < act_issued; ++s)
+        drain_wait(&act_full[s % kOpStages], (uint32_t)((s / kOpStages) & 1), p.timeout_ns, p.err);
+    }
+  } else if (warp >= kWarpDq0 && warp < kWarpDq0 + kDqWarps) {
+    // -------------------------------------------------------------------------- decode
+    const int r = tid - kWarpDq0 * 32;  // weight row of the tile, 0 .. 255
+    const int64_t row = w0 + r;
+    const bool valid = row < n;
+    const int64_t rs_s = k / 16;
+    const uint8_t* srow = p.Ws + (valid ? row : 0) * rs_s;
+    const uint32_t wdst = (uint32_t)(r >> 7) * (kWopBytes / 2) + (uint32_t)(r & 127) * 128u;
+    const uint32_t swz = (uint32_t)(r & 7);
+    for (int s = 0; s < KS; ++s) {
+      const int rsn = s % kRawStages, os = s % kOpStages;
+      const uint32_t sc4 = valid ? *reinterpret_cast<const uint32_t*>(srow + s * 4) : 0u;
+      // every lane waits; the warp continues only if all of them saw both phases (a timeout is
+      // seen lane by lane, and the warp must stay converged for __syncwarp below)
+      const bool ok =
+          mbar_wait_bounded(&raw_full[rsn], (uint32_t)((s / kRawStages) & 1), &abort_flag, p.timeout_ns, p.err, 1u) &&
+          (s < kOpStages || mbar_wait_bounded(&op_empty[os], (uint32_t)((s / kOpStages - 1) & 1), &abort_flag,
+                                              p.timeout_ns, p.err, 1u));
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const uint4 c0 = lds_v4m(raw_addr(rsn) + (uint32_t)r * 32u);
+      const uint4 c1 = lds_v4m(raw_addr(rsn) + (uint32_t)r * 32u + 16u);
+      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      const uint32_t dst = wop_addr(os) + wdst;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {  // 16-k block b: words 2b, 2b+1; chunks 2b, 2b+1 of the row
+        const uint32_t sf2 = e4m3x2_to_f16x2(__byte_perm(sc4, 0u, (uint32_t)(b | (b << 4))));
+        uint32_t h[8];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const uint32_t wd = words[2 * b + q];
+          h[4 * q + 0] = hmul2(e2m1x2_byte_to_f16x2<0>(wd), sf2);
+          h[4 * q + 1] = hmul2(e2m1x2_byte_to_f16x2<1>(wd), sf2);
+          h[4 * q + 2] = hmul2(e2m1x2_byte_to_f16x2<2>(wd), sf2);
+          h[4 * q + 3] = hmul2(e2m1x2_byte_to_f16x2<3>(wd), sf2);
+        }
+        sts_v4(dst + ((((uint32_t)(2 * b)) ^ swz) << 4), h[0], h[1], h[2], h[3]);
+        sts_v4(dst + ((((uint32_t)(2 * b + 1)) ^ swz) << 4), h[4], h[5], h[6], h[7]);
+      }
+      // make the generic-proxy stores visible to the tensor core (async proxy)
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&op_full[os]);
+        mbar_arrive(&raw_empty[rsn]);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ----------------------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idesc = f16_idesc(128, N);
+      for (int s = 0; s < KS; ++s) {
+        const int os = s % kOpStages;
+        const uint32_t par = (uint32_t)((s / kOpStages) & 1);
+        if (!mbar_wait_bounded(&act_full[os], par, &abort_flag, p.timeout_ns, p.err, 4u)) break;
+        if (!mbar_wait_bounded(&op_full[os], par, &abort_flag, p.timeout_ns, p.err, 4u)) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+        for (int kk = 0; kk < kMmaKStep / 16; ++kk) {
+          const uint64_t bdesc = sw128_desc(act_addr(os) + (uint32_t)kk * 32u);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint64_t adesc = sw128_desc(wop_addr(os) + (uint32_t)h * (kWopBytes / 2) + (uint32_t)kk * 32u);
+            umma_f16(tmem + (uint32_t)(h * N), adesc, bdesc, idesc, (s | kk) != 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(&op_empty[os]);  // frees the stage when these MMAs have read it
+      }
+      umma_commit(tmem_full);  // the accumulator is complete when every MMA issued has finished
+      umma_commit(drain);
+      drain_wait(drain, 0, p.timeout_ns, p.err);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------------ epilogue
+    pdl_wait();
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int i = q * 32 + lane;
+    // warp-uniform: the TMEM loads below are collective over the warp
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(tmem_full, 0, &abort_flag, p.timeout_ns, p.err, 16u) &&
+                                                !abort_flag);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (ok) {
+      const float g = *p.gscale;
+      for (int h = 0; h < 2; ++h) {
+        const int64_t row = w0 + h * 128 + i;
+        for (int j0 = 0; j0 < N; j0 += 16) {
+          float v[16];
+          tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * N + j0), v);
+          if (row < n) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int j = j0 + jj;
+              if (j < m) p.out[(int64_t)j * n + row] = f32_to_bf16_rn(__fmul_rn(__fmul_rn(v[jj], p.rs[j]), g));
+            }
+          }
+        }
+      }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  }
+
+  __syncthreads();
+  if (warp == kWarpMma) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------- host side
+
+namespace {
+
+// cuTensorMapEncodeTiled from the driver, found once through the runtime (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      (void)cudaGetLastError();
+  });
+  return fn;
+}
+
+int encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return set_error(FI_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(FI_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FI_OK;
+}
+
+}  // namespace
+
+int64_t mma_smem_bytes() { return (int64_t)kBarOff + kNumBars * 8 + 1024; }
+
+int launch_mma(const MmaArgs& a, cudaStream_t stream) {
+  if (a.k % kMmaKStep != 0 || a.m_pad < 16 || a.m_pad > kMmaMaxM || a.m_pad % 16 != 0)
+    return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA path: k must be a multiple of %d and m <= %d", kMmaKStep,
+                     kMmaMaxM);
+  CUtensorMap tmap_a, tmap_w;
+  // activations: f16 [m_pad, k], box 64 k x m_pad rows, 128-byte swizzle (the MMA's B operand)
+  int rc = encode_2d(&tmap_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.a16, (uint64_t)a.k, (uint64_t)a.m_pad,
+                     (uint64_t)a.k * 2, kMmaKStep, (uint32_t)a.m_pad, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != FI_OK) return rc;
+  // packed codes: u8 [n, k/2], box 32 bytes x 256 rows (rows past n read as zero codes)
+  rc = encode_2d(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, (uint64_t)(a.k / 2), (uint64_t)a.n,
+                 (uint64_t)(a.k / 2), 32, kMmaTileRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc != FI_OK) return rc;
+
+  static int configured[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return set_cuda_error("cudaGetDevice");
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(mma_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)mma_smem_bytes()) != cudaSuccess)
+      return set_cuda_error("cudaFuncSetAttribute(mma smem)");
+    configured[dev] = 1;
+  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+
+  cudaLaunchConfig_t pre = {};
+  pre.gridDim = dim3((unsigned)a.m_pad);
+  pre.blockDim = dim3(256);
+  pre.stream = stream;
+  pre.attrs = attr;
+  pre.numAttrs = 1;
+  if (cudaLaunchKernelEx(&pre, act_to_f16_kernel, a.A, a.m, a.k, a.a16, a.rs) != cudaSuccess)
+    return set_cuda_error("act_to_f16_kernel launch");
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((a.n + kMmaTileRows - 1) / kMmaTileRows));
+  cfg.blockDim = dim3(kMmaThreads);
+  cfg.dynamicSmemBytes = (size_t)mma_smem_bytes();
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, mma_nvfp4_kernel, a, tmap_a, tmap_w) != cudaSuccess)
+    return set_cuda_error("mma_nvfp4_kernel launch");
+  return FI_OK;
+}
+
+}  // namespace fi

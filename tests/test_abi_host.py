@@ -180,3 +180,30 @@ def test_debug_hooks_validate_arguments():
     fi.debug_set(fi.DEBUG_STALL_PRODUCER, 0)
     fi.debug_set(fi.DEBUG_WAIT_TIMEOUT_NS, 1_000_000_000)
     assert fi.library().fi_get_device_error(None) == -1
+
+
+def test_mma_tactic_resolution():
+    t = fi.make_tactic(fi.KIND_MMA, 1, 0, 0)
+    info = fi.resolve_tactic(256, 152064, 5120, t, B200_SMS)
+    assert info["kind"] == fi.KIND_MMA and info["splits"] == 1
+    assert info["grid_x"] == 152064 // 256 and info["threads"] == 14 * 32
+    assert 0 < info["smem_bytes"] <= 227 * 1024
+    # workspace: f16 activations [256, k] then 256 fp32 row scales
+    assert info["workspace_bytes"] == 256 * 5120 * 2 + 256 * 4
+    assert fi.resolve_tactic(33, 100, 64, t, B200_SMS)["workspace_bytes"] == 48 * 64 * 2 + 48 * 4
+    # the default table takes the MMA above m = 32 and the GEMV up to it
+    assert fi.resolve_tactic(33, 4096, 4096, fi.TACTIC_DEFAULT, B200_SMS)["kind"] == fi.KIND_MMA
+    assert fi.resolve_tactic(32, 4096, 4096, fi.TACTIC_DEFAULT, B200_SMS)["kind"] == fi.KIND_GEMV
+    assert t in fi.list_tactics(64, 4096, 4096, B200_SMS)
+
+
+@pytest.mark.parametrize("m,n,k,tactic,status", [
+    (257, 64, 64, fi.make_tactic(1, 1, 0, 0), -2),   # m beyond 256
+    (64, 64, 96, fi.make_tactic(1, 1, 0, 0), -2),    # k not a multiple of 64
+    (64, 64, 64, fi.make_tactic(1, 2, 0, 0), -1),    # no split-K on the MMA path
+    (64, 64, 64, fi.make_tactic(1, 1, 0, 3), -1),    # no variants
+])
+def test_mma_resolve_rejects(m, n, k, tactic, status):
+    with pytest.raises(fi.FiError) as e:
+        fi.resolve_tactic(m, n, k, tactic, B200_SMS)
+    assert e.value.status == status

@@ -1,0 +1,110 @@
+"""GPU tensor-core path (MMA tactics: TMA + tcgen05 + TMEM) against the oracle.
+
+Tolerance for bf16 outputs: |out - ref| <= 1e-2*|ref| + 1e-2*rms(ref row), ref the oracle's
+unrounded fp64 result. Exact cases (small-integer activations, weights with power-of-two
+scales) must match bit for bit; the path must be bitwise deterministic over 10 reruns, and a
+row's bits must not depend on m (an output element depends only on its weight row and its
+activation row).
+"""
+import numpy as np
+import pytest
+import torch
+
+import bf16_activations_nvfp4_b200 as fi
+import oracle
+from bf16_activations_nvfp4_b200 import inputs
+from tests import _gpu
+from tests.test_gpu_mm import _exact_case
+
+pytestmark = pytest.mark.gpu
+
+MMA = fi.make_tactic(fi.KIND_MMA, 1, 0, 0)
+
+
+def _mm(A_bits, dev_w, tactic=MMA):
+    Wq, Ws, g = dev_w
+    out = fi.mm_bf16_fp4(_gpu.dev_bf16(A_bits), Wq, Ws, g, tactic=tactic)
+    torch.cuda.synchronize()
+    return _gpu.host_bits(out)
+
+
+@pytest.mark.parametrize("m,n,k,seed", [(64, 512, 512, 1), (33, 300, 2048, 2), (100, 1000, 1024, 3),
+                                        (256, 768, 4096, 4), (1, 256, 512, 5), (17, 257, 320, 6),
+                                        (128, 4096, 1024, 7), (40, 200, 128, 13)])
+def test_parity_against_oracle(m, n, k, seed):
+    A = inputs.activations(m, k, seed=seed, outliers=True)
+    W, (Wq, Ws, g) = _gpu.weights(n, k, seed)
+    ref = oracle.mm(A, Wq, Ws, g)
+    _gpu.assert_within_tolerance(_mm(A, _gpu.device_weights(n, k, seed)), ref, f"MMA {m}x{n}x{k}")
+
+
+def test_default_table_takes_mma_above_m32():
+    info = fi.resolve_tactic(64, 4096, 14336, fi.TACTIC_DEFAULT)
+    assert info["kind"] == fi.KIND_MMA
+    m, n, k = 64, 1000, 2048
+    A = inputs.activations(m, k, seed=8)
+    W, (Wq, Ws, g) = _gpu.weights(n, k, 8)
+    ref = oracle.mm(A, Wq, Ws, g)
+    _gpu.assert_within_tolerance(_mm(A, _gpu.device_weights(n, k, 8), fi.TACTIC_DEFAULT), ref, "default m=64")
+
+
+@pytest.mark.parametrize("m,n,k", [(40, 300, 512), (256, 512, 1024)])
+def test_integer_exact_bitwise(m, n, k):
+    """Small-integer activations and weights whose block scales and tensor scale are powers of
+    two: every product and partial sum is exact in fp32, so the bf16 output must be the
+    correctly rounded exact result bit for bit (the same case as the GEMV's)."""
+    A, W = _exact_case(m, n, k, seed=m + n)
+    Wq, Ws, g = oracle.pack(W)
+    ref = oracle.mm(A, Wq, Ws, g)
+    assert np.array_equal(ref.astype(np.float32).astype(np.float64), ref)  # exact in fp32
+    want = np.array([[oracle.f32_to_bf16_bits(v) for v in row] for row in ref.astype(np.float32)], np.uint16)
+    got = _mm(A, fi.pack_weights(torch.from_numpy(W).cuda()))
+    assert np.array_equal(got, want)
+
+
+def test_determinism_ten_reruns():
+    m, n, k = 96, 1024, 2048
+    A = inputs.activations(m, k, seed=9, outliers=True)
+    dw = _gpu.device_weights(n, k, 9)
+    base = _mm(A, dw)
+    for _ in range(10):
+        assert np.array_equal(_mm(A, dw), base)
+
+
+def test_rows_do_not_depend_on_m():
+    """Row r of the output has the same bits whether it is computed with m = 33, 64, 128 or
+    256 rows (the MMA's N dimension changes with m)."""
+    n, k = 768, 1024
+    A256 = inputs.activations(256, k, seed=10, outliers=True)
+    dw = _gpu.device_weights(n, k, 10)
+    base = _mm(A256, dw)
+    for m in (1, 16, 33, 64, 128, 200):
+        assert np.array_equal(_mm(A256[:m], dw), base[:m]), m
+
+
+def test_k_not_multiple_of_64_is_refused():
+    m, n, k = 64, 256, 96
+    with pytest.raises(fi.FiError) as e:
+        fi.resolve_tactic(m, n, k, MMA)
+    assert e.value.status == -2
+
+
+def test_stalled_producer_reports_timeout_and_recovers():
+    m, n, k = 64, 512, 1024
+    A = inputs.activations(m, k, seed=12)
+    W, (Wq, Ws, g) = _gpu.weights(n, k, 12)
+    ref = oracle.mm(A, Wq, Ws, g)
+    dw = _gpu.device_weights(n, k, 12)
+    assert fi.get_device_error() == 0
+    fi.debug_set(fi.DEBUG_WAIT_TIMEOUT_NS, 20_000_000)
+    fi.debug_set(fi.DEBUG_STALL_PRODUCER, 1)
+    try:
+        _mm(A, dw)
+        code = fi.get_device_error()
+        assert code != 0, code
+        assert fi.get_device_error() == 0
+    finally:
+        fi.debug_set(fi.DEBUG_STALL_PRODUCER, 0)
+        fi.debug_set(fi.DEBUG_WAIT_TIMEOUT_NS, 1_000_000_000)
+    _gpu.assert_within_tolerance(_mm(A, dw), ref, "after recovery")
+    assert fi.get_device_error() == 0
