@@ -63,14 +63,71 @@ def algorithmic_bytes(m: int, n: int, k: int) -> int:
     return n * k // 2 + n * k // 16 + 2 * m * k + 2 * m * n
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+# lm_head-like GEMM (n=152064, k=5120): m=1 runs the GEMV, m=64 and m=256 the tensor-core path
+LM_HEAD = (152064, 5120)
+LM_HEAD_M = (1, 64, 256)
+
+
 def _peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "source": "measured"}
     except Exception:
-        return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS, "source": "fallback"}
+
+
+def run_lm_head(dev, stream, peaks) -> dict:
+    """The lm_head-like workload at m in LM_HEAD_M, each timed as a CUDA graph of 5 calls (the
+    438 MB of packed weights exceed L2, so every call streams them from HBM). The f16 tensor
+    rate equals the bf16 one, so the tensor fraction is against the measured bf16 peak."""
+    import torch
+
+    import bf16_activations_nvfp4_b200 as fi
+    from bf16_activations_nvfp4_b200 import inputs
+    n, k = LM_HEAD
+    W = torch.from_numpy(inputs.weights(n, k, seed=0, jitter=True)).to(dev)
+    Wq, Ws, g = fi.pack_weights(W)
+    del W
+    ws_bytes = max(fi.workspace_bytes(m, n, k) for m in LM_HEAD_M)
+    ws = torch.empty(max(ws_bytes, 256) // 4 + 64, dtype=torch.float32, device=dev)
+    fi.set_workspace(ws)
+    torch.cuda.synchronize(dev)
+    rows = []
+    for m in LM_HEAD_M:
+        A = torch.from_numpy(inputs.activations(m, k, seed=0).view(np.int16)).view(torch.bfloat16).to(dev)
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        with torch.cuda.stream(stream):
+            fi.mm_bf16_fp4(A, Wq, Ws, g, out=out)
+            torch.cuda.synchronize(dev)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                for _ in range(5):
+                    fi.mm_bf16_fp4(A, Wq, Ws, g, out=out)
+            for _ in range(3):
+                graph.replay()
+            torch.cuda.synchronize(dev)
+            times = []
+            for _ in range(5):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                times.append(e0.elapsed_time(e1) * 1e3 / 5)
+        us = statistics.median(times)
+        info = fi.resolve_tactic(m, n, k)
+        flops, nbytes = 2 * m * n * k, algorithmic_bytes(m, n, k)
+        rows.append({"m": m, "kind": "gemv" if info["kind"] == fi.KIND_GEMV else "mma", "us": round(us, 2),
+                     "tflops": round(flops / us / 1e6, 1), "gbs": round(nbytes / us / 1e3, 1),
+                     "frac_tensor": round(flops / us / 1e6 / peaks["bf16_tflops"], 4),
+                     "frac_hbm": round(nbytes / us / 1e3 / peaks["hbm_gbs"], 4)})
+        del graph, A, out
+    return {"workload": f"lm_head-like GEMM n={n} k={k}, weights N(0,0.02) with per-row U(0.5,2) jitter",
+            "peak_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"] + " bf16 dense (cuBLAS, burst)",
+            "per_m": rows}
 
 
 def _gemv_source_sha() -> str:
@@ -252,6 +309,7 @@ def run_fi(args, rank: int, world: int) -> dict | None:
         default_us = [statistics.median(time_replays(g_, 15)) / nrep for g_, nrep in default_graphs]
     if world > 1:
         dist.barrier()
+    lm_head = run_lm_head(dev, stream, peaks) if world == 1 and not args.no_lm_head else None
 
     # ---- end to end through the public op with host buffers (eager calls)
     e2e_steps = max(5, args.steps // 10)
@@ -340,6 +398,7 @@ def run_fi(args, rank: int, world: int) -> dict | None:
                      "kernel": roof_kernel},
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall1 - wall0, 3),
+        "lm_head": lm_head,
     }
 
 
@@ -477,6 +536,7 @@ def main(argv=None) -> int:
     ap.add_argument("--splits", default=None, help="comma-separated subset of the split menu (0 = device-sized)")
     ap.add_argument("--sweep", action="store_true", help="print per-call µs of every listed tactic and exit")
     ap.add_argument("--m", type=int, default=1, help="activation rows for --sweep")
+    ap.add_argument("--no-lm-head", action="store_true", help="skip the lm_head-like GEMM measurement")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
