@@ -60,18 +60,23 @@ typedef enum {
 /* ------------------------------------------------------------------------- tactics
  * A tactic is a 32-bit code built by FI_TACTIC(kind, splits, ctas_per_sm, variant):
  *   kind         FI_KIND_GEMV (streaming GEMV, 1 <= m <= 32) or FI_KIND_MMA (tcgen05
- *                tensor-core GEMM, 1 <= m <= 256);
+ *                tensor-core GEMM, 1 <= m <= 256, k a multiple of 64, one split);
  *   splits       number of K partitions S (1..4095); 0 = device-sized ("knee") split:
  *                the smallest S that gives the device enough concurrent weight streams
- *                (PR #4038, Description, "What it does": the device-sized GEMV split);
- *   ctas_per_sm  co-resident CTAs per SM used to size the grid (1..15); 0 = automatic
- *                (PR #4038, Description, "What it does": occupancy tactics);
- *   variant      GEMV: weight rows per pipeline stage, computed together by one warp
- *                (1, 2, 4 or 8, at most 16 / m rounded to a power of two; 0 = automatic).
- *                MMA: 0.
+ *                (PR #4038, Description, "What it does": the device-sized GEMV split).
+ *                MMA: 0 or 1;
+ *   ctas_per_sm  CTAs per SM the grid is sized for (PR #4038, Description, "What it
+ *                does": occupancy tactics); 0 = automatic. GEMV stream pipeline: 1 = one
+ *                16-warp CTA per SM, 2 = two 8-warp CTAs per SM; ring pipeline: 1..15.
+ *                MMA: 0 or 1;
+ *   variant      GEMV: low nibble = weight rows computed together by one warp (stream
+ *                pipeline 1, 2 or 4; ring pipeline 1, 2, 4 or 8, at most 16 / m rounded to a
+ *                power of two; 0 = automatic); high nibble = pipeline (0 = automatic =
+ *                1 = per-warp asynchronous copies, 2 = producer-warp ring). MMA: 0.
  * Only `kind` and the resolved S change the arithmetic: two tactics with the same kind
- * and S give bitwise identical outputs, and for a fixed tactic every output row is
- * bitwise independent of m. FI_TACTIC_DEFAULT (-1) selects from the built-in per-shape
+ * and S give bitwise identical outputs (whatever their pipeline, rows or CTAs), and for a
+ * fixed tactic every output row is bitwise independent of m. GEMV and MMA results differ
+ * in their last bits, both within the accuracy of fp32 accumulation. FI_TACTIC_DEFAULT (-1) selects from the built-in per-shape
  * table (PR #4038, Description, "What it does": the untuned m=1 route to the GEMV); the
  * table's choice of kind and S depends on m, so the default is batch-invariant only
  * within the m range of one table entry.
@@ -97,7 +102,7 @@ typedef struct {
   int32_t grid_y;      /* CTAs along k (= splits) */
   int32_t threads;     /* threads per CTA */
   int32_t smem_bytes;  /* dynamic shared memory per CTA */
-  int64_t workspace_bytes; /* fp32 partials needed (0 when S == 1) */
+  int64_t workspace_bytes; /* scratch: GEMV fp32 partials (0 if S == 1), MMA f16 A */
 } fi_tactic_info;
 
 /* ------------------------------------------------------------------ entry points */
@@ -130,10 +135,11 @@ FI_API int fi_nvfp4_pack_weights(const float* W, int64_t n, int64_t k, uint8_t* 
  *   out     device bf16 bits [m, n], 2-byte aligned; must not overlap the inputs.
  *   tactic  FI_TACTIC_DEFAULT or an FI_TACTIC(...) code (see above).
  * Preconditions: m >= 0, n >= 0, k >= 0, k % 32 == 0; m <= 32 for GEMV tactics and
- * m <= 256 for MMA tactics (FI_ERR_UNSUPPORTED_SHAPE otherwise). m == 0 or n == 0 is a
- * no-op; k == 0 writes zeros.
- * Split-K workspace: when the resolved S > 1 the call needs fi_mm_workspace_bytes()
- * bytes of device memory for fp32 partials. It uses the buffer registered with
+ * m <= 256 with k % 64 == 0 for MMA tactics (FI_ERR_UNSUPPORTED_SHAPE otherwise). m == 0
+ * or n == 0 is a no-op; k == 0 writes zeros.
+ * Workspace: a GEMV call with S > 1 needs fi_mm_workspace_bytes() bytes of device memory
+ * for fp32 partials; an MMA call needs them for its f16 copy of A (each row times a power
+ * of two) and the per-row scales. It uses the buffer registered with
  * fi_set_workspace() for the current device (FI_ERR_WORKSPACE if that is too small); if
  * none is registered, the library allocates one with cudaMalloc (growing it when needed)
  * and keeps it until process exit, except while `stream` is capturing a CUDA graph,
@@ -160,20 +166,22 @@ FI_API int fi_mm_bf16_fp4_ex(const uint16_t* A, const uint8_t* Wq, const uint8_t
  * as an operator plugin inside a serving engine that has already reserved the device's memory
  * for weights and the KV cache, or a component whose memory plan is fixed at start-up and
  * that owns no buffer it could pass to fi_mm_bf16_fp4_ex. fi_mm_bf16_fp4 would cudaMalloc its
- * split-K workspace on first use; this variant keeps the fp32 partials in a static device
- * array compiled into the library instead: FI_NOALLOC_SCRATCH_BYTES (4 MiB) on every GPU that
- * loads the library, held until the process exits.
+ * workspace on first use; this variant keeps the workspace (the split-K fp32 partials, or
+ * for MMA tactics the f16 copy of the activations) in a static device array compiled into
+ * the library instead: FI_NOALLOC_SCRATCH_BYTES (4 MiB) on every GPU that loads the library,
+ * held until the process exits.
  * Arguments, tactics, preconditions and results are those of fi_mm_bf16_fp4.
- * Limit: the resolved tactic's fi_mm_workspace_bytes() (4 * splits * m * n) must not exceed
- * FI_NOALLOC_SCRATCH_BYTES; a larger call returns FI_ERR_WORKSPACE and launches nothing.
- * Single-split tactics use no scratch.
+ * Limit: the resolved tactic's fi_mm_workspace_bytes() (GEMV: 4 * splits * m * n; MMA: about
+ * 2 * m * k) must not exceed FI_NOALLOC_SCRATCH_BYTES; a larger call returns
+ * FI_ERR_WORKSPACE and launches nothing. Single-split GEMV tactics use no scratch.
  * Set-up: the first call on a device that reaches a launch looks up the array's device
  * address (cudaGetSymbolAddress, with that device current); make that first call before any
  * stream capture begins.
- * Sharing: all calls on a device use the same array, and it keeps the last call's partials.
+ * Sharing: all calls on a device use the same array, and it keeps the last call's contents.
  * Nothing in it needs to start at zero (each split writes all of its partials before the
- * reduce reads them), but calls whose kernels can overlap on the GPU (different streams,
- * parallel graph branches) race on it and must be serialised by the caller.
+ * reduce reads them; the MMA path writes its whole activation copy before reading it), but
+ * calls whose kernels can overlap on the GPU (different streams, parallel graph branches)
+ * race on it and must be serialised by the caller.
  * Never calls cudaMalloc, cudaFree or any other allocating routine.
  */
 #define FI_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
@@ -212,8 +220,8 @@ FI_API int64_t fi_default_tactic(int64_t m, int64_t n, int64_t k, int num_sms);
  * (which may exceed cap), or a negative status. */
 FI_API int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, int cap);
 
-/* Workspace bytes a call with this shape and tactic needs (0 when S == 1), or 0 for an
- * invalid tactic. */
+/* Workspace bytes a call with this shape and tactic needs (GEMV: 0 when S == 1; MMA: the
+ * f16 activations and their row scales), or 0 for an invalid tactic. */
 FI_API size_t fi_mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms);
 
 /* Register a caller-owned split-K workspace for the current device (device pointer,
