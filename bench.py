@@ -358,7 +358,7 @@ def run_fi(args, rank: int, world: int) -> dict | None:
     keys = [key(c["shape"]) for c in on]
     if NCU_TRAFFIC["source_sha256"] == _gemv_source_sha() and all(k_ in NCU_TRAFFIC["bytes"] for k_ in keys):
         traffic = round(statistics.fmean(NCU_TRAFFIC["bytes"][k_] for k_ in keys))
-    roof_kernel = "gemv_nvfp4_kernel, split 1, one launch per call, on " + ", ".join(sorted(set(keys)))
+    roof_kernel = "gemv_stream_kernel, split 1, one launch per call, on " + ", ".join(sorted(set(keys)))
     def_bytes = sum(shapes[d["shape"]]["bytes"] for d in defaults)
     return {
         "metric": METRIC,
