@@ -151,7 +151,7 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
   const int64_t nch = (C + S - 1) / S;  // chunks of the largest split
   const int ctas = ctas_per_sm > 0 ? ctas_per_sm : (stream_wide(n, sms) ? 2 : 1);
   if (ctas > 2) return set_error(FI_ERR_INVALID_ARG, "GEMV stream pipeline: at most 2 CTAs per SM");
-  const int nw = ctas == 1 ? 16 : 8;
+  int nw = ctas == 1 ? 16 : 8;
   const int64_t budget = ctas == 1 ? kSmemBudget : kStreamHalfBudget;
   const int64_t a_bytes = round_up(m * ((nch + 31) / 32) * 2048, 128);
   const int64_t as_bytes = round_up(m * nch * 8, 128);
@@ -163,6 +163,13 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
                      (long long)m);
   const int64_t slot = (int64_t)kStreamIters * r * kStreamCellBytes;
   const int64_t fixed = a_bytes + as_bytes;
+  // Rows go to warps in whole groups of r. When the groups of a split would fill fewer than
+  // its share of CTA slots, the CTAs get fewer warps (at least 4) so that the work spreads over
+  // every SM (4096 x 14336 at m = 1: 2048 groups of 2 rows on 147 CTAs of 14 warps instead of
+  // 128 CTAs of 16).
+  const int64_t groups = (n + r - 1) / r;
+  const int64_t gx_cap = std::max<int64_t>(1, (int64_t)sms * ctas / S);
+  if ((groups + nw - 1) / nw < gx_cap) nw = (int)std::max<int64_t>(4, (groups + gx_cap - 1) / gx_cap);
   int ns = 4;
   if (fixed + (int64_t)nw * ns * slot > budget) ns = 2;
   if (fixed + (int64_t)nw * ns * slot > budget)
@@ -170,9 +177,7 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
                      "GEMV: m=%lld over %lld k per split leaves no room for the weight slots in shared memory; "
                      "use more splits",
                      (long long)m, (long long)(nch * kChunkK));
-  const int64_t groups = (n + r - 1) / r;
-  int64_t gx = std::max<int64_t>(1, (int64_t)sms * ctas / S);
-  gx = std::max<int64_t>(1, std::min<int64_t>(gx, (groups + nw - 1) / nw));
+  const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(gx_cap, (groups + nw - 1) / nw));
   g->pipeline = kPipeStream;
   g->threads = nw * 32;
   g->S = S;
@@ -202,10 +207,13 @@ static int gemv_knee(int pipe, int64_t n, int64_t k, int sms, int64_t m_fit, int
   for (int64_t S = 1; S <= maxS; ++S) {
     GemvGeometry g;
     if (geometry_for(pipe, m_fit, n, k, (int)S, rs, ctas, sms, &g) != FI_OK) continue;
-    // enough: the split's CTAs cover at least 40% of the SMs' CTA slots. Measured on B200:
-    // idle SMs cost less than a second kernel and the partials' traffic until well below that
-    // (2048 x 7168 at m = 1 runs faster on 64 CTAs than split in two).
-    const bool enough = (int64_t)g.grid_x * S * 5 >= (int64_t)sms * g.ctas_per_sm * 2;
+    // enough: the splits' warps cover at least 40% of the SMs' warp slots (16 per SM; the ring
+    // pipeline's CTAs always have 16 consumer warps). Measured on B200: idle warp slots cost
+    // less than a second kernel and the partials' traffic until well below that (2048 x 7168
+    // at m = 1 ran faster on 64 CTAs of 16 warps than split in two).
+    const int64_t warps = (int64_t)g.grid_x * (pipe == kPipeRing ? 16 : g.threads / 32);
+    const int64_t slots = pipe == kPipeRing ? (int64_t)sms * g.ctas_per_sm * 16 : (int64_t)sms * 16;
+    const bool enough = warps * S * 5 >= slots * 2;
     const bool last = S == maxS || (C / (S + 1)) < 32;  // a split keeps at least one warp step
     if (enough || last) {
       *S_out = (int)S;
@@ -454,6 +462,9 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.grid_x = g.grid_x;
     a.threads = g.threads;
     a.pdl = 1;
+    // whole aligned 16-byte scale pieces per row and iteration: k % 256 == 0 and every split
+    // boundary on a multiple of 8 chunks
+    a.scale16 = k % 256 == 0 && (k / kChunkK) % (8 * (int64_t)g.S) == 0 ? 1 : 0;
     a.debug_stall = g_debug_stall_launches > 0 ? 1 : 0;
     if (g_debug_stall_launches > 0) --g_debug_stall_launches;
     a.stage_bytes = g.stage_bytes;

@@ -106,28 +106,6 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
   return r;
 }
 
-// ------------------------------------------------------------ mixed-precision FMA
-
-// acc + a.lo * b.lo and acc + a.hi * b.hi with f16 multiplicands and an fp32 addend/result
-// (sm_100 mixed-precision fma: the f16 product is exact in fp32, one rounding per step).
-__device__ __forceinline__ float fma_lo_f16(uint32_t a2, uint32_t b2, float acc) {
-  float d;
-  asm("{\n .reg .b16 al, ah, bl, bh;\n mov.b32 {al, ah}, %1;\n mov.b32 {bl, bh}, %2;\n"
-      " fma.rn.f32.f16 %0, al, bl, %3;\n}"
-      : "=f"(d)
-      : "r"(a2), "r"(b2), "f"(acc));
-  return d;
-}
-
-__device__ __forceinline__ float fma_hi_f16(uint32_t a2, uint32_t b2, float acc) {
-  float d;
-  asm("{\n .reg .b16 al, ah, bl, bh;\n mov.b32 {al, ah}, %1;\n mov.b32 {bl, bh}, %2;\n"
-      " fma.rn.f32.f16 %0, ah, bh, %3;\n}"
-      : "=f"(d)
-      : "r"(a2), "r"(b2), "f"(acc));
-  return d;
-}
-
 // ------------------------------------------------------------------- bf16 output
 
 __device__ __forceinline__ uint16_t f32_to_bf16_rn(float x) {

@@ -26,13 +26,18 @@
 //    tensor the producer copies the scales with plain loads). With S > 1 each row's slice is
 //    copied on its own.
 //  * Arithmetic (fixed by k and S alone, hence bitwise identical for every m, RS, NST, G and
-//    CTAs per SM): A is staged as f16 with one power-of-two scale per 16-block (exact for
-//    every element within 2^28 of its block maximum); codes are decoded by
-//    cvt.rn.f16x2.e2m1x2 (exact) and multiplied by the mixed-precision fma.rn.f32.f16 (exact
-//    product, fp32 accumulate). Lane L takes chunks L, L+32, L+64, ... of the split: per
-//    16-block p = sum_i a_i * e2m1_i in element order, then acc = fma(p, sf_w * sf_a, acc);
-//    the lanes combine through a fixed xor butterfly (all lanes end with the same bits).
-//    S == 1 writes bf16_rn(acc * gscale); S > 1 writes fp32 partials for the reduce kernel.
+//    CTAs per SM): A is staged as f16 with one power-of-two scale sf_a per 16-block that puts
+//    the block maximum in [2^9, 2^10) (exact for every element within 2^26 of its block
+//    maximum); codes are decoded by cvt.rn.f16x2.e2m1x2 (exact). Per 16-block, packed f16
+//    fused multiply-adds sum the even and the odd elements' products in element order (8
+//    steps each, partial sums below 2^16); the two half sums times the block's E4M3 scale go
+//    to fp32 through the mixed-precision fma.rn.f32.f16, and acc = fma(t, sf_a, acc). Lane L
+//    takes chunks L, L+32, L+64, ... of the split; the lanes combine through a fixed xor
+//    butterfly (all lanes end with the same bits). S == 1 writes bf16_rn(acc * gscale); S > 1
+//    writes fp32 partials for the reduce kernel. The f16 half sums are what make the inner loop
+//    cheap on sm_100: the packed f16 FMA issues to the other FMA port than the e2m1 conversion,
+//    so decode and products run side by side; their rounding (one f16 rounding per step on
+//    magnitudes below 2^16) stays far below the bf16 output's own.
 //  * Bounded waits. Every mbarrier wait gives up after a time limit (%globaltimer): it sets a
 //    device error flag and a CTA-wide abort flag, the CTA finishes its control flow without
 //    computing, and the producer waits (bounded) for the copies it issued before exiting.
@@ -95,7 +100,7 @@ __device__ __forceinline__ void stage_block(const uint4 v0, const uint4 v1, int 
     e = max(e, (w[i] >> 7) & 0xFFu);
     e = max(e, (w[i] >> 23) & 0xFFu);
   }
-  int sh = 141 - (int)e;  // biased exponent E -> block maximum in [2^14, 2^15)
+  int sh = 136 - (int)e;  // biased exponent E -> block maximum in [2^9, 2^10)
   sh = sh < -126 ? -126 : (sh > 126 ? 126 : sh);
   const float up = __uint_as_float((uint32_t)(sh + 127) << 23);
   const float down = __uint_as_float((uint32_t)(127 - sh) << 23);
@@ -117,7 +122,7 @@ __device__ __forceinline__ void stage_block(const uint4 v0, const uint4 v1, int 
 // chunk c (32 k) of row r is 4 16-byte quads at uint4 index ((r * GA + c / 32) * 4 + q) * 32 +
 // c % 32 (GA = ceil(nch / 32)), so a warp reading 32 consecutive chunks touches 512
 // contiguous bytes per quad. Values are f16 scaled by a power of two per 16-block that puts
-// the block maximum in [2^14, 2^15); As[r][b] holds the inverse scale. A thread loads up to four
+// the block maximum in [2^9, 2^10); As[r][b] holds the inverse scale. A thread loads up to four
 // of its blocks before converting any, so their global-memory latencies overlap.
 __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A, int64_t k, int m,
                                                   int64_t kbase, int nch, uint4* Ah4, float* As, int tid,
@@ -148,14 +153,48 @@ __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A
   }
 }
 
-// p += a_i * w_i for the 8 f16 pairs of one 16-block, in element order.
-__device__ __forceinline__ float dot16(const uint32_t* a, const uint32_t* w, float p) {
+// The 8 f16 pairs of one 16-block multiplied lane-wise and summed in element order in packed
+// f16: the low half sums the block's even elements, the high half its odd ones, one fused
+// multiply-add (one rounding) per step. The activations are staged below 2^10 and |e2m1| <= 6,
+// so every partial sum stays below 8 * 6 * 2^10 < 2^16: no overflow.
+__device__ __forceinline__ uint32_t hdot8(const uint32_t* a, const uint32_t* w) {
+  uint32_t h;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h) : "r"(a[0]), "r"(w[0]));
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    p = fma_lo_f16(a[i], w[i], p);
-    p = fma_hi_f16(a[i], w[i], p);
+  for (int i = 1; i < 8; ++i) asm("fma.rn.f16x2 %0, %1, %2, %0;" : "+r"(h) : "r"(a[i]), "r"(w[i]));
+  return h;
+}
+
+// acc + (h.lo * sw + h.hi * sw) * sa for one 16-block: its two f16 half sums times the block's
+// E4M3 weight scale sw (an f16: the low half of sh for HALF 0, the high half for HALF 1) in
+// fp32 (the first product exact, the second added with one rounding), then times the
+// activation block's power-of-two scale sa and added to acc (one rounding).
+template <int HALF>
+__device__ __forceinline__ float block_acc(uint32_t h, uint32_t sh, float sa, float acc) {
+  float t;
+  if constexpr (HALF == 0) {
+    asm("{\n .reg .b16 hl, hh, sl, su;\n mov.b32 {hl, hh}, %1;\n mov.b32 {sl, su}, %2;\n"
+        " fma.rn.f32.f16 %0, hl, sl, 0f00000000;\n fma.rn.f32.f16 %0, hh, sl, %0;\n}"
+        : "=f"(t)
+        : "r"(h), "r"(sh));
+  } else {
+    asm("{\n .reg .b16 hl, hh, sl, su;\n mov.b32 {hl, hh}, %1;\n mov.b32 {sl, su}, %2;\n"
+        " fma.rn.f32.f16 %0, hl, su, 0f00000000;\n fma.rn.f32.f16 %0, hh, su, %0;\n}"
+        : "=f"(t)
+        : "r"(h), "r"(sh));
   }
-  return p;
+  return fmaf(t, sa, acc);
+}
+
+// One 32-k chunk of one weight row against one activation row: av the chunk's 16 staged f16
+// pairs, sa its two block scales, wf the decoded codes, sh the two E4M3 block scales as f16x2.
+// Both pipelines call this, so their bits agree.
+__device__ __forceinline__ float chunk_acc(const uint32_t (&av)[16], float2 sa, const uint32_t (&wf)[16], uint32_t sh,
+                                           float acc) {
+  const uint32_t h0 = hdot8(av, wf);
+  const uint32_t h1 = hdot8(av + 8, wf + 8);
+  acc = block_acc<0>(h0, sh, sa.x, acc);
+  return block_acc<1>(h1, sh, sa.y, acc);
 }
 
 // Decode one 16-byte code quad (32 E2M1 codes) into 16 f16x2 words.
@@ -199,11 +238,7 @@ __device__ __forceinline__ void stage_rows(uint32_t code0, int cstride, uint32_t
         const uint32_t sc = lds_u16(scale0[i] + (uint32_t)(c * 2));
         uint32_t wf[16];
         decode32(cq, wf);
-        const float p0 = dot16(av, wf, 0.0f);
-        const float p1 = dot16(av + 8, wf + 8, 0.0f);
-        const uint32_t sh = e4m3x2_to_f16x2(sc);
-        acc[i][0] = fmaf(p0, f16_lo_to_f32(sh) * sa.x, acc[i][0]);
-        acc[i][0] = fmaf(p1, f16_hi_to_f32(sh) * sa.y, acc[i][0]);
+        acc[i][0] = chunk_acc(av, sa, wf, e4m3x2_to_f16x2(sc), acc[i][0]);
       }
     } else {
 #pragma unroll
@@ -213,7 +248,6 @@ __device__ __forceinline__ void stage_rows(uint32_t code0, int cstride, uint32_t
         uint32_t wf[16];
         decode32(cq, wf);
         const uint32_t sh = e4m3x2_to_f16x2(sc);
-        const float sw0 = f16_lo_to_f32(sh), sw1 = f16_hi_to_f32(sh);
 #pragma unroll
         for (int r = 0; r < MT; ++r) {
           if (r < m) {
@@ -221,11 +255,7 @@ __device__ __forceinline__ void stage_rows(uint32_t code0, int cstride, uint32_t
             const uint4 a0 = lds_v4(apr), a1 = lds_v4(apr + 512), a2 = lds_v4(apr + 1024), a3 = lds_v4(apr + 1536);
             const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
                                      a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-            const float2 sa = lds_f2(sp + (uint32_t)r * as_row);
-            const float p0 = dot16(av, wf, 0.0f);
-            const float p1 = dot16(av + 8, wf + 8, 0.0f);
-            acc[i][r] = fmaf(p0, sw0 * sa.x, acc[i][r]);
-            acc[i][r] = fmaf(p1, sw1 * sa.y, acc[i][r]);
+            acc[i][r] = chunk_acc(av, lds_f2(sp + (uint32_t)r * as_row), wf, sh, acc[i][r]);
           }
         }
       }
@@ -470,19 +500,16 @@ __device__ __forceinline__ void sts_u16(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"((unsigned short)v) : "memory");
 }
 
-// One chunk c of the split for R weight rows against MT activation rows. code_s is the lane's
-// cell of row 0 in the slot, scale_s the lane's scale word of row 0; soff[i] is the offset (0
-// or 2) of the lane's two scale bytes within row i's word. Every weight row is computed
-// without a branch, so the compiler can interleave the rows' independent FMA chains; rows of a
-// partial group compute on stale cells and are never written. Same arithmetic per chunk as
-// stage_rows.
+// One chunk of the split for R weight rows against MT activation rows. code_s is the lane's
+// cell of row 0 in the slot, scale_s + soff[i] the address of the lane's two scale bytes of row
+// i (rows 128 bytes apart); ap / sp are the lane's staged activations of the chunk (4 quads 512
+// bytes apart) and their two block scales, for activation row 0 (rows a_row / as_row apart).
+// Every weight row is computed without a branch, so the compiler can interleave the rows'
+// independent chains; rows of a partial group compute on stale cells and are never written.
 template <int MT, int R>
-__device__ __forceinline__ void item_rows(uint32_t code_s, uint32_t scale_s, const uint32_t (&soff)[R], uint32_t a_s,
-                                          uint32_t as_s, int m, int nch, int GA, int c, float (&acc)[R][MT]) {
-  const uint32_t a_row = (uint32_t)GA * 4 * 32 * 16;
-  const uint32_t as_row = (uint32_t)nch * 8;
-  const uint32_t ap = a_s + (uint32_t)(((c >> 5) * 4 * 32 + (c & 31)) * 16);
-  const uint32_t sp = as_s + (uint32_t)c * 8;
+__device__ __forceinline__ void item_rows(uint32_t code_s, uint32_t scale_s, const uint32_t (&soff)[R], uint32_t ap,
+                                          uint32_t sp, uint32_t a_row, uint32_t as_row, int m,
+                                          float (&acc)[R][MT]) {
   if (MT == 1) {
     const uint4 a0 = lds_v4(ap), a1 = lds_v4(ap + 512), a2 = lds_v4(ap + 1024), a3 = lds_v4(ap + 1536);
     const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
@@ -494,11 +521,7 @@ __device__ __forceinline__ void item_rows(uint32_t code_s, uint32_t scale_s, con
       const uint32_t sc = lds_u16(scale_s + (uint32_t)(i * 128) + soff[i]);
       uint32_t wf[16];
       decode32(cq, wf);
-      const float p0 = dot16(av, wf, 0.0f);
-      const float p1 = dot16(av + 8, wf + 8, 0.0f);
-      const uint32_t sh = e4m3x2_to_f16x2(sc);
-      acc[i][0] = fmaf(p0, f16_lo_to_f32(sh) * sa.x, acc[i][0]);
-      acc[i][0] = fmaf(p1, f16_hi_to_f32(sh) * sa.y, acc[i][0]);
+      acc[i][0] = chunk_acc(av, sa, wf, e4m3x2_to_f16x2(sc), acc[i][0]);
     }
   } else {
 #pragma unroll
@@ -508,7 +531,6 @@ __device__ __forceinline__ void item_rows(uint32_t code_s, uint32_t scale_s, con
       uint32_t wf[16];
       decode32(cq, wf);
       const uint32_t sh = e4m3x2_to_f16x2(sc);
-      const float sw0 = f16_lo_to_f32(sh), sw1 = f16_hi_to_f32(sh);
 #pragma unroll
       for (int r = 0; r < MT; ++r) {
         if (r < m) {
@@ -516,11 +538,7 @@ __device__ __forceinline__ void item_rows(uint32_t code_s, uint32_t scale_s, con
           const uint4 a0 = lds_v4(apr), a1 = lds_v4(apr + 512), a2 = lds_v4(apr + 1024), a3 = lds_v4(apr + 1536);
           const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
                                    a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
-          const float2 sa = lds_f2(sp + (uint32_t)r * as_row);
-          const float p0 = dot16(av, wf, 0.0f);
-          const float p1 = dot16(av + 8, wf + 8, 0.0f);
-          acc[i][r] = fmaf(p0, sw0 * sa.x, acc[i][r]);
-          acc[i][r] = fmaf(p1, sw1 * sa.y, acc[i][r]);
+          acc[i][r] = chunk_acc(av, lds_f2(sp + (uint32_t)r * as_row), wf, sh, acc[i][r]);
         }
       }
     }
@@ -561,21 +579,30 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_stream_kernel(GemvA
   const uint8_t* const ws_end = p.Ws + n * rs_s;
   const uint32_t a_s = smem_addr(smem), as_s = smem_addr(smem + p.off_as);
   // this warp's ring: NS slots; in a slot, the cell of (iteration ti, row i) for lane L at
-  // (ti*R + i)*512 + L*16, and its scale word at TI*R*512 + (ti*R + i)*128 + L*4
+  // (ti*R + i)*512 + L*16, and the scale cell of (ti, i) at TI*R*512 + (ti*R + i)*128
   const uint32_t ring = smem_addr(smem + p.off_ring) + (uint32_t)warp * NS * kSlot;
   const uint32_t my_code = ring + (uint32_t)lane * 16;
-  const uint32_t my_scale = ring + (uint32_t)(TI * R) * 512 + (uint32_t)lane * 4;
+  const uint32_t scale_area = ring + (uint32_t)(TI * R) * 512;
   const int64_t lane_k = (c0 + lane) * 2;  // the lane's first scale byte within a row's split
+  // Scale copies. s16 (k % 256 == 0 and every split starts and ends on 8 chunks, so a row's
+  // scales of one iteration are four aligned 16-byte pieces): lane L < 4*TI*R copies piece pc
+  // of (iteration ti_L, row i_L) of every item into the first 64 bytes of that cell, and lane
+  // L's two bytes of a cell sit at 2L. Otherwise every lane copies the 4-byte aligned word
+  // holding its two bytes to cell + 4L.
+  const bool s16 = p.scale16 != 0;
+  const int pc = lane & 3, i_l = (lane >> 2) % R, ti_l = lane / (4 * R);
+  const bool s_lane = lane < 4 * TI * R;
+  const uint32_t my_scale = scale_area + (s16 ? 0u : (uint32_t)lane * 4);
+  const uint32_t my_s16 = scale_area + (uint32_t)((ti_l * R + i_l) * 128 + pc * 16);
 
   pdl_launch_dependents();
 
-  // ---- issue cursor: item iq = (group ig, item itt of the row group). One code pointer and
-  // one scale pointer (row j0 of the group, this lane's cell at the item's first iteration)
-  // advance by TI*512 and TI*64 bytes per item; row i adds i * k/2 to the code pointer and a
-  // per-group offset to the scale pointer (the 4-byte aligned word with the lane's two bytes).
-  const uint32_t rsq = (uint32_t)rs_q;
+  // ---- issue cursor: item iq = (group ig, item itt of the row group). Row i's code pointer
+  // q[i] (this lane's cell at the item's first iteration) advances by TI*512 bytes per item;
+  // the scale pointer sp (s16: this lane's piece; else the 4-byte word of row 0, row i at
+  // sdel[i] beyond it) by TI*64.
   int ig = 0, itt = 0, iq = 0;
-  const uint8_t* qp = nullptr;
+  const uint8_t* q[R];
   const uint8_t* sp = nullptr;
   uint32_t sdel[R];
   int irows = 0;
@@ -583,36 +610,49 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_stream_kernel(GemvA
   auto issue_group = [&]() {
     const int64_t j0 = r_lo + (int64_t)ig * R;
     irows = (int)max((int64_t)0, min((int64_t)R, r_hi - j0));
-    const int64_t x0 = j0 * rs_s + lane_k;
-    qp = p.Wq + j0 * rs_q + (c0 + lane) * 16;
-    sp = p.Ws + (x0 & ~(int64_t)3);
 #pragma unroll
-    for (int i = 0; i < R; ++i) sdel[i] = (uint32_t)(((x0 + i * rs_s) & ~(int64_t)3) - (x0 & ~(int64_t)3));
-    iedge = (n * rs_s) % 4 != 0 && j0 + irows >= n;
+    for (int i = 0; i < R; ++i) q[i] = p.Wq + (j0 + (i < irows ? i : 0)) * rs_q + (c0 + lane) * 16;
+    if (s16) {
+      sp = p.Ws + (j0 + (i_l < irows ? i_l : 0)) * rs_s + c0 * 2 + ti_l * 64 + pc * 16;
+    } else {
+      const int64_t x0 = j0 * rs_s + lane_k;
+      sp = p.Ws + (x0 & ~(int64_t)3);
+#pragma unroll
+      for (int i = 0; i < R; ++i) sdel[i] = (uint32_t)(((x0 + i * rs_s) & ~(int64_t)3) - (x0 & ~(int64_t)3));
+      iedge = (n * rs_s) % 4 != 0 && j0 + irows >= n;
+    }
   };
   // copy item iq into the slot at byte offset uo; always commits one group (empty past the
   // warp's last item) so that wait_group counts stay uniform
   auto issue = [&](uint32_t uo) {
     if (iq < Q) {
       const int t0 = itt * TI;
+      if (irows == R && (t0 + TI) * 32 <= nch) {  // warp-uniform: no row or lane is cut
 #pragma unroll
-      for (int ti = 0; ti < TI; ++ti) {
-        if ((t0 + ti) * 32 + lane < nch) {
-          const uint32_t cdst = my_code + uo + (uint32_t)(ti * R * 512);
-          const uint32_t sdst = my_scale + uo + (uint32_t)(ti * R * 128);
-          if (irows == R && !iedge) {
+        for (int ti = 0; ti < TI; ++ti)
 #pragma unroll
-            for (int i = 0; i < R; ++i) {
-              cp_async_16(cdst + (uint32_t)(i * 512), qp + i * rsq + ti * 512);
-              cp_async_4(sdst + (uint32_t)(i * 128), sp + sdel[i] + ti * 64);
-            }
-          } else {
+          for (int i = 0; i < R; ++i) cp_async_16(my_code + uo + (uint32_t)((ti * R + i) * 512), q[i] + ti * 512);
+        if (s16 && s_lane) cp_async_16(my_s16 + uo, sp);
+      } else {
+#pragma unroll
+        for (int ti = 0; ti < TI; ++ti)
+          if ((t0 + ti) * 32 + lane < nch) {
+#pragma unroll
+            for (int i = 0; i < R; ++i)
+              if (i < irows) cp_async_16(my_code + uo + (uint32_t)((ti * R + i) * 512), q[i] + ti * 512);
+          }
+        if (s16 && s_lane && i_l < irows && (t0 + ti_l) * 32 + pc * 8 < nch) cp_async_16(my_s16 + uo, sp);
+      }
+      if (!s16) {
+#pragma unroll
+        for (int ti = 0; ti < TI; ++ti) {
+          if ((t0 + ti) * 32 + lane < nch) {
+            const uint32_t sdst = my_scale + uo + (uint32_t)(ti * R * 128);
 #pragma unroll
             for (int i = 0; i < R; ++i) {
               if (i < irows) {
-                cp_async_16(cdst + (uint32_t)(i * 512), qp + i * rsq + ti * 512);
                 const uint8_t* w = sp + sdel[i] + ti * 64;
-                if (w + 4 <= ws_end) {
+                if (!iedge || w + 4 <= ws_end) {
                   cp_async_4(sdst + (uint32_t)(i * 128), w);
                 } else {  // the tensor's last scale pair when its size is 2 mod 4: plain load
                   const uint32_t off = (uint32_t)(((r_lo + (int64_t)ig * R + i) * rs_s + lane_k) & 2);
@@ -623,7 +663,8 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_stream_kernel(GemvA
           }
         }
       }
-      qp += TI * 512;
+#pragma unroll
+      for (int i = 0; i < R; ++i) q[i] += TI * 512;
       sp += TI * 64;
       ++iq;
       if (++itt == TT) {
@@ -647,7 +688,10 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_stream_kernel(GemvA
   __syncthreads();
   const float g = (S == 1) ? *p.gscale : 1.0f;
 
-  // ---- compute cursor
+  // ---- compute cursor: the lane's staged activations of chunk 32 t + L sit at a_s + t*2048 +
+  // L*16 and their block scales at as_s + t*256 + L*8
+  const uint32_t a_row = (uint32_t)GA * 2048, as_row = (uint32_t)nch * 8;
+  const uint32_t a_lane = a_s + (uint32_t)lane * 16, as_lane = as_s + (uint32_t)lane * 8;
   float acc[R][MT];
 #pragma unroll
   for (int i = 0; i < R; ++i)
@@ -656,22 +700,32 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_stream_kernel(GemvA
   int64_t j0 = r_lo;
   int ctt = 0;
   uint32_t uo = 0;  // byte offset of the slot being computed
-  uint32_t soff[R];  // 0 or 2: the lane's scale bytes within its word (the same for every chunk of a row)
+  uint32_t ac = a_lane, asc = as_lane;  // the item's first iteration
+  // the lane's scale bytes within a cell, beyond my_scale (the same for every chunk of a row):
+  // 2L with 16-byte scale copies, else 0 or 2 within the lane's word
+  uint32_t soff[R];
 #pragma unroll
-  for (int i = 0; i < R; ++i) soff[i] = (uint32_t)(((j0 + i) * rs_s + lane_k) & 2);
-  for (int q = 0; q < Q; ++q) {
-    cp_async_wait<NS - 1>();  // this lane's copies of item q have landed
+  for (int i = 0; i < R; ++i) soff[i] = s16 ? (uint32_t)lane * 2 : (uint32_t)(((j0 + i) * rs_s + lane_k) & 2);
+  for (int q_ = 0; q_ < Q; ++q_) {
+    cp_async_wait<NS - 1>();  // this lane's copies of item q_ have landed
     const int t0 = ctt * TI;
+    if ((t0 + TI) * 32 <= nch) {  // warp-uniform: every lane has every chunk of the item
 #pragma unroll
-    for (int ti = 0; ti < TI; ++ti) {
-      const int c = (t0 + ti) * 32 + lane;
-      if (c < nch)
+      for (int ti = 0; ti < TI; ++ti)
         item_rows<MT, R>(my_code + uo + (uint32_t)(ti * R * 512), my_scale + uo + (uint32_t)(ti * R * 128), soff,
-                         a_s, as_s, m, nch, GA, c, acc);
+                         ac + (uint32_t)ti * 2048, asc + (uint32_t)ti * 256, a_row, as_row, m, acc);
+    } else {
+#pragma unroll
+      for (int ti = 0; ti < TI; ++ti)
+        if ((t0 + ti) * 32 + lane < nch)
+          item_rows<MT, R>(my_code + uo + (uint32_t)(ti * R * 512), my_scale + uo + (uint32_t)(ti * R * 128), soff,
+                           ac + (uint32_t)ti * 2048, asc + (uint32_t)ti * 256, a_row, as_row, m, acc);
     }
-    // refill the slot just read with item q + NS (the reads above are complete: their
+    // refill the slot just read with item q_ + NS (the reads above are complete: their
     // results have been consumed)
     issue(uo);
+    ac += TI * 2048;
+    asc += TI * 256;
     if (++ctt == TT) {
       finish_rows<MT, R>(acc, p, j0, (int)min((int64_t)R, r_hi - j0), m, S, s, g, lane, true);
 #pragma unroll
@@ -679,9 +733,11 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_stream_kernel(GemvA
 #pragma unroll
         for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
       ctt = 0;
+      ac = a_lane;
+      asc = as_lane;
       j0 += R;
 #pragma unroll
-      for (int i = 0; i < R; ++i) soff[i] = (uint32_t)(((j0 + i) * rs_s + lane_k) & 2);
+      for (int i = 0; i < R; ++i) soff[i] = s16 ? (uint32_t)lane * 2 : (uint32_t)(((j0 + i) * rs_s + lane_k) & 2);
     }
     uo = (uo == (uint32_t)(NS - 1) * kSlot) ? 0u : uo + kSlot;
   }

@@ -85,6 +85,7 @@ struct GemvArgs {
   int grid_x;          // CTAs per split
   int threads;         // threads per CTA
   int pdl;             // launch with programmatic stream serialization
+  int scale16;         // stream pipeline: copy the E4M3 scales in aligned 16-byte pieces (k % 256 == 0, splits on 8 chunks)
   int debug_stall;     // test hook: the producer issues nothing (consumer waits time out)
   int64_t stage_bytes, off_as, off_bar, off_ring, smem_bytes;
   uint64_t timeout_ns; // limit of every mbarrier wait
