@@ -145,11 +145,13 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_p
 // SM with four rows per item; below that, one 16-warp CTA per SM with two rows per item.
 static bool stream_wide(int64_t n, int sms) { return n >= (int64_t)sms * 64; }
 
+// overlap: CTAs sized for half an SM, but only one per SM, so that the next call's CTAs (launched
+// early by programmatic dependent launch) are resident beside them and prefetch their weights.
 int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int ctas_per_sm, int sms,
-                         GemvGeometry* g) {
+                         GemvGeometry* g, bool overlap) {
   const int64_t C = k / kChunkK;
   const int64_t nch = (C + S - 1) / S;  // chunks of the largest split
-  const int ctas = ctas_per_sm > 0 ? ctas_per_sm : (stream_wide(n, sms) ? 2 : 1);
+  const int ctas = overlap ? 2 : (ctas_per_sm > 0 ? ctas_per_sm : (stream_wide(n, sms) ? 2 : 1));
   if (ctas > 2) return set_error(FI_ERR_INVALID_ARG, "GEMV stream pipeline: at most 2 CTAs per SM");
   int nw = ctas == 1 ? 16 : 8;
   const int64_t budget = ctas == 1 ? kSmemBudget : kStreamHalfBudget;
@@ -168,7 +170,7 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
   // every SM (4096 x 14336 at m = 1: 2048 groups of 2 rows on 147 CTAs of 14 warps instead of
   // 128 CTAs of 16).
   const int64_t groups = (n + r - 1) / r;
-  const int64_t gx_cap = std::max<int64_t>(1, (int64_t)sms * ctas / S);
+  const int64_t gx_cap = std::max<int64_t>(1, (int64_t)sms * (overlap ? 1 : ctas) / S);
   if ((groups + nw - 1) / nw < gx_cap) nw = (int)std::max<int64_t>(4, (groups + gx_cap - 1) / gx_cap);
   int ns = 4;
   if (fixed + (int64_t)nw * ns * slot > budget) ns = 2;
@@ -178,7 +180,7 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
                      "use more splits",
                      (long long)m, (long long)(nch * kChunkK));
   const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(gx_cap, (groups + nw - 1) / nw));
-  g->pipeline = kPipeStream;
+  g->pipeline = overlap ? kPipeOverlap : kPipeStream;
   g->threads = nw * 32;
   g->S = S;
   g->RS = (int)r;
@@ -187,15 +189,15 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
   g->grid_x = (int)gx;
   g->stage_bytes = slot;
   g->off_as = a_bytes;
-  g->off_bar = fixed;
   g->off_ring = fixed;
+  g->off_bar = fixed;
   g->smem_bytes = fixed + (int64_t)nw * ns * slot;
   return FI_OK;
 }
 
 static int geometry_for(int pipe, int64_t m, int64_t n, int64_t k, int S, int r, int ctas, int sms, GemvGeometry* g) {
   return pipe == kPipeRing ? gemv_geometry(m, n, k, S, r, ctas, sms, g)
-                           : gemv_stream_geometry(m, n, k, S, r, ctas, sms, g);
+                           : gemv_stream_geometry(m, n, k, S, r, ctas, sms, g, pipe == kPipeOverlap);
 }
 
 // Device-sized split (PR #4038, Description, "What it does": the device-sized GEMV split): the fewest splits S
@@ -254,9 +256,9 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
   const int rsel = var & 0xF;
   const bool pipe_auto = (var >> 4) == kPipeAuto;
   int pipe = pipe_auto ? kPipeStream : var >> 4;
-  if (var < 0 || pipe > kPipeRing || rsel > 8)
-    return set_error(FI_ERR_INVALID_ARG, "GEMV variant 0x%x: rows must be 0, 1, 2, 4 or 8 and the pipeline 0, 1 or 2",
-                     var);
+  if (var < 0 || pipe > kPipeOverlap || rsel > 8)
+    return set_error(FI_ERR_INVALID_ARG,
+                     "GEMV variant 0x%x: rows must be 0, 1, 2, 4 or 8 and the pipeline 0, 1, 2 or 3", var);
   int S = S_req;
   if (S == 0) {
     const int rc = gemv_knee(pipe, n, k, sms, kGemvMaxM, 0, ctas, &S);
@@ -312,7 +314,7 @@ static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req,
   out->grid_x = (int32_t)std::max<int64_t>(1, (n + kMmaTileRows - 1) / kMmaTileRows);
   out->grid_y = 1;
   out->threads = kMmaThreads;
-  out->smem_bytes = (int32_t)mma_smem_bytes();
+  out->smem_bytes = (int32_t)mma_smem_bytes(mma_m_pad(m));
   out->workspace_bytes = (m > 0 && k > 0) ? mma_workspace_bytes(m, k) : 0;
   return FI_OK;
 }
@@ -465,6 +467,9 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     // whole aligned 16-byte scale pieces per row and iteration: k % 256 == 0 and every split
     // boundary on a multiple of 8 chunks
     a.scale16 = k % 256 == 0 && (k / kChunkK) % (8 * (int64_t)g.S) == 0 ? 1 : 0;
+    // overlapped pipeline: weights that fit the L2 with room to spare (two consecutive calls'
+    // worth) are prefetched into it whole at kernel start, while the preceding call computes
+    a.prefetch_l2 = g.pipeline == kPipeOverlap && n * (k / 2 + k / 16) <= ((int64_t)40 << 20) ? 1 : 0;
     a.debug_stall = g_debug_stall_launches > 0 ? 1 : 0;
     if (g_debug_stall_launches > 0) --g_debug_stall_launches;
     a.stage_bytes = g.stage_bytes;
@@ -490,6 +495,8 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.n = n;
     a.k = k;
     a.m_pad = mma_m_pad(m);
+    a.op_stages = mma_op_stages(a.m_pad);
+    a.stage_bytes = (uint32_t)mma_stage_bytes(a.m_pad);
     a.debug_stall = g_debug_stall_launches > 0 ? 1 : 0;
     if (g_debug_stall_launches > 0) --g_debug_stall_launches;
     a.err = device_error_word();
@@ -580,6 +587,7 @@ int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, 
     for (int R : {0, 1, 2})
       for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, R | (pipe << 4));
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 2, kPipeStream << 4);
+  for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeOverlap << 4);
   cand[nc++] = FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
   fi_tactic_info seen[64];
   int nseen = 0, count = 0;

@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "fi_nvfp4.h"
@@ -19,6 +20,11 @@ void clear_error();
 // SM count of the current device (cached per device).
 int device_sm_count();
 
+// TMA tensor map over `base` (rank dims, innermost first; strides in bytes of dims 1..rank-1;
+// box extents per dim), no interleave, 256-byte L2 promotion, zero fill out of bounds.
+int encode_tensor_map(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base, const uint64_t* dims,
+                      const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swizzle);
+
 // ------------------------------------------------------------------------ GEMV
 constexpr int kGemvConsumerWarps = 16;                    // warps that decode and multiply
 constexpr int kGemvThreads = (kGemvConsumerWarps + 1) * 32;  // + one producer warp
@@ -34,7 +40,7 @@ constexpr int kStreamIters = 2;                            // chunk iterations p
 constexpr int kStreamCellBytes = 32 * 16 + 32 * 4;         // one iteration of one row: code cells + scale words
 constexpr int kStreamHalfBudget = 228 * 1024 / 2 - 1024;   // dynamic shared memory per CTA, two CTAs per SM
 // pipelines (the high nibble of the GEMV tactic variant)
-constexpr int kPipeAuto = 0, kPipeStream = 1, kPipeRing = 2;
+constexpr int kPipeAuto = 0, kPipeStream = 1, kPipeRing = 2, kPipeOverlap = 3;
 
 // Activation rows the GEMV kernel instance for m is compiled for (1, 2, 4, ..., 32).
 inline int gemv_mt(int64_t m) {
@@ -68,7 +74,7 @@ int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_p
 // The same for the per-warp async-copy pipeline: R rows per item (0 = automatic), ring slots
 // per warp (4, else 2 when the activations leave room for only two).
 int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int ctas_per_sm, int sms,
-                         GemvGeometry* g);
+                         GemvGeometry* g, bool overlap = false);
 
 struct GemvArgs {
   const uint16_t* A;
@@ -86,6 +92,7 @@ struct GemvArgs {
   int threads;         // threads per CTA
   int pdl;             // launch with programmatic stream serialization
   int scale16;         // stream pipeline: copy the E4M3 scales in aligned 16-byte pieces (k % 256 == 0, splits on 8 chunks)
+  int prefetch_l2;     // stream pipeline: each warp asks the L2 to prefetch its whole weight range first
   int debug_stall;     // test hook: the producer issues nothing (consumer waits time out)
   int64_t stage_bytes, off_as, off_bar, off_ring, smem_bytes;
   uint64_t timeout_ns; // limit of every mbarrier wait
@@ -100,11 +107,15 @@ int gemv_read_error(unsigned* bits);
 constexpr int kMmaTileRows = 256;
 constexpr int kMmaKStep = 64;
 constexpr int kMmaMaxM = 256;
-constexpr int kMmaThreads = 14 * 32;
+constexpr int kMmaThreads = 15 * 32;
 inline int mma_m_pad(int64_t m) { return (int)((m + 15) / 16 * 16); }
 inline int64_t mma_rs_offset(int64_t m, int64_t k) { return round_up((int64_t)mma_m_pad(m) * k * 2, 256); }
 inline int64_t mma_workspace_bytes(int64_t m, int64_t k) { return mma_rs_offset(m, k) + (int64_t)mma_m_pad(m) * 4; }
-int64_t mma_smem_bytes();
+// operand stages (decoded weights + activation tile of one 64-k step): as many as fit, 2..4
+constexpr int kMmaMaxOpStages = 4;
+inline int64_t mma_stage_bytes(int m_pad) { return (int64_t)kMmaTileRows * 128 + round_up((int64_t)m_pad * 128, 1024); }
+int mma_op_stages(int m_pad);
+int64_t mma_smem_bytes(int m_pad);
 
 struct MmaArgs {
   const uint16_t* A;
@@ -116,6 +127,8 @@ struct MmaArgs {
   float* rs;      // workspace: per-row inverse scales [m_pad]
   int64_t m, n, k;
   int m_pad;
+  int op_stages;        // operand stages in shared memory (mma_op_stages)
+  uint32_t stage_bytes; // bytes of one operand stage (mma_stage_bytes)
   int debug_stall;      // test hook: the producer issues nothing (the waits time out)
   unsigned* err;        // the device error word
   uint64_t timeout_ns;  // limit of every mbarrier wait

@@ -9,18 +9,19 @@
 //    by act_to_f16_kernel to f16 times a per-row power of two that puts the row maximum in
 //    [2^14, 2^15) (exact for every element within 2^29 of its row maximum), so the tensor core
 //    accumulates sum_k W'[i][k] * A'[j][k] in fp32 and one per-row factor undoes the scale.
-//  * Roles (one CTA per 256 weight rows, 14 warps):
-//      warp 0      TMA producer: raw codes of the tile (256 rows x 32 bytes per 64-k step) into
-//                  a 4-stage ring, issued before the grid-dependency wait (weights never depend
-//                  on the preceding kernel); f16 activation tiles (m_pad rows x 64 k, 128-byte
-//                  swizzled) into a 2-stage ring;
+//  * Roles (one CTA per 256 weight rows, 15 warps):
+//      warp 0      TMA producer of the raw codes of the tile (256 rows x 32 bytes per 64-k step)
+//                  into a 4-stage ring, issued before the grid-dependency wait (weights never
+//                  depend on the preceding kernel);
+//      warp 10     TMA producer of the f16 activation tiles (m_pad rows x 64 k, 128-byte
+//                  swizzled) into the operand stages (2 to 4, as many as shared memory holds);
 //      warps 2-9   decode: one weight row per thread, codes -> f16 (cvt.rn.f16x2.e2m1x2) times
 //                  the block scale (exact f16 multiply), stored in the 128-byte-swizzled
-//                  K-major layout the MMA reads;
+//                  K-major layout the MMA reads; the block scales are loaded 8-11 steps ahead;
 //      warp 1      TMEM allocation and, from one thread, the MMAs: per 64-k step 4 K=16 steps x
 //                  2 M=128 halves, N = m_pad, accumulating in TMEM; tcgen05.commit frees the
 //                  stage;
-//      warps 10-13 epilogue: tcgen05.ld of the accumulator, out[j][i] = bf16_rn(D[i][j] *
+//      warps 11-14 epilogue: tcgen05.ld of the accumulator, out[j][i] = bf16_rn(D[i][j] *
 //                  rs[j] * gscale).
 //  * The weight tile is decoded once per call (the activations, m_pad <= 256 rows, are one MMA
 //    N tile), so the decode work is one cvt and one f16 multiply per two codes.
@@ -32,10 +33,8 @@
 // on its weight row and activation row); results are deterministic run to run.
 #include <cstdint>
 #include <cstring>
-#include <mutex>
 
 #include <cuda.h>
-#include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -45,17 +44,16 @@ namespace fi {
 
 namespace {
 
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpDq0 = 2, kDqWarps = 8, kWarpEpi0 = 10, kEpiWarps = 4;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpDq0 = 2, kDqWarps = 8, kWarpAct = 10, kWarpEpi0 = 11, kEpiWarps = 4;
 static_assert((kWarpEpi0 + kEpiWarps) * 32 == kMmaThreads, "warp roles cover the CTA");
-static_assert(kWarpDq0 + kDqWarps == kWarpEpi0 && kDqWarps * 32 == kMmaTileRows, "one decode thread per tile row");
-constexpr int kOpStages = 2, kRawStages = 4;
+static_assert(kWarpDq0 + kDqWarps == kWarpAct && kWarpAct + 1 == kWarpEpi0 && kDqWarps * 32 == kMmaTileRows,
+              "one decode thread per tile row");
+constexpr int kRawStages = 4;
+constexpr uint32_t kRawBytes = kMmaTileRows * 32;  // 256 rows x 32 code bytes
 constexpr uint32_t kWopBytes = kMmaTileRows * 128;  // 256 rows x 64 f16, 128-byte swizzled
-constexpr uint32_t kActBytes = 256 * 128;           // up to 256 activation rows x 64 f16
-constexpr uint32_t kStageBytes = kWopBytes + kActBytes;
-constexpr uint32_t kRawBytes = kMmaTileRows * 32;   // 256 rows x 32 code bytes
-// barriers: raw_full, raw_empty, act_full, op_full, op_empty, tmem_full, drain
-constexpr int kNumBars = 2 * kRawStages + 3 * kOpStages + 2;
-constexpr uint32_t kBarOff = kOpStages * kStageBytes + kRawStages * kRawBytes;
+// barriers: raw_full, raw_empty, then act_full, op_full, op_empty per operand stage, tmem_full,
+// drain
+constexpr int kNumBars = 2 * kRawStages + 3 * kMmaMaxOpStages + 2;
 
 // Shared-memory matrix descriptor of a K-major tile with 128-byte rows in the 128-byte swizzle
 // (8-row atoms of 1024 bytes): start address >> 4 in bits 0-13, leading-dimension offset 1
@@ -182,21 +180,24 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ volatile int abort_flag;
   __shared__ uint32_t tmem_slot;
-  // 1024-byte aligned base for the swizzled tiles
+  // 1024-byte aligned base for the swizzled tiles: the raw-code ring, then NST operand stages
+  // (decoded weights, then activations, each stage stage_bytes), then the barriers
+  const int NST = p.op_stages;
+  const uint32_t stage_bytes = p.stage_bytes;
   const uint32_t raw_s = smem_addr(smem_raw);
   const uint32_t base = (raw_s + 1023u) & ~1023u;
   uint8_t* const basep = smem_raw + (base - raw_s);
-  uint64_t* const bars = reinterpret_cast<uint64_t*>(basep + kBarOff);
+  uint64_t* const bars = reinterpret_cast<uint64_t*>(basep + kRawStages * kRawBytes + (uint32_t)NST * stage_bytes);
   uint64_t* const raw_full = bars;
   uint64_t* const raw_empty = bars + kRawStages;
   uint64_t* const act_full = bars + 2 * kRawStages;
-  uint64_t* const op_full = act_full + kOpStages;
-  uint64_t* const op_empty = op_full + kOpStages;
-  uint64_t* const tmem_full = op_empty + kOpStages;
+  uint64_t* const op_full = act_full + kMmaMaxOpStages;
+  uint64_t* const op_empty = op_full + kMmaMaxOpStages;
+  uint64_t* const tmem_full = op_empty + kMmaMaxOpStages;
   uint64_t* const drain = tmem_full + 1;
-  auto wop_addr = [&](int st) { return base + (uint32_t)st * kStageBytes; };
-  auto act_addr = [&](int st) { return base + (uint32_t)st * kStageBytes + kWopBytes; };
-  auto raw_addr = [&](int st) { return base + kOpStages * kStageBytes + (uint32_t)st * kRawBytes; };
+  auto raw_addr = [&](int st) { return base + (uint32_t)st * kRawBytes; };
+  auto wop_addr = [&](int st) { return base + kRawStages * kRawBytes + (uint32_t)st * stage_bytes; };
+  auto act_addr = [&](int st) { return wop_addr(st) + kWopBytes; };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n = p.n, k = p.k;
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       mbar_init(&raw_full[i], 1);
       mbar_init(&raw_empty[i], kDqWarps);
     }
-    for (int i = 0; i < kOpStages; ++i) {
+    for (int i = 0; i < NST; ++i) {
       mbar_init(&act_full[i], 1);
       mbar_init(&op_full[i], kDqWarps);
       mbar_init(&op_empty[i], 1);
@@ -233,40 +234,50 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   pdl_launch_dependents();
 
   if (warp == kWarpTma) {
-    // ------------------------------------------------------------------------ producer
+    // ------------------------------------------------------------------------ producers
+    // one thread streams the raw codes, gated by the decode warps freeing raw stages (the
+    // activation tiles have their own warp: two lanes of one warp in divergent loops with
+    // suspending waits progress one at a time, which serialised the two streams)
     if (lane == 0 && !p.debug_stall) {
-      int raw_issued = 0, act_issued = 0;
+      int issued = 0;
       const int pro = KS < kRawStages ? KS : kRawStages;
       for (int s = 0; s < pro; ++s) {
         mbar_arrive_expect_tx(&raw_full[s], kRawBytes);
         tma_load_2d(raw_addr(s), &tmap_w, s * 32, (int)w0, smem_addr(&raw_full[s]));
-        ++raw_issued;
+        ++issued;
       }
-      pdl_wait();
-      for (int s = 0; s < KS && !abort_flag; ++s) {
-        const int os = s % kOpStages;
-        if (s >= kOpStages &&
-            !mbar_wait_bounded(&op_empty[os], (uint32_t)((s / kOpStages - 1) & 1), &abort_flag, p.timeout_ns, p.err, 2u))
+      for (int s = 0; s + kRawStages < KS && !abort_flag; ++s) {
+        const int rs = s % kRawStages;
+        if (!mbar_wait_bounded(&raw_empty[rs], (uint32_t)((s / kRawStages) & 1), &abort_flag, p.timeout_ns, p.err,
+                               2u))
           break;
-        mbar_arrive_expect_tx(&act_full[os], (uint32_t)N * 128u);
-        tma_load_2d(act_addr(os), &tmap_a, s * kMmaKStep, 0, smem_addr(&act_full[os]));
-        ++act_issued;
-        const int sn = s + kRawStages;
-        if (sn < KS) {
-          const int rs = s % kRawStages;
-          if (!mbar_wait_bounded(&raw_empty[rs], (uint32_t)((s / kRawStages) & 1), &abort_flag, p.timeout_ns, p.err,
-                                 2u))
-            break;
-          mbar_arrive_expect_tx(&raw_full[rs], kRawBytes);
-          tma_load_2d(raw_addr(rs), &tmap_w, sn * 32, (int)w0, smem_addr(&raw_full[rs]));
-          ++raw_issued;
-        }
+        mbar_arrive_expect_tx(&raw_full[rs], kRawBytes);
+        tma_load_2d(raw_addr(rs), &tmap_w, (s + kRawStages) * 32, (int)w0, smem_addr(&raw_full[rs]));
+        ++issued;
       }
       // drain: every copy issued must have landed before the CTA exits
-      for (int s = raw_issued - kRawStages < 0 ? 0 : raw_issued - kRawStages; s < raw_issued; ++s)
+      for (int s = issued - kRawStages < 0 ? 0 : issued - kRawStages; s < issued; ++s)
         drain_wait(&raw_full[s % kRawStages], (uint32_t)((s / kRawStages) & 1), p.timeout_ns, p.err);
-      for (int s = act_issued - kOpStages < 0 ? 0 : act_issued - kOpStages; s < act_issued; ++s)
-        drain_wait(&act_full[s % kOpStages], (uint32_t)((s / kOpStages) & 1), p.timeout_ns, p.err);
+    }
+  } else if (warp == kWarpAct) {
+    // --------------------------------------------------------------- activation producer
+    // one thread streams the f16 activation tiles, gated by the MMAs freeing operand stages
+    if (lane == 0 && !p.debug_stall) {
+      pdl_wait();  // the activations come from the conversion kernel launched just before
+      int issued = 0, os = 0;
+      uint32_t ph = 0;  // phase of op_empty[os] to wait for once every stage has been used
+      for (int s = 0; s < KS && !abort_flag; ++s) {
+        if (s >= NST && !mbar_wait_bounded(&op_empty[os], ph, &abort_flag, p.timeout_ns, p.err, 2u)) break;
+        mbar_arrive_expect_tx(&act_full[os], (uint32_t)N * 128u);
+        tma_load_2d(act_addr(os), &tmap_a, s * kMmaKStep, 0, smem_addr(&act_full[os]));
+        ++issued;
+        if (++os == NST) {
+          os = 0;
+          if (s >= NST) ph ^= 1u;
+        }
+      }
+      for (int s = issued - NST < 0 ? 0 : issued - NST; s < issued; ++s)
+        drain_wait(&act_full[s % NST], (uint32_t)((s / NST) & 1), p.timeout_ns, p.err);
     }
   } else if (warp >= kWarpDq0 && warp < kWarpDq0 + kDqWarps) {
     // -------------------------------------------------------------------------- decode
@@ -277,15 +288,42 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     const uint8_t* srow = p.Ws + (valid ? row : 0) * rs_s;
     const uint32_t wdst = (uint32_t)(r >> 7) * (kWopBytes / 2) + (uint32_t)(r & 127) * 128u;
     const uint32_t swz = (uint32_t)(r & 7);
+    // The row's four E4M3 scales of step s are the 4 bytes at srow + 4s. They are loaded in
+    // groups of 4 steps, three groups ahead of their use, so the global-memory latency of the
+    // scales (cold: they are read once per call) is off the per-step path.
+    const bool al16 = rs_s % 16 == 0;
+    auto load_group = [&](int gi) -> uint4 {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      const int s0 = gi * 4;
+      if (valid && s0 < KS) {
+        if (al16 && s0 + 3 < KS) {
+          v = ldg_v4(srow + s0 * 4);
+        } else {
+          v.x = ldg_u32(srow + s0 * 4);
+          if (s0 + 1 < KS) v.y = ldg_u32(srow + s0 * 4 + 4);
+          if (s0 + 2 < KS) v.z = ldg_u32(srow + s0 * 4 + 8);
+          if (s0 + 3 < KS) v.w = ldg_u32(srow + s0 * 4 + 12);
+        }
+      }
+      return v;
+    };
+    uint4 sg0 = load_group(0), sg1 = load_group(1), sg2 = load_group(2);
+    int os = 0;        // operand stage of step s
+    uint32_t eph = 0;  // phase of op_empty[os] to wait for (steps s >= NST)
     for (int s = 0; s < KS; ++s) {
-      const int rsn = s % kRawStages, os = s % kOpStages;
-      const uint32_t sc4 = valid ? *reinterpret_cast<const uint32_t*>(srow + s * 4) : 0u;
+      const int rsn = s % kRawStages;
+      const int sj = s & 3;
+      const uint32_t sc4 = sj == 0 ? sg0.x : (sj == 1 ? sg0.y : (sj == 2 ? sg0.z : sg0.w));
+      if (sj == 3) {
+        sg0 = sg1;
+        sg1 = sg2;
+        sg2 = load_group(s / 4 + 3);
+      }
       // every lane waits; the warp continues only if all of them saw both phases (a timeout is
       // seen lane by lane, and the warp must stay converged for __syncwarp below)
       const bool ok =
           mbar_wait_bounded(&raw_full[rsn], (uint32_t)((s / kRawStages) & 1), &abort_flag, p.timeout_ns, p.err, 1u) &&
-          (s < kOpStages || mbar_wait_bounded(&op_empty[os], (uint32_t)((s / kOpStages - 1) & 1), &abort_flag,
-                                              p.timeout_ns, p.err, 1u));
+          (s < NST || mbar_wait_bounded(&op_empty[os], eph, &abort_flag, p.timeout_ns, p.err, 1u));
       if (!__all_sync(0xffffffffu, ok)) break;
       const uint4 c0 = lds_v4m(raw_addr(rsn) + (uint32_t)r * 32u);
       const uint4 c1 = lds_v4m(raw_addr(rsn) + (uint32_t)r * 32u + 16u);
@@ -313,14 +351,18 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         mbar_arrive(&op_full[os]);
         mbar_arrive(&raw_empty[rsn]);
       }
+      if (++os == NST) {
+        os = 0;
+        if (s >= NST) eph ^= 1u;
+      }
     }
   } else if (warp == kWarpMma) {
     // ----------------------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t idesc = f16_idesc(128, N);
+      int os = 0;
+      uint32_t par = 0;  // phase of act_full[os] and op_full[os] for step s
       for (int s = 0; s < KS; ++s) {
-        const int os = s % kOpStages;
-        const uint32_t par = (uint32_t)((s / kOpStages) & 1);
         if (!mbar_wait_bounded(&act_full[os], par, &abort_flag, p.timeout_ns, p.err, 4u)) break;
         if (!mbar_wait_bounded(&op_full[os], par, &abort_flag, p.timeout_ns, p.err, 4u)) break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -334,6 +376,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
           }
         }
         umma_commit(&op_empty[os]);  // frees the stage when these MMAs have read it
+        if (++os == NST) {
+          os = 0;
+          par ^= 1u;
+        }
       }
       umma_commit(tmem_full);  // the accumulator is complete when every MMA issued has finished
       umma_commit(drain);
@@ -380,44 +426,34 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
 
 namespace {
 
-// cuTensorMapEncodeTiled from the driver, found once through the runtime (no libcuda link).
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static std::once_flag once;
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    else
-      (void)cudaGetLastError();
-  });
-  return fn;
-}
-
 int encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,
               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return set_error(FI_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return set_error(FI_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-  return FI_OK;
+  const uint64_t dims[2] = {inner, outer};
+  const uint64_t strides[1] = {row_bytes};
+  const uint32_t box[2] = {box_inner, box_outer};
+  return encode_tensor_map(map, type, 2, base, dims, strides, box, swizzle);
 }
 
 }  // namespace
 
-int64_t mma_smem_bytes() { return (int64_t)kBarOff + kNumBars * 8 + 1024; }
+int mma_op_stages(int m_pad) {
+  const int64_t per = mma_stage_bytes(m_pad);
+  const int64_t room = kSmemBudget - 1024 - (int64_t)kRawStages * kRawBytes - kNumBars * 8;
+  return (int)std::max<int64_t>(2, std::min<int64_t>(kMmaMaxOpStages, room / per));
+}
+
+int64_t mma_smem_bytes(int m_pad) {
+  return 1024 + (int64_t)kRawStages * kRawBytes + (int64_t)mma_op_stages(m_pad) * mma_stage_bytes(m_pad) +
+         kNumBars * 8;
+}
 
 int launch_mma(const MmaArgs& a, cudaStream_t stream) {
   if (a.k % kMmaKStep != 0 || a.m_pad < 16 || a.m_pad > kMmaMaxM || a.m_pad % 16 != 0)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA path: k must be a multiple of %d and m <= %d", kMmaKStep,
                      kMmaMaxM);
+  if (a.op_stages < 2 || a.op_stages > kMmaMaxOpStages || (int64_t)a.stage_bytes != mma_stage_bytes(a.m_pad))
+    return set_error(FI_ERR_INVALID_ARG, "MMA path: %d operand stages of %u bytes do not match m_pad=%d", a.op_stages,
+                     a.stage_bytes, a.m_pad);
   CUtensorMap tmap_a, tmap_w;
   // activations: f16 [m_pad, k], box 64 k x m_pad rows, 128-byte swizzle (the MMA's B operand)
   int rc = encode_2d(&tmap_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.a16, (uint64_t)a.k, (uint64_t)a.m_pad,
@@ -432,8 +468,8 @@ int launch_mma(const MmaArgs& a, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return set_cuda_error("cudaGetDevice");
   if (!configured[dev]) {
-    if (cudaFuncSetAttribute(mma_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)mma_smem_bytes()) != cudaSuccess)
+    if (cudaFuncSetAttribute(mma_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) !=
+        cudaSuccess)
       return set_cuda_error("cudaFuncSetAttribute(mma smem)");
     configured[dev] = 1;
   }
@@ -453,7 +489,7 @@ int launch_mma(const MmaArgs& a, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((a.n + kMmaTileRows - 1) / kMmaTileRows));
   cfg.blockDim = dim3(kMmaThreads);
-  cfg.dynamicSmemBytes = (size_t)mma_smem_bytes();
+  cfg.dynamicSmemBytes = (size_t)mma_smem_bytes(a.m_pad);
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;

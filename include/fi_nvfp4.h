@@ -235,22 +235,23 @@ FI_API size_t fi_mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int64_t tac
 FI_API int fi_set_workspace(void* ptr, size_t bytes);
 
 /* ------------------------------------------------------------ failure detection
- * Every wait of one warp on another inside the kernels (the ring pipeline's mbarriers) is
- * bounded in time: when a wait runs out, the kernel records a bit in a sticky per-device
- * error word, stops computing, lets its in-flight copies land and returns; the outputs of
- * that call are then undefined. (The stream pipeline has no such waits: each thread waits
- * only for its own copies.) The library has no counterpart on the pages; it exists so that a
- * stuck pipeline ends with an error instead of a hung GPU.
+ * Every mbarrier wait inside the kernels (the ring pipeline's and the MMA path's) is bounded
+ * in time: when a wait runs out, the kernel records a bit in a sticky per-device error word,
+ * stops computing, lets its in-flight copies land and returns; the outputs of that call are
+ * then undefined. (The stream pipeline has no waits between threads: each thread waits only
+ * for its own copies.) The library has no counterpart on the pages; it exists so that a stuck
+ * pipeline ends with an error instead of a hung GPU.
  */
 
-/* Read and clear the current device's sticky kernel error word (0 = no error; bit 0: a
- * consumer wait ran out, bit 1: a producer wait ran out, bit 2: the final drain ran out).
- * Synchronizes the device. */
+/* Read and clear the current device's sticky kernel error word (0 = no error): bit 0 a
+ * consumer (decode) wait, bit 1 a producer wait, bit 2 a final drain, bit 3 (MMA) a drain
+ * before exit, bit 4 (MMA) the epilogue's wait ran out. Synchronizes the device. */
 FI_API int fi_get_device_error(unsigned* code);
 
-/* Test hooks. FI_DEBUG_STALL_PRODUCER: the producer warp of the next `value` GEMV launches
- * issues no copies, so their waits run out (exercises the path above without a GPU fault;
- * only ring-pipeline launches have a producer, other launches still count down).
+/* Test hooks. FI_DEBUG_STALL_PRODUCER: the producers of the next `value` launches (the ring
+ * pipeline's producer warp, the MMA path's producers) issue no copies, so their waits run out
+ * (exercises the path above without a GPU fault; stream-pipeline launches have no producer
+ * and still count down).
  * FI_DEBUG_WAIT_TIMEOUT_NS: limit of every kernel wait in ns (default 1e9). */
 #define FI_DEBUG_STALL_PRODUCER 1
 #define FI_DEBUG_WAIT_TIMEOUT_NS 2

@@ -125,7 +125,7 @@ def test_workspace_bytes():
     (32, 64, 14336, fi.make_tactic(0, 1, 0, 1), -2),      # A slice does not fit shared memory
     (32, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),       # one row per stage above m = 8
     (5, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),        # two rows per stage above m = 4
-    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x32), -1),     # pipeline 3
+    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x42), -1),     # pipeline 4
     (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x19), -1),     # rows 9 on the stream pipeline
     (1, 8, 65536, fi.make_tactic(0, 1, 0, 0x22), -2),     # ring: two 36 KB rows per stage do not fit twice
     (1, 8, 65536, fi.make_tactic(0, 1, 2, 0x11), -2),     # stream, half-SM CTAs: 128 KB of activations
@@ -192,7 +192,7 @@ def test_mma_tactic_resolution():
     t = fi.make_tactic(fi.KIND_MMA, 1, 0, 0)
     info = fi.resolve_tactic(256, 152064, 5120, t, B200_SMS)
     assert info["kind"] == fi.KIND_MMA and info["splits"] == 1
-    assert info["grid_x"] == 152064 // 256 and info["threads"] == 14 * 32
+    assert info["grid_x"] == 152064 // 256 and info["threads"] == 15 * 32
     assert 0 < info["smem_bytes"] <= 227 * 1024
     # workspace: f16 activations [256, k] then 256 fp32 row scales
     assert info["workspace_bytes"] == 256 * 5120 * 2 + 256 * 4

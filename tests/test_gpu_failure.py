@@ -43,3 +43,4 @@ def test_stalled_pipeline_reports_timeout_and_recovers():
     torch.cuda.synchronize()
     _gpu.assert_within_tolerance(_gpu.host_bits(out), ref, "after recovery")
     assert fi.get_device_error() == 0
+

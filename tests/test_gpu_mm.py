@@ -53,6 +53,8 @@ def test_tiny_workload_every_tactic():
     (2, 1, 32, 5),          # single chunk, single row
     (16, 300, 2048, 6),
     (32, 96, 1024, 7),
+    (1, 1001, 1536, 8),     # tensor-copy items: 48 chunks (a half-filled last iteration), odd n
+    (4, 515, 5120, 9),      # tensor-copy items: 160 chunks (an empty last iteration), partial group
 ])
 def test_parity_spanning_tiles(m, n, k, seed):
     A = inputs.activations(m, k, seed, outliers=True)
