@@ -52,8 +52,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per launch of the GEMV kernel (dram__bytes_read.sum + dram__bytes_write.sum)
 # from one ncu capture per shape, keyed by the sha256 of the kernel source they were taken
 # on; ignored (traffic = null) when the source has changed since.
-NCU_TRAFFIC = {"source_sha256": "b54394e288e1eed97b4504cff3d0a7151a5ceddae72ada637a92a20c10f328ac",
-               "bytes": {"14336x4096": 33_089_536, "4096x14336": 33_110_784}}
+NCU_TRAFFIC = {"source_sha256": "590fe5d56d1b360e49ebeb493d1af06ca603f71cd5ebe66af27d6a52e83206fa",
+               "bytes": {"14336x4096": 33_105_481, "4096x14336": 33_125_888}}
 # the roofline's dominant-kernel figure: the GEMV alone (split 1, one launch per call) on the
 # two 33 MB serving shapes
 ROOFLINE_SHAPES = [(4096, 14336), (14336, 4096)]
@@ -402,6 +402,39 @@ def run_fi(args, rank: int, world: int) -> dict | None:
     }
 
 
+def mma_wave(args) -> None:
+    """Profiling case for the tensor-core path: one wave of CTAs (n = 148 x 256 rows, k = 5120,
+    the lm_head-like k) at m = 64 and 256, each timed over 10 eager calls after 3 warm-up
+    calls. Small enough for a multi-pass ncu capture of single launches."""
+    import torch
+
+    import bf16_activations_nvfp4_b200 as fi
+    from bf16_activations_nvfp4_b200 import inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    n, k = 148 * 256, LM_HEAD[1]
+    W = torch.from_numpy(inputs.weights(n, k, seed=0)).to(dev)
+    Wq, Ws, g = fi.pack_weights(W)
+    del W
+    ws = torch.empty(max(fi.workspace_bytes(m, n, k) for m in (64, 256)) // 4 + 64, dtype=torch.float32, device=dev)
+    fi.set_workspace(ws)
+    for m in (64, 256):
+        A = torch.from_numpy(inputs.activations(m, k, seed=0).view(np.int16)).view(torch.bfloat16).to(dev)
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            fi.mm_bf16_fp4(A, Wq, Ws, g, out=out)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            fi.mm_bf16_fp4(A, Wq, Ws, g, out=out)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        us = e0.elapsed_time(e1) * 1e3 / 10
+        print(json.dumps({"n": n, "k": k, "m": m, "kind": fi.resolve_tactic(m, n, k)["kind"], "us": round(us, 2),
+                          "tflops": round(2 * m * n * k / us / 1e6, 1)}), flush=True)
+
+
 def sweep(args) -> None:
     """Print per-call µs of every listed tactic for each shape (cold-L2 graph method)."""
     import torch
@@ -537,6 +570,8 @@ def main(argv=None) -> int:
     ap.add_argument("--sweep", action="store_true", help="print per-call µs of every listed tactic and exit")
     ap.add_argument("--m", type=int, default=1, help="activation rows for --sweep")
     ap.add_argument("--no-lm-head", action="store_true", help="skip the lm_head-like GEMM measurement")
+    ap.add_argument("--mma-wave", action="store_true",
+                    help="profiling case: the tensor-core path on one wave of CTAs at m = 64 and 256, then exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -555,6 +590,9 @@ def main(argv=None) -> int:
         return 0
     if args.sweep:
         sweep(args)
+        return 0
+    if args.mma_wave:
+        mma_wave(args)
         return 0
 
     if world > 1:

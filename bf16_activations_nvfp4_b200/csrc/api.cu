@@ -159,7 +159,7 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
   const int64_t as_bytes = round_up(m * nch * 8, 128);
   const int rmax = std::min(4, gemv_rows_per_stage_max(m));  // registers: at most 4 rows per item
   int64_t r = r_req;
-  if (r == 0) r = std::min(ctas == 2 ? 4 : 2, rmax);
+  if (r == 0) r = std::min(ctas == 2 && !overlap ? 4 : 2, rmax);
   if (r < 1 || r > rmax || (r & (r - 1)) != 0)
     return set_error(FI_ERR_INVALID_ARG, "GEMV rows per item must be a power of two in 1..%d for m=%lld", rmax,
                      (long long)m);
@@ -195,9 +195,50 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
   return FI_OK;
 }
 
+// Register pipeline: shared memory holds only the staged activations; each warp keeps
+// kRegDepth chunk iterations of its rows in registers. CTAs of up to 16 warps (one per SM) or
+// up to 8 (two per SM), spread over every SM like the stream pipeline's.
+static int gemv_reg_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int ctas_per_sm, int sms,
+                             GemvGeometry* g) {
+  const int64_t C = k / kChunkK;
+  const int64_t nch = (C + S - 1) / S;
+  const int ctas = ctas_per_sm > 0 ? ctas_per_sm : 1;
+  if (ctas > 2) return set_error(FI_ERR_INVALID_ARG, "GEMV register pipeline: at most 2 CTAs per SM");
+  int nw = ctas == 1 ? 16 : 8;
+  const int64_t budget = ctas == 1 ? kSmemBudget : kStreamHalfBudget;
+  const int64_t a_bytes = round_up(m * ((nch + 31) / 32) * 2048, 128);
+  const int64_t as_bytes = round_up(m * nch * 8, 128);
+  if (a_bytes + as_bytes > budget)
+    return set_error(FI_ERR_UNSUPPORTED_SHAPE,
+                     "GEMV: m=%lld over %lld k per split does not fit shared memory; use more splits", (long long)m,
+                     (long long)(nch * kChunkK));
+  const int rmax = std::min(2, gemv_rows_per_stage_max(m));  // the register ring of 4 rows would spill
+  int64_t r = r_req ? r_req : rmax;
+  if (r < 1 || r > rmax || (r & (r - 1)) != 0)
+    return set_error(FI_ERR_INVALID_ARG, "GEMV rows per warp must be a power of two in 1..%d for m=%lld", rmax,
+                     (long long)m);
+  const int64_t groups = (n + r - 1) / r;
+  const int64_t gx_cap = std::max<int64_t>(1, (int64_t)sms * ctas / S);
+  if ((groups + nw - 1) / nw < gx_cap) nw = (int)std::max<int64_t>(4, (groups + gx_cap - 1) / gx_cap);
+  g->pipeline = kPipeReg;
+  g->threads = nw * 32;
+  g->S = S;
+  g->RS = (int)r;
+  g->stages = kRegDepth;
+  g->ctas_per_sm = ctas;
+  g->grid_x = (int)std::max<int64_t>(1, std::min<int64_t>(gx_cap, (groups + nw - 1) / nw));
+  g->stage_bytes = 0;
+  g->off_as = a_bytes;
+  g->off_bar = a_bytes + as_bytes;
+  g->off_ring = a_bytes + as_bytes;
+  g->smem_bytes = a_bytes + as_bytes;
+  return FI_OK;
+}
+
 static int geometry_for(int pipe, int64_t m, int64_t n, int64_t k, int S, int r, int ctas, int sms, GemvGeometry* g) {
-  return pipe == kPipeRing ? gemv_geometry(m, n, k, S, r, ctas, sms, g)
-                           : gemv_stream_geometry(m, n, k, S, r, ctas, sms, g, pipe == kPipeOverlap);
+  if (pipe == kPipeRing) return gemv_geometry(m, n, k, S, r, ctas, sms, g);
+  if (pipe == kPipeReg) return gemv_reg_geometry(m, n, k, S, r, ctas, sms, g);
+  return gemv_stream_geometry(m, n, k, S, r, ctas, sms, g, pipe == kPipeOverlap);
 }
 
 // Device-sized split (PR #4038, Description, "What it does": the device-sized GEMV split): the fewest splits S
@@ -233,10 +274,20 @@ static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms,
 static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms) {
   if (m <= kDefaultGemvMaxM) {
     const int64_t m_fit = m <= 1 ? 1 : (m <= 8 ? 8 : kGemvMaxM);
-    // stream pipeline with its automatic CTA shape and rows per item (see gemv_stream_geometry)
+    // stream pipeline with its automatic CTA shape and rows per item (see gemv_stream_geometry);
+    // weights of at most 12 MB take the overlapped variant (half-SM CTAs, one per SM, weights
+    // prefetched into L2 while the preceding call computes). Measured on B200 at m = 1 in
+    // PDL-chained graphs: 2048 x 7168 4.03 against 4.33 us, 4096 x 4096 3.73 against 4.19 us;
+    // from 15 MB on the whole-SM CTAs were faster.
+    // Where k % 256 != 0 the stream pipeline takes its general path (4-byte scale words, lane
+    // predicates): there the register pipeline with two CTAs per SM was faster (10304 x 2688:
+    // 6.60 against 7.46 us).
+    const bool small = n * (k / 2 + k / 16) <= ((int64_t)12 << 20);
+    const int pipe = small ? kPipeOverlap : (k % 256 != 0 ? kPipeReg : kPipeStream);
+    const int ctas = pipe == kPipeReg ? 2 : 0;
     int S = 1;
-    if (gemv_knee(kPipeStream, n, k, num_sms, m_fit, 0, 0, &S) != FI_OK) S = 1;
-    return FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeStream << 4);
+    if (gemv_knee(pipe, n, k, num_sms, m_fit, 0, ctas, &S) != FI_OK) S = 1;
+    return FI_TACTIC(FI_KIND_GEMV, S, ctas, pipe << 4);
   }
   return FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
 }
@@ -256,9 +307,9 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
   const int rsel = var & 0xF;
   const bool pipe_auto = (var >> 4) == kPipeAuto;
   int pipe = pipe_auto ? kPipeStream : var >> 4;
-  if (var < 0 || pipe > kPipeOverlap || rsel > 8)
+  if (var < 0 || pipe > kPipeReg || rsel > 8)
     return set_error(FI_ERR_INVALID_ARG,
-                     "GEMV variant 0x%x: rows must be 0, 1, 2, 4 or 8 and the pipeline 0, 1, 2 or 3", var);
+                     "GEMV variant 0x%x: rows must be 0, 1, 2, 4 or 8 and the pipeline 0 to 4", var);
   int S = S_req;
   if (S == 0) {
     const int rc = gemv_knee(pipe, n, k, sms, kGemvMaxM, 0, ctas, &S);
@@ -588,6 +639,7 @@ int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, 
       for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, R | (pipe << 4));
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 2, kPipeStream << 4);
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeOverlap << 4);
+  for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeReg << 4);
   cand[nc++] = FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
   fi_tactic_info seen[64];
   int nseen = 0, count = 0;

@@ -857,6 +857,163 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_stream_kernel(GemvA
   cp_async_wait<0>();
 }
 
+// ---------------------------------------------------------------------------------------
+// Register pipeline (pipeline 4): the weights go from global memory straight to registers
+// with 16-byte loads, as in the pages' streaming GEMV; nothing is copied to shared memory but
+// the staged activations. Each warp keeps the loads of its next D chunk iterations in flight
+// in a register ring (the loop is unrolled by D so every ring index is static). Same rows per
+// warp, lane-to-chunk mapping and per-chunk arithmetic as the other pipelines, so the same
+// bits for the same S.
+
+// One chunk of R weight rows from registers (codes cq[i], the lane's two scale bytes sc[i]).
+template <int MT, int R>
+__device__ __forceinline__ void chunk_rows_reg(const uint4 (&cq)[R], const uint32_t (&sc)[R], uint32_t ap,
+                                               uint32_t sp, uint32_t a_row, uint32_t as_row, int m,
+                                               float (&acc)[R][MT]) {
+  if (MT == 1) {
+    const uint4 a0 = lds_v4(ap), a1 = lds_v4(ap + 512), a2 = lds_v4(ap + 1024), a3 = lds_v4(ap + 1536);
+    const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                             a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+    const float2 sa = lds_f2(sp);
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      uint32_t wf[16];
+      decode32(cq[i], wf);
+      acc[i][0] = chunk_acc(av, sa, wf, e4m3x2_to_f16x2(sc[i]), acc[i][0]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      uint32_t wf[16];
+      decode32(cq[i], wf);
+      const uint32_t sh = e4m3x2_to_f16x2(sc[i]);
+#pragma unroll
+      for (int r = 0; r < MT; ++r) {
+        if (r < m) {
+          const uint32_t apr = ap + (uint32_t)r * a_row;
+          const uint4 a0 = lds_v4(apr), a1 = lds_v4(apr + 512), a2 = lds_v4(apr + 1024), a3 = lds_v4(apr + 1536);
+          const uint32_t av[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                                   a2.x, a2.y, a2.z, a2.w, a3.x, a3.y, a3.z, a3.w};
+          acc[i][r] = chunk_acc(av, lds_f2(sp + (uint32_t)r * as_row), wf, sh, acc[i][r]);
+        }
+      }
+    }
+  }
+}
+
+template <int MT, int R, int D>
+__global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_reg_kernel(GemvArgs p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int NW = (int)(blockDim.x >> 5);
+  const int m = (int)p.m;
+  const int64_t n = p.n, k = p.k;
+  const int S = p.splits;
+  const int s = blockIdx.y;
+
+  const int64_t C = k / kChunkK;
+  const int64_t c0 = (int64_t)s * C / S;
+  const int nch = (int)((int64_t)(s + 1) * C / S - c0);
+  const int T = (nch + 31) / 32;  // chunk iterations of a row
+
+  // rows of this warp: whole groups of R rows, balanced over all warps of the split
+  const int64_t GW = (int64_t)gridDim.x * NW;
+  const int64_t gw = (int64_t)blockIdx.x * NW + warp;
+  const int64_t ngr = (n + R - 1) / R;
+  const int64_t g_lo = gw * ngr / GW, g_hi = (gw + 1) * ngr / GW;
+  const int64_t r_lo = g_lo * R, r_hi = min(n, g_hi * R);
+  const int Q = (int)(g_hi - g_lo) * T;  // chunk iterations of this warp, row group by row group
+
+  const int64_t rs_q = k / 2, rs_s = k / 16;
+  pdl_launch_dependents();
+
+  // ---- load cursor: iteration (group lg, chunk iteration lt); row i's code and scale pointers
+  // for this lane's chunk
+  int lt = 0, iq = 0;
+  int64_t lj0 = r_lo;
+  const uint8_t* qp[R];
+  const uint8_t* spp[R];
+  auto load_group = [&]() {
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int64_t j = min(lj0 + i, n - 1);  // rows past n load row n-1 and are never written
+      qp[i] = p.Wq + j * rs_q + (c0 + lane) * 16;
+      spp[i] = p.Ws + j * rs_s + (c0 + lane) * 2;
+    }
+  };
+  uint4 rq[D][R];
+  uint32_t rsc[D][R];
+  // load iteration iq into ring slot u (u compile-time at every call site)
+  auto load = [&](uint4 (&q)[R], uint32_t (&sc)[R]) {
+    if (iq < Q && lt * 32 + lane < nch) {
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        q[i] = ldg_stream_v4(qp[i]);
+        sc[i] = ldg_stream_u16(spp[i]);
+      }
+    }
+    if (iq < Q) {
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        qp[i] += 512;
+        spp[i] += 64;
+      }
+      if (++lt == T) {
+        lt = 0;
+        lj0 += R;
+        load_group();
+      }
+    }
+    ++iq;
+  };
+  load_group();
+#pragma unroll
+  for (int u = 0; u < D; ++u) load(rq[u], rsc[u]);
+
+  pdl_wait();
+  stage_activations(p.A, k, m, c0 * kChunkK, nch, reinterpret_cast<uint4*>(smem),
+                    reinterpret_cast<float*>(smem + p.off_as), tid, (int)blockDim.x);
+  __syncthreads();
+  const float g = (S == 1) ? *p.gscale : 1.0f;
+
+  const int GA = (nch + 31) / 32;
+  const uint32_t a_row = (uint32_t)GA * 2048, as_row = (uint32_t)nch * 8;
+  const uint32_t a_lane = smem_addr(smem) + (uint32_t)lane * 16;
+  const uint32_t as_lane = smem_addr(smem + p.off_as) + (uint32_t)lane * 8;
+  float acc[R][MT];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
+  int64_t j0 = r_lo;
+  int ct = 0;
+  uint32_t ac = a_lane, asc = as_lane;
+  for (int q0 = 0; q0 < Q; q0 += D) {
+#pragma unroll
+    for (int u = 0; u < D; ++u) {
+      if (q0 + u < Q) {
+        if (ct * 32 + lane < nch) chunk_rows_reg<MT, R>(rq[u], rsc[u], ac, asc, a_row, as_row, m, acc);
+        load(rq[u], rsc[u]);  // the slot's registers are consumed: refill with iteration q0 + u + D
+        ac += 2048;
+        asc += 256;
+        if (++ct == T) {
+          finish_rows<MT, R>(acc, p, j0, (int)min((int64_t)R, r_hi - j0), m, S, s, g, lane, true);
+#pragma unroll
+          for (int i = 0; i < R; ++i)
+#pragma unroll
+            for (int r = 0; r < MT; ++r) acc[i][r] = 0.0f;
+          ct = 0;
+          ac = a_lane;
+          asc = as_lane;
+          j0 += R;
+        }
+      }
+    }
+  }
+}
+
 namespace {
 
 template <int MT, int RS>
@@ -913,7 +1070,37 @@ int launch_stream_one(const GemvArgs& a, cudaStream_t stream) {
 }
 
 template <int MT, int R>
+int launch_reg(const GemvArgs& a, cudaStream_t stream) {
+  auto kern = gemv_reg_kernel<MT, R, kRegDepth>;
+  static int configured[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return set_cuda_error("cudaGetDevice");
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) != cudaSuccess)
+      return set_cuda_error("cudaFuncSetAttribute(gemv register smem)");
+    configured[dev] = 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.grid_x, (unsigned)a.splits);
+  cfg.blockDim = dim3((unsigned)a.threads);
+  cfg.dynamicSmemBytes = (size_t)a.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return set_cuda_error("gemv register kernel launch");
+  return FI_OK;
+}
+
+template <int MT, int R>
 int launch_stream_ns(const GemvArgs& a, cudaStream_t stream) {
+  if (a.pipeline == kPipeReg) {
+    if constexpr (R <= 2) return launch_reg<MT, R>(a, stream);  // R = 4 would spill the register ring
+    return set_error(FI_ERR_INVALID_ARG, "GEMV register pipeline: at most 2 rows per warp");
+  }
   if (a.stages == 4) return launch_stream_one<MT, R, 4>(a, stream);
   if (a.stages == 2) return launch_stream_one<MT, R, 2>(a, stream);
   return set_error(FI_ERR_INVALID_ARG, "GEMV stream pipeline: %d slots per warp is not available", a.stages);

@@ -40,7 +40,8 @@ constexpr int kStreamIters = 2;                            // chunk iterations p
 constexpr int kStreamCellBytes = 32 * 16 + 32 * 4;         // one iteration of one row: code cells + scale words
 constexpr int kStreamHalfBudget = 228 * 1024 / 2 - 1024;   // dynamic shared memory per CTA, two CTAs per SM
 // pipelines (the high nibble of the GEMV tactic variant)
-constexpr int kPipeAuto = 0, kPipeStream = 1, kPipeRing = 2, kPipeOverlap = 3;
+constexpr int kPipeAuto = 0, kPipeStream = 1, kPipeRing = 2, kPipeOverlap = 3, kPipeReg = 4;
+constexpr int kRegDepth = 4;  // register pipeline: chunk iterations in flight per warp
 
 // Activation rows the GEMV kernel instance for m is compiled for (1, 2, 4, ..., 32).
 inline int gemv_mt(int64_t m) {
@@ -107,7 +108,7 @@ int gemv_read_error(unsigned* bits);
 constexpr int kMmaTileRows = 256;
 constexpr int kMmaKStep = 64;
 constexpr int kMmaMaxM = 256;
-constexpr int kMmaThreads = 15 * 32;
+constexpr int kMmaThreads = 24 * 32;
 inline int mma_m_pad(int64_t m) { return (int)((m + 15) / 16 * 16); }
 inline int64_t mma_rs_offset(int64_t m, int64_t k) { return round_up((int64_t)mma_m_pad(m) * k * 2, 256); }
 inline int64_t mma_workspace_bytes(int64_t m, int64_t k) { return mma_rs_offset(m, k) + (int64_t)mma_m_pad(m) * 4; }

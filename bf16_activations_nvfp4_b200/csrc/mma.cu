@@ -9,19 +9,19 @@
 //    by act_to_f16_kernel to f16 times a per-row power of two that puts the row maximum in
 //    [2^14, 2^15) (exact for every element within 2^29 of its row maximum), so the tensor core
 //    accumulates sum_k W'[i][k] * A'[j][k] in fp32 and one per-row factor undoes the scale.
-//  * Roles (one CTA per 256 weight rows, 15 warps):
+//  * Roles (one CTA per 256 weight rows, 24 warps):
 //      warp 0      TMA producer of the raw codes of the tile (256 rows x 32 bytes per 64-k step)
 //                  into a 4-stage ring, issued before the grid-dependency wait (weights never
 //                  depend on the preceding kernel);
-//      warp 10     TMA producer of the f16 activation tiles (m_pad rows x 64 k, 128-byte
+//      warp 18     TMA producer of the f16 activation tiles (m_pad rows x 64 k, 128-byte
 //                  swizzled) into the operand stages (2 to 4, as many as shared memory holds);
-//      warps 2-9   decode: one weight row per thread, codes -> f16 (cvt.rn.f16x2.e2m1x2) times
+//      warps 2-17  decode: two threads per weight row (32 k each), codes -> f16 (cvt.rn.f16x2.e2m1x2) times
 //                  the block scale (exact f16 multiply), stored in the 128-byte-swizzled
 //                  K-major layout the MMA reads; the block scales are loaded 8-11 steps ahead;
-//      warp 1      TMEM allocation and, from one thread, the MMAs: per 64-k step 4 K=16 steps x
-//                  2 M=128 halves, N = m_pad, accumulating in TMEM; tcgen05.commit frees the
-//                  stage;
-//      warps 11-14 epilogue: tcgen05.ld of the accumulator, out[j][i] = bf16_rn(D[i][j] *
+//      warps 1, 23 the MMAs, one thread each, one M = 128 half of the tile each (warp 1 also
+//                  allocates TMEM): per 64-k step 4 K=16 steps, N = m_pad, accumulating in
+//                  TMEM; tcgen05.commit frees the stage once both halves have read it;
+//      warps 19-22 epilogue: tcgen05.ld of the accumulator, out[j][i] = bf16_rn(D[i][j] *
 //                  rs[j] * gscale).
 //  * The weight tile is decoded once per call (the activations, m_pad <= 256 rows, are one MMA
 //    N tile), so the decode work is one cvt and one f16 multiply per two codes.
@@ -44,16 +44,17 @@ namespace fi {
 
 namespace {
 
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpDq0 = 2, kDqWarps = 8, kWarpAct = 10, kWarpEpi0 = 11, kEpiWarps = 4;
-static_assert((kWarpEpi0 + kEpiWarps) * 32 == kMmaThreads, "warp roles cover the CTA");
-static_assert(kWarpDq0 + kDqWarps == kWarpAct && kWarpAct + 1 == kWarpEpi0 && kDqWarps * 32 == kMmaTileRows,
-              "one decode thread per tile row");
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpDq0 = 2, kDqWarps = 16, kWarpAct = 18, kWarpEpi0 = 19, kEpiWarps = 4,
+              kWarpMma2 = 23;
+static_assert((kWarpMma2 + 1) * 32 == kMmaThreads, "warp roles cover the CTA");
+static_assert(kWarpDq0 + kDqWarps == kWarpAct && kWarpAct + 1 == kWarpEpi0 && kDqWarps * 32 == 2 * kMmaTileRows,
+              "two decode threads per tile row");
 constexpr int kRawStages = 4;
 constexpr uint32_t kRawBytes = kMmaTileRows * 32;  // 256 rows x 32 code bytes
 constexpr uint32_t kWopBytes = kMmaTileRows * 128;  // 256 rows x 64 f16, 128-byte swizzled
 // barriers: raw_full, raw_empty, then act_full, op_full, op_empty per operand stage, tmem_full,
-// drain
-constexpr int kNumBars = 2 * kRawStages + 3 * kMmaMaxOpStages + 2;
+// and one drain barrier per MMA-issuing thread
+constexpr int kNumBars = 2 * kRawStages + 3 * kMmaMaxOpStages + 3;
 
 // Shared-memory matrix descriptor of a K-major tile with 128-byte rows in the 128-byte swizzle
 // (8-row atoms of 1024 bytes): start address >> 4 in bits 0-13, leading-dimension offset 1
@@ -215,10 +216,11 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     for (int i = 0; i < NST; ++i) {
       mbar_init(&act_full[i], 1);
       mbar_init(&op_full[i], kDqWarps);
-      mbar_init(&op_empty[i], 1);
+      mbar_init(&op_empty[i], 2);  // both MMA issuers commit
     }
-    mbar_init(tmem_full, 1);
-    mbar_init(drain, 1);
+    mbar_init(tmem_full, 2);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kWarpMma) {
@@ -281,7 +283,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     }
   } else if (warp >= kWarpDq0 && warp < kWarpDq0 + kDqWarps) {
     // -------------------------------------------------------------------------- decode
-    const int r = tid - kWarpDq0 * 32;  // weight row of the tile, 0 .. 255
+    const int r = (tid - kWarpDq0 * 32) >> 1;  // weight row of the tile, 0 .. 255
+    const int hb = tid & 1;                     // this thread's half of the step: blocks 2hb, 2hb+1
     const int64_t row = w0 + r;
     const bool valid = row < n;
     const int64_t rs_s = k / 16;
@@ -325,24 +328,25 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
           mbar_wait_bounded(&raw_full[rsn], (uint32_t)((s / kRawStages) & 1), &abort_flag, p.timeout_ns, p.err, 1u) &&
           (s < NST || mbar_wait_bounded(&op_empty[os], eph, &abort_flag, p.timeout_ns, p.err, 1u));
       if (!__all_sync(0xffffffffu, ok)) break;
-      const uint4 c0 = lds_v4m(raw_addr(rsn) + (uint32_t)r * 32u);
-      const uint4 c1 = lds_v4m(raw_addr(rsn) + (uint32_t)r * 32u + 16u);
-      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      const uint4 c0 = lds_v4m(raw_addr(rsn) + (uint32_t)r * 32u + (uint32_t)hb * 16u);
+      const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
       const uint32_t dst = wop_addr(os) + wdst;
+      const uint32_t sc2 = hb ? (sc4 >> 16) : sc4;  // the scales of blocks 2hb, 2hb+1
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {  // 16-k block b: words 2b, 2b+1; chunks 2b, 2b+1 of the row
-        const uint32_t sf2 = e4m3x2_to_f16x2(__byte_perm(sc4, 0u, (uint32_t)(b | (b << 4))));
+      for (int bb = 0; bb < 2; ++bb) {  // 16-k block b = 2hb + bb: words 2bb, 2bb+1; chunks 2b, 2b+1
+        const uint32_t b = 2u * (uint32_t)hb + (uint32_t)bb;
+        const uint32_t sf2 = e4m3x2_to_f16x2(__byte_perm(sc2, 0u, (uint32_t)(bb | (bb << 4))));
         uint32_t h[8];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          const uint32_t wd = words[2 * b + q];
+          const uint32_t wd = words[2 * bb + q];
           h[4 * q + 0] = hmul2(e2m1x2_byte_to_f16x2<0>(wd), sf2);
           h[4 * q + 1] = hmul2(e2m1x2_byte_to_f16x2<1>(wd), sf2);
           h[4 * q + 2] = hmul2(e2m1x2_byte_to_f16x2<2>(wd), sf2);
           h[4 * q + 3] = hmul2(e2m1x2_byte_to_f16x2<3>(wd), sf2);
         }
-        sts_v4(dst + ((((uint32_t)(2 * b)) ^ swz) << 4), h[0], h[1], h[2], h[3]);
-        sts_v4(dst + ((((uint32_t)(2 * b + 1)) ^ swz) << 4), h[4], h[5], h[6], h[7]);
+        sts_v4(dst + (((2u * b) ^ swz) << 4), h[0], h[1], h[2], h[3]);
+        sts_v4(dst + (((2u * b + 1u) ^ swz) << 4), h[4], h[5], h[6], h[7]);
       }
       // make the generic-proxy stores visible to the tensor core (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -356,34 +360,45 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         if (s >= NST) eph ^= 1u;
       }
     }
-  } else if (warp == kWarpMma) {
+  } else if (warp == kWarpMma || warp == kWarpMma2) {
     // ----------------------------------------------------------------------------- MMA
+    // Two issuing threads, one per M = 128 half of the tile (disjoint TMEM columns, same
+    // activation operand): at small N the issue of MMA instructions by one thread, not the
+    // tensor core, set the pace. Each commits to the stage's op_empty (count 2), to tmem_full
+    // (count 2) and to its own drain barrier.
     if (lane == 0) {
+      const int h = warp == kWarpMma ? 0 : 1;
       const uint32_t idesc = f16_idesc(128, N);
+      // the descriptors differ only in the start-address field: a constant high part plus a
+      // 32-bit running start (address >> 4) per stage
+      const uint64_t desc_fixed = sw128_desc(0);
+      const uint32_t a_first = (wop_addr(0) >> 4) & 0x3FFFu, a_stride = stage_bytes >> 4;
+      constexpr uint32_t kHalf = kWopBytes / 2 / 16, kAct = kWopBytes / 16;  // in 16-byte units
+      uint32_t a_lo = a_first;
       int os = 0;
       uint32_t par = 0;  // phase of act_full[os] and op_full[os] for step s
       for (int s = 0; s < KS; ++s) {
         if (!mbar_wait_bounded(&act_full[os], par, &abort_flag, p.timeout_ns, p.err, 4u)) break;
         if (!mbar_wait_bounded(&op_full[os], par, &abort_flag, p.timeout_ns, p.err, 4u)) break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t acc0 = s != 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kMmaKStep / 16; ++kk) {
-          const uint64_t bdesc = sw128_desc(act_addr(os) + (uint32_t)kk * 32u);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint64_t adesc = sw128_desc(wop_addr(os) + (uint32_t)h * (kWopBytes / 2) + (uint32_t)kk * 32u);
-            umma_f16(tmem + (uint32_t)(h * N), adesc, bdesc, idesc, (s | kk) != 0 ? 1u : 0u);
-          }
+          const uint64_t bdesc = desc_fixed | (uint64_t)(a_lo + kAct + (uint32_t)kk * 2u);
+          const uint64_t adesc = desc_fixed | (uint64_t)(a_lo + (uint32_t)h * kHalf + (uint32_t)kk * 2u);
+          umma_f16(tmem + (uint32_t)(h * N), adesc, bdesc, idesc, kk != 0 ? 1u : acc0);
         }
         umma_commit(&op_empty[os]);  // frees the stage when these MMAs have read it
+        a_lo += a_stride;
         if (++os == NST) {
           os = 0;
           par ^= 1u;
+          a_lo = a_first;
         }
       }
       umma_commit(tmem_full);  // the accumulator is complete when every MMA issued has finished
-      umma_commit(drain);
-      drain_wait(drain, 0, p.timeout_ns, p.err);
+      umma_commit(&drain[h]);
+      drain_wait(&drain[h], 0, p.timeout_ns, p.err);
     }
     __syncwarp();
   } else {

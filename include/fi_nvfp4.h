@@ -72,7 +72,10 @@ typedef enum {
  *   variant      GEMV: low nibble = weight rows computed together by one warp (stream
  *                pipeline 1, 2 or 4; ring pipeline 1, 2, 4 or 8, at most 16 / m rounded to a
  *                power of two; 0 = automatic); high nibble = pipeline (0 = automatic =
- *                1 = per-warp asynchronous copies, 2 = producer-warp ring). MMA: 0.
+ *                1 = per-warp asynchronous copies, 2 = producer-warp ring, 3 = per-warp
+ *                copies in one half-SM CTA per SM, so that consecutive calls overlap, with
+ *                an L2 prefetch of weights up to 40 MB; its CTAs-per-SM field is ignored;
+ *                4 = weights loaded straight to registers, 1 or 2 rows per warp). MMA: 0.
  * Only `kind` and the resolved S change the arithmetic: two tactics with the same kind
  * and S give bitwise identical outputs (whatever their pipeline, rows or CTAs), and for a
  * fixed tactic every output row is bitwise independent of m. GEMV and MMA results differ

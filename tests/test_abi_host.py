@@ -50,9 +50,12 @@ def test_default_gemv_tactic_resolves_for_decode_shapes(n, k):
     # one persistent wave: the grid never asks for more CTAs than the SMs hold
     assert info["grid_x"] * info["grid_y"] <= B200_SMS * info["ctas_per_sm"]
     # the default runs the per-warp async-copy pipeline: one CTA of up to 16 warps per SM, or
-    # two of up to 8 warps within half an SM each; fewer warps only where the row groups would
-    # otherwise leave SMs idle, and then the grid spans every SM of the split's share
-    assert info["variant"] >> 4 == 1
+    # two of up to 8 warps within half an SM each; weights of at most 12 MB take the overlapped
+    # variant (one half-SM CTA per SM). Fewer warps only where the row groups would otherwise
+    # leave SMs idle, and then the grid spans every SM of the split's share
+    pipe = info["variant"] >> 4
+    small = n * (k // 2 + k // 16) <= 12 << 20
+    assert pipe == (3 if small else (4 if k % 256 else 1))
     warps = info["threads"] // 32
     if info["ctas_per_sm"] == 1:
         assert 4 <= warps <= 16 and 0 < info["smem_bytes"] <= 227 * 1024 - 1024
@@ -60,7 +63,7 @@ def test_default_gemv_tactic_resolves_for_decode_shapes(n, k):
         assert 4 <= warps <= 8 and 0 < info["smem_bytes"] <= 228 * 1024 // 2 - 1024
     full = 16 if info["ctas_per_sm"] == 1 else 8
     if warps < full:
-        share = B200_SMS * info["ctas_per_sm"] // info["splits"]
+        share = B200_SMS * (1 if pipe == 3 else info["ctas_per_sm"]) // info["splits"]
         assert info["grid_x"] >= share - 1 or warps == 4, info
     assert info["workspace_bytes"] == (info["splits"] * n * 4 if info["splits"] > 1 else 0)
 
@@ -125,7 +128,7 @@ def test_workspace_bytes():
     (32, 64, 14336, fi.make_tactic(0, 1, 0, 1), -2),      # A slice does not fit shared memory
     (32, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),       # one row per stage above m = 8
     (5, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),        # two rows per stage above m = 4
-    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x42), -1),     # pipeline 4
+    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x52), -1),     # pipeline 5
     (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x19), -1),     # rows 9 on the stream pipeline
     (1, 8, 65536, fi.make_tactic(0, 1, 0, 0x22), -2),     # ring: two 36 KB rows per stage do not fit twice
     (1, 8, 65536, fi.make_tactic(0, 1, 2, 0x11), -2),     # stream, half-SM CTAs: 128 KB of activations
@@ -192,7 +195,7 @@ def test_mma_tactic_resolution():
     t = fi.make_tactic(fi.KIND_MMA, 1, 0, 0)
     info = fi.resolve_tactic(256, 152064, 5120, t, B200_SMS)
     assert info["kind"] == fi.KIND_MMA and info["splits"] == 1
-    assert info["grid_x"] == 152064 // 256 and info["threads"] == 15 * 32
+    assert info["grid_x"] == 152064 // 256 and info["threads"] == 24 * 32
     assert 0 < info["smem_bytes"] <= 227 * 1024
     # workspace: f16 activations [256, k] then 256 fp32 row scales
     assert info["workspace_bytes"] == 256 * 5120 * 2 + 256 * 4

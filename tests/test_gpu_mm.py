@@ -53,8 +53,8 @@ def test_tiny_workload_every_tactic():
     (2, 1, 32, 5),          # single chunk, single row
     (16, 300, 2048, 6),
     (32, 96, 1024, 7),
-    (1, 1001, 1536, 8),     # tensor-copy items: 48 chunks (a half-filled last iteration), odd n
-    (4, 515, 5120, 9),      # tensor-copy items: 160 chunks (an empty last iteration), partial group
+    (1, 1001, 1536, 8),     # 48 chunks: a half-filled last iteration, odd n
+    (4, 515, 5120, 9),      # 160 chunks: an item whose second iteration is empty, partial group
 ])
 def test_parity_spanning_tiles(m, n, k, seed):
     A = inputs.activations(m, k, seed, outliers=True)
@@ -150,8 +150,9 @@ def test_rows_per_stage_and_occupancy_do_not_change_bits():
 
 
 def test_pipelines_give_identical_bits():
-    """The per-warp async-copy pipeline and the producer-warp ring run the same per-chunk
-    arithmetic in the same order, so for one S their outputs are bitwise equal."""
+    """The per-warp async-copy pipeline, the producer-warp ring, the overlapped variant and the
+    register pipeline run the same per-chunk arithmetic in the same order, so for one S their
+    outputs are bitwise equal."""
     for m, n, k in [(1, 2048, 7168), (3, 1000, 4096), (8, 515, 2688), (32, 300, 2048)]:
         A = inputs.activations(m, k, seed=21, outliers=True)
         dw = _gpu.device_weights(n, k, 2)
@@ -161,8 +162,13 @@ def test_pipelines_give_identical_bits():
             except fi.FiError as e:  # activations of this split do not fit half an SM
                 assert e.status == -2
                 continue
-            ring = _mm(A, dw, fi.make_tactic(GEMV, S, 0, 0x20))
-            assert np.array_equal(stream, ring), (m, n, k, S)
+            for var in (0x20, 0x30, 0x40, 0x41):
+                try:
+                    other = _mm(A, dw, fi.make_tactic(GEMV, S, 0, var))
+                except fi.FiError as e:  # the overlapped variant's half SM cannot hold these activations
+                    assert e.status == -2 and var == 0x30, (m, n, k, S, hex(var))
+                    continue
+                assert np.array_equal(stream, other), (m, n, k, S, hex(var))
 
 
 def test_multi_slab_rows_and_many_splits():
