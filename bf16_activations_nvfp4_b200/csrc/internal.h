@@ -114,7 +114,12 @@ inline int64_t mma_rs_offset(int64_t m, int64_t k) { return round_up((int64_t)mm
 inline int64_t mma_workspace_bytes(int64_t m, int64_t k) { return mma_rs_offset(m, k) + (int64_t)mma_m_pad(m) * 4; }
 // operand stages (decoded weights + activation tile of one 64-k step): as many as fit, 2..4
 constexpr int kMmaMaxOpStages = 4;
-inline int64_t mma_stage_bytes(int m_pad) { return (int64_t)kMmaTileRows * 128 + round_up((int64_t)m_pad * 128, 1024); }
+// m_pad <= kMmaTmemMaxM: the decoded weights live in tensor memory, a stage is the activation
+// tile only; above, a stage also holds the decoded weight tile in shared memory
+constexpr int kMmaTmemMaxM = 128;
+inline int64_t mma_stage_bytes(int m_pad) {
+  return (m_pad <= kMmaTmemMaxM ? 0 : (int64_t)kMmaTileRows * 128) + round_up((int64_t)m_pad * 128, 1024);
+}
 int mma_op_stages(int m_pad);
 int64_t mma_smem_bytes(int m_pad);
 

@@ -32,6 +32,7 @@
 // of m, so for a fixed tactic a row's bits do not depend on m (an output element depends only
 // on its weight row and activation row); results are deterministic run to run.
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 
 #include <cuda.h>
@@ -84,6 +85,27 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(
           d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// tcgen05.mma with the A operand (the weights) in tensor memory at a_tmem.
+__device__ __forceinline__ void umma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane (32x32b shape: the warp's 32 lanes
+// from the lane in taddr, which must be the warp's own quarter).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 
@@ -175,6 +197,10 @@ __global__ void __launch_bounds__(256) act_to_f16_kernel(const uint16_t* __restr
   if (tid == 0) rs[row] = __uint_as_float((uint32_t)(127 - sh) << 23);
 }
 
+// TA: the decoded weights go to tensor memory (tcgen05.st) and the MMAs read A from there
+// (m_pad <= 128: the accumulator takes 2 m_pad <= 256 columns, the A stages columns 256-511);
+// otherwise they go to shared memory in the 128-byte swizzle.
+template <bool TA>
 __global__ void __launch_bounds__(kMmaThreads, 1)
     mma_nvfp4_kernel(const MmaArgs p, const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_w) {
@@ -198,14 +224,16 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   uint64_t* const drain = tmem_full + 1;
   auto raw_addr = [&](int st) { return base + (uint32_t)st * kRawBytes; };
   auto wop_addr = [&](int st) { return base + kRawStages * kRawBytes + (uint32_t)st * stage_bytes; };
-  auto act_addr = [&](int st) { return wop_addr(st) + kWopBytes; };
+  auto act_addr = [&](int st) { return wop_addr(st) + (TA ? 0u : kWopBytes); };
+  // TA: columns of the A operand of stage st, half h (32 columns: 64 k as f16 pairs)
+  auto a_col = [&](int st, int h) { return 256u + (uint32_t)st * 64u + (uint32_t)h * 32u; };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n = p.n, k = p.k;
   const int m = (int)p.m, N = p.m_pad;
   const int KS = (int)(k / kMmaKStep);
   const int64_t w0 = (int64_t)blockIdx.x * kMmaTileRows;
-  const uint32_t ncols = N <= 16 ? 32u : (N <= 64 ? 128u : (N <= 128 ? 256u : 512u));  // >= 2N, a power of two
+  const uint32_t ncols = TA ? 512u : (N <= 16 ? 32u : (N <= 64 ? 128u : (N <= 128 ? 256u : 512u)));  // >= 2N
 
   if (tid == 0) {
     abort_flag = 0;
@@ -283,8 +311,14 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     }
   } else if (warp >= kWarpDq0 && warp < kWarpDq0 + kDqWarps) {
     // -------------------------------------------------------------------------- decode
-    const int r = (tid - kWarpDq0 * 32) >> 1;  // weight row of the tile, 0 .. 255
-    const int hb = tid & 1;                     // this thread's half of the step: blocks 2hb, 2hb+1
+    // shared-memory operand: two threads per row (adjacent lanes), blocks 2hb, 2hb+1 each.
+    // TA: a warp may only reach its own quarter of the TMEM lanes, so warp w takes rows
+    // h*128 + 32(w % 4) + lane of half h and k half hb, (h, hb) from the warp's index among
+    // the four decode warps of its quarter.
+    const int dq = (warp - kWarpDq0) >> 2;
+    const int tq = warp & 3;
+    const int r = TA ? (dq & 1) * 128 + tq * 32 + lane : (tid - kWarpDq0 * 32) >> 1;  // tile row, 0 .. 255
+    const int hb = TA ? dq >> 1 : tid & 1;  // this thread's half of the step: blocks 2hb, 2hb+1
     const int64_t row = w0 + r;
     const bool valid = row < n;
     const int64_t rs_s = k / 16;
@@ -330,26 +364,34 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       const uint4 c0 = lds_v4m(raw_addr(rsn) + (uint32_t)r * 32u + (uint32_t)hb * 16u);
       const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
-      const uint32_t dst = wop_addr(os) + wdst;
       const uint32_t sc2 = hb ? (sc4 >> 16) : sc4;  // the scales of blocks 2hb, 2hb+1
+      uint32_t hv[16];  // the 32 k of this thread as f16 pairs, in k order
 #pragma unroll
-      for (int bb = 0; bb < 2; ++bb) {  // 16-k block b = 2hb + bb: words 2bb, 2bb+1; chunks 2b, 2b+1
-        const uint32_t b = 2u * (uint32_t)hb + (uint32_t)bb;
+      for (int bb = 0; bb < 2; ++bb) {  // 16-k block b = 2hb + bb: words 2bb, 2bb+1
         const uint32_t sf2 = e4m3x2_to_f16x2(__byte_perm(sc2, 0u, (uint32_t)(bb | (bb << 4))));
-        uint32_t h[8];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const uint32_t wd = words[2 * bb + q];
-          h[4 * q + 0] = hmul2(e2m1x2_byte_to_f16x2<0>(wd), sf2);
-          h[4 * q + 1] = hmul2(e2m1x2_byte_to_f16x2<1>(wd), sf2);
-          h[4 * q + 2] = hmul2(e2m1x2_byte_to_f16x2<2>(wd), sf2);
-          h[4 * q + 3] = hmul2(e2m1x2_byte_to_f16x2<3>(wd), sf2);
+          hv[8 * bb + 4 * q + 0] = hmul2(e2m1x2_byte_to_f16x2<0>(wd), sf2);
+          hv[8 * bb + 4 * q + 1] = hmul2(e2m1x2_byte_to_f16x2<1>(wd), sf2);
+          hv[8 * bb + 4 * q + 2] = hmul2(e2m1x2_byte_to_f16x2<2>(wd), sf2);
+          hv[8 * bb + 4 * q + 3] = hmul2(e2m1x2_byte_to_f16x2<3>(wd), sf2);
         }
-        sts_v4(dst + (((2u * b) ^ swz) << 4), h[0], h[1], h[2], h[3]);
-        sts_v4(dst + (((2u * b + 1u) ^ swz) << 4), h[4], h[5], h[6], h[7]);
       }
-      // make the generic-proxy stores visible to the tensor core (async proxy)
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      if constexpr (TA) {
+        // lane r & 127 of half r >> 7: columns a_col + 16 hb .. + 15 hold k 32 hb .. 32 hb + 31
+        tmem_st16(tmem + ((uint32_t)(tq * 32) << 16) + a_col(os, r >> 7) + (uint32_t)hb * 16u, hv);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      } else {
+        const uint32_t dst = wop_addr(os) + wdst;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)  // chunk 4hb + c of the row (8 k each), 128-byte swizzle
+          sts_v4(dst + (((4u * (uint32_t)hb + (uint32_t)c) ^ swz) << 4), hv[4 * c], hv[4 * c + 1], hv[4 * c + 2],
+                 hv[4 * c + 3]);
+        // make the generic-proxy stores visible to the tensor core (async proxy)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&op_full[os]);
@@ -384,9 +426,15 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         const uint32_t acc0 = s != 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kMmaKStep / 16; ++kk) {
-          const uint64_t bdesc = desc_fixed | (uint64_t)(a_lo + kAct + (uint32_t)kk * 2u);
-          const uint64_t adesc = desc_fixed | (uint64_t)(a_lo + (uint32_t)h * kHalf + (uint32_t)kk * 2u);
-          umma_f16(tmem + (uint32_t)(h * N), adesc, bdesc, idesc, kk != 0 ? 1u : acc0);
+          if constexpr (TA) {
+            const uint64_t bdesc = desc_fixed | (uint64_t)(a_lo + (uint32_t)kk * 2u);
+            umma_f16_ta(tmem + (uint32_t)(h * N), tmem + a_col(os, h) + (uint32_t)kk * 8u, bdesc, idesc,
+                        kk != 0 ? 1u : acc0);
+          } else {
+            const uint64_t bdesc = desc_fixed | (uint64_t)(a_lo + kAct + (uint32_t)kk * 2u);
+            const uint64_t adesc = desc_fixed | (uint64_t)(a_lo + (uint32_t)h * kHalf + (uint32_t)kk * 2u);
+            umma_f16(tmem + (uint32_t)(h * N), adesc, bdesc, idesc, kk != 0 ? 1u : acc0);
+          }
         }
         umma_commit(&op_empty[os]);  // frees the stage when these MMAs have read it
         a_lo += a_stride;
@@ -454,6 +502,7 @@ int encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint
 int mma_op_stages(int m_pad) {
   const int64_t per = mma_stage_bytes(m_pad);
   const int64_t room = kSmemBudget - 1024 - (int64_t)kRawStages * kRawBytes - kNumBars * 8;
+  // with the weights in tensor memory, its columns 256-511 hold at most 4 stages of A
   return (int)std::max<int64_t>(2, std::min<int64_t>(kMmaMaxOpStages, room / per));
 }
 
@@ -479,14 +528,15 @@ int launch_mma(const MmaArgs& a, cudaStream_t stream) {
                  (uint64_t)(a.k / 2), 32, kMmaTileRows, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc != FI_OK) return rc;
 
+  const bool ta = a.m_pad <= kMmaTmemMaxM;
+  auto kern = ta ? mma_nvfp4_kernel<true> : mma_nvfp4_kernel<false>;
   static int configured[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return set_cuda_error("cudaGetDevice");
-  if (!configured[dev]) {
-    if (cudaFuncSetAttribute(mma_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) !=
-        cudaSuccess)
+  if (!(configured[dev] & (ta ? 2 : 1))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) != cudaSuccess)
       return set_cuda_error("cudaFuncSetAttribute(mma smem)");
-    configured[dev] = 1;
+    configured[dev] |= ta ? 2 : 1;
   }
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -504,11 +554,13 @@ int launch_mma(const MmaArgs& a, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((a.n + kMmaTileRows - 1) / kMmaTileRows));
   cfg.blockDim = dim3(kMmaThreads);
-  cfg.dynamicSmemBytes = (size_t)mma_smem_bytes(a.m_pad);
+  // at most one CTA per SM: with the weights in tensor memory a CTA takes all 512 columns, and
+  // a second CTA on the SM would wait in its allocation
+  cfg.dynamicSmemBytes = (size_t)std::max<int64_t>(mma_smem_bytes(a.m_pad), kSmemBudget / 2 + 4096);
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, mma_nvfp4_kernel, a, tmap_a, tmap_w) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kern, a, tmap_a, tmap_w) != cudaSuccess)
     return set_cuda_error("mma_nvfp4_kernel launch");
   return FI_OK;
 }
