@@ -310,6 +310,7 @@ def run_fi(args, rank: int, world: int) -> dict | None:
     if world > 1:
         dist.barrier()
     lm_head = run_lm_head(dev, stream, peaks) if world == 1 and not args.no_lm_head else None
+    extra = run_extra_shapes(dev, stream, peaks) if world == 1 and not args.no_lm_head else None
 
     # ---- end to end through the public op with host buffers (eager calls)
     e2e_steps = max(5, args.steps // 10)
@@ -399,7 +400,58 @@ def run_fi(args, rank: int, world: int) -> dict | None:
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall1 - wall0, 3),
         "lm_head": lm_head,
+        "decode_grid": extra,
     }
+
+
+def run_extra_shapes(dev, stream, peaks) -> dict:
+    """Default-tactic µs per call, cold L2 (each call reads its own weight copy, copies >= 300
+    MB per shape), PDL-chained graph replays: the narrow-n decode grid at m = 1 and the
+    small-batch sweep of 4096 x 14336 at m in {1, 2, 4, 8, 16, 32}."""
+    import torch
+
+    import bf16_activations_nvfp4_b200 as fi
+    from bf16_activations_nvfp4_b200 import inputs
+
+    def time_case(m, n, k):
+        W = torch.from_numpy(inputs.weights(n, k, seed=0)).to(dev)
+        Wq, Ws, g = fi.pack_weights(W)
+        del W
+        b = algorithmic_bytes(m, n, k)
+        wbytes = n * (k // 2 + k // 16)
+        copies = [(Wq, Ws)] + [(Wq.clone(), Ws.clone()) for _ in range(-(-COLD_BYTES // wbytes) - 1)]
+        A = torch.from_numpy(inputs.activations(m, k, seed=0, outliers=True).view(np.int16)).view(torch.bfloat16).to(dev)
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        t = fi.default_tactic(m, n, k)
+        ws = torch.empty(max(fi.workspace_bytes(m, n, k, t), 256) // 4 + 64, dtype=torch.float32, device=dev)
+        nrep = 2 * len(copies)
+        with torch.cuda.stream(stream):
+            fi.mm_bf16_fp4(A, Wq, Ws, g, tactic=t, out=out, workspace=ws)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                for r in range(nrep):
+                    q, s_ = copies[r % len(copies)]
+                    fi.mm_bf16_fp4(A, q, s_, g, tactic=t, out=out, workspace=ws)
+            ts = []
+            for _ in range(8):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3 / nrep)
+        us = statistics.median(ts[2:])
+        info = fi.resolve_tactic(m, n, k, t)
+        del graph, copies
+        return {"m": m, "n": n, "k": k, "us": round(us, 3), "gbs": round(b / (us * 1e-6) / 1e9, 1),
+                "frac_hbm": round(b / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                "tflops": round(2 * m * n * k / us / 1e6, 3), "splits": info["splits"],
+                "pipeline": info["variant"] >> 4 if info["kind"] == fi.KIND_GEMV else "mma"}
+
+    narrow = [time_case(1, n, k) for n, k in inputs.NARROW_N]
+    small = [time_case(m, *inputs.SMALL_BATCH_NK) for m in inputs.SMALL_BATCH_M]
+    return {"narrow_n": narrow, "small_batch": small,
+            "method": "default tactic, PDL-chained CUDA-graph replays over >= 300 MB of weight copies (cold L2)"}
 
 
 def mma_wave(args) -> None:

@@ -85,8 +85,11 @@ static int check_arch() {
 
 // ----------------------------------------------------------------- tactics
 
-// Largest m the default table sends to the GEMV.
-constexpr int64_t kDefaultGemvMaxM = 32;
+// Largest m the default table sends to the GEMV. Measured on B200 (cold L2, PDL-chained
+// graphs): the split-K MMA path is faster from m = 8 on every serving shape (4096 x 14336 at
+// m = 8: 25.6 against 47.5 us; at m = 32: 29.6 against 176 us) and level at m = 4; the GEMV
+// keeps m = 1..4.
+constexpr int64_t kDefaultGemvMaxM = 4;
 
 int gemv_geometry(int64_t m, int64_t n, int64_t k, int S, int rs_req, int ctas_per_sm, int sms, GemvGeometry* g) {
   const int64_t C = k / kChunkK;
@@ -269,11 +272,11 @@ static int gemv_knee(int pipe, int64_t n, int64_t k, int sms, int64_t m_fit, int
 
 static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms, fi_tactic_info* out);
 
-// The built-in table. m = 1, 2..8 and 9..32 are separate buckets: the tactic (and so the bits
+// The built-in table. m = 1, 2..4 and 5..256 are separate buckets: the tactic (and so the bits
 // of a row) is the same for every m inside a bucket.
 static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms) {
   if (m <= kDefaultGemvMaxM) {
-    const int64_t m_fit = m <= 1 ? 1 : (m <= 8 ? 8 : kGemvMaxM);
+    const int64_t m_fit = m <= 1 ? 1 : kDefaultGemvMaxM;
     // stream pipeline with its automatic CTA shape and rows per item (see gemv_stream_geometry);
     // weights of at most 12 MB take the overlapped variant (half-SM CTAs, one per SM, weights
     // prefetched into L2 while the preceding call computes). Measured on B200 at m = 1 in
@@ -289,7 +292,7 @@ static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms)
     if (gemv_knee(pipe, n, k, num_sms, m_fit, 0, ctas, &S) != FI_OK) S = 1;
     return FI_TACTIC(FI_KIND_GEMV, S, ctas, pipe << 4);
   }
-  return FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
+  return FI_TACTIC(FI_KIND_MMA, 0, 0, 0);  // device-sized K split
 }
 
 // GEMV variant byte: low nibble = weight rows computed together by one warp (ring pipeline:
@@ -350,23 +353,47 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
 
 // MMA tactic: splits 0 or 1 (one split), CTAs per SM 0 or 1, variant 0. Needs m <= 256 and k a
 // multiple of 64; the workspace holds the f16 activations and their row scales.
-static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var, fi_tactic_info* out) {
+static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var, int sms,
+                       fi_tactic_info* out) {
   if (m > kMmaMaxM)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA tactics support m <= %d (got m=%lld)", kMmaMaxM, (long long)m);
   if (k % kMmaKStep != 0)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA tactics need k to be a multiple of %d (got k=%lld)", kMmaKStep,
                      (long long)k);
-  if (S_req > 1 || ctas_req > 1 || var != 0)
-    return set_error(FI_ERR_INVALID_ARG, "MMA tactics take splits 0/1, CTAs per SM 0/1 and variant 0");
+  if (ctas_req > 1 || var != 0)
+    return set_error(FI_ERR_INVALID_ARG, "MMA tactics take CTAs per SM 0/1 and variant 0");
+  const int64_t tiles = std::max<int64_t>(1, (n + kMmaTileRows - 1) / kMmaTileRows);
+  const int64_t KS = k / kMmaKStep;
+  int64_t S = S_req;
+  if (S > 1 && S > KS)
+    return set_error(FI_ERR_INVALID_ARG, "splits=%lld exceeds k/%d=%lld", (long long)S, kMmaKStep, (long long)KS);
+  if (S == 0) {
+    // device-sized split: one CTA per SM, so a launch of tiles * S CTAs takes ceil(tiles * S /
+    // sms) waves of ceil(KS / S) steps plus about 4 steps of per-CTA start and epilogue. A
+    // split adds 3 steps for the reduce launch and the partials' write and read (2 S m n 4
+    // bytes at about 4 MB per step, a step being about 0.6 us measured on B200). Take the S
+    // (1..16) of least cost.
+    S = 1;
+    double best = -1.0;
+    for (int64_t c = 1; c <= std::min<int64_t>(16, std::max<int64_t>(1, KS)); ++c) {
+      const double cost = (double)((tiles * c + sms - 1) / sms) * (double)((KS + c - 1) / c + 4) +
+                          (c > 1 ? 3.0 + 2.0 * (double)c * (double)m * (double)n * 4.0 / 4.0e6 : 0.0);
+      if (best < 0 || cost < best) {
+        best = cost;
+        S = c;
+      }
+    }
+  }
+  if (S < 1) S = 1;
   out->kind = FI_KIND_MMA;
-  out->splits = 1;
+  out->splits = (int32_t)S;
   out->ctas_per_sm = 1;
   out->variant = 0;
-  out->grid_x = (int32_t)std::max<int64_t>(1, (n + kMmaTileRows - 1) / kMmaTileRows);
-  out->grid_y = 1;
+  out->grid_x = (int32_t)tiles;
+  out->grid_y = (int32_t)S;
   out->threads = kMmaThreads;
   out->smem_bytes = (int32_t)mma_smem_bytes(mma_m_pad(m));
-  out->workspace_bytes = (m > 0 && k > 0) ? mma_workspace_bytes(m, k) : 0;
+  out->workspace_bytes = (m > 0 && k > 0) ? (S > 1 ? mma_partials_offset(m, k) + S * m * n * 4 : mma_workspace_bytes(m, k)) : 0;
   return FI_OK;
 }
 
@@ -383,7 +410,7 @@ static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms,
   const int var = FI_TACTIC_VARIANT(tactic);
   memset(out, 0, sizeof(*out));
   if (kind == FI_KIND_GEMV) return resolve_gemv(m, n, k, S, ctas, var, num_sms, out);
-  if (kind == FI_KIND_MMA) return resolve_mma(m, n, k, S, ctas, var, out);
+  if (kind == FI_KIND_MMA) return resolve_mma(m, n, k, S, ctas, var, num_sms, out);
   return set_error(FI_ERR_INVALID_ARG, "unknown tactic kind %d", kind);
 }
 
@@ -546,6 +573,8 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.n = n;
     a.k = k;
     a.m_pad = mma_m_pad(m);
+    a.splits = info.splits;
+    a.partials = reinterpret_cast<float*>(ws + mma_partials_offset(m, k));
     a.op_stages = mma_op_stages(a.m_pad);
     a.stage_bytes = (uint32_t)mma_stage_bytes(a.m_pad);
     a.debug_stall = g_debug_stall_launches > 0 ? 1 : 0;
@@ -555,6 +584,7 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.timeout_ns = g_wait_timeout_ns;
     rc = launch_mma(a, stream);
     if (rc != FI_OK) return rc;
+    if (info.splits > 1) return launch_splitk_reduce(a.partials, info.splits, m, n, gscale, out, true, stream);
     return FI_OK;
   }
   if (info.splits > 1) return launch_splitk_reduce(partials, info.splits, m, n, gscale, out, true, stream);

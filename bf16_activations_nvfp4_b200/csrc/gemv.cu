@@ -928,6 +928,7 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_reg_kernel(GemvArgs
 
   const int64_t rs_q = k / 2, rs_s = k / 16;
   pdl_launch_dependents();
+  if (p.prefetch_l2 && lane == 0 && r_lo < r_hi) prefetch_rows_l2(p, r_lo, r_hi, c0, nch);
 
   // ---- load cursor: iteration (group lg, chunk iteration lt); row i's code and scale pointers
   // for this lane's chunk

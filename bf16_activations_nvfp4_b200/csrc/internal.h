@@ -112,6 +112,8 @@ constexpr int kMmaThreads = 24 * 32;
 inline int mma_m_pad(int64_t m) { return (int)((m + 15) / 16 * 16); }
 inline int64_t mma_rs_offset(int64_t m, int64_t k) { return round_up((int64_t)mma_m_pad(m) * k * 2, 256); }
 inline int64_t mma_workspace_bytes(int64_t m, int64_t k) { return mma_rs_offset(m, k) + (int64_t)mma_m_pad(m) * 4; }
+// split-K partials [splits, m, n] fp32 follow the activations at the next 256-byte boundary
+inline int64_t mma_partials_offset(int64_t m, int64_t k) { return round_up(mma_workspace_bytes(m, k), 256); }
 // operand stages (decoded weights + activation tile of one 64-k step): as many as fit, 2..4
 constexpr int kMmaMaxOpStages = 4;
 // m_pad <= kMmaTmemMaxM: the decoded weights live in tensor memory, a stage is the activation
@@ -133,6 +135,8 @@ struct MmaArgs {
   float* rs;      // workspace: per-row inverse scales [m_pad]
   int64_t m, n, k;
   int m_pad;
+  int splits;           // K splits (grid.y); > 1 writes fp32 partials [splits, m, n] to `partials`
+  float* partials;
   int op_stages;        // operand stages in shared memory (mma_op_stages)
   uint32_t stage_bytes; // bytes of one operand stage (mma_stage_bytes)
   int debug_stall;      // test hook: the producer issues nothing (the waits time out)

@@ -231,7 +231,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n = p.n, k = p.k;
   const int m = (int)p.m, N = p.m_pad;
-  const int KS = (int)(k / kMmaKStep);
+  // split blockIdx.y of gridDim.y takes the 64-k steps [ks0, ks0 + KS) in order
+  const int KS_all = (int)(k / kMmaKStep), S = (int)gridDim.y, sp = (int)blockIdx.y;
+  const int ks0 = (int)((int64_t)sp * KS_all / S);
+  const int KS = (int)((int64_t)(sp + 1) * KS_all / S) - ks0;
   const int64_t w0 = (int64_t)blockIdx.x * kMmaTileRows;
   const uint32_t ncols = TA ? 512u : (N <= 16 ? 32u : (N <= 64 ? 128u : (N <= 128 ? 256u : 512u)));  // >= 2N
 
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       const int pro = KS < kRawStages ? KS : kRawStages;
       for (int s = 0; s < pro; ++s) {
         mbar_arrive_expect_tx(&raw_full[s], kRawBytes);
-        tma_load_2d(raw_addr(s), &tmap_w, s * 32, (int)w0, smem_addr(&raw_full[s]));
+        tma_load_2d(raw_addr(s), &tmap_w, (ks0 + s) * 32, (int)w0, smem_addr(&raw_full[s]));
         ++issued;
       }
       for (int s = 0; s + kRawStages < KS && !abort_flag; ++s) {
@@ -282,7 +285,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                                2u))
           break;
         mbar_arrive_expect_tx(&raw_full[rs], kRawBytes);
-        tma_load_2d(raw_addr(rs), &tmap_w, (s + kRawStages) * 32, (int)w0, smem_addr(&raw_full[rs]));
+        tma_load_2d(raw_addr(rs), &tmap_w, (ks0 + s + kRawStages) * 32, (int)w0, smem_addr(&raw_full[rs]));
         ++issued;
       }
       // drain: every copy issued must have landed before the CTA exits
@@ -299,7 +302,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       for (int s = 0; s < KS && !abort_flag; ++s) {
         if (s >= NST && !mbar_wait_bounded(&op_empty[os], ph, &abort_flag, p.timeout_ns, p.err, 2u)) break;
         mbar_arrive_expect_tx(&act_full[os], (uint32_t)N * 128u);
-        tma_load_2d(act_addr(os), &tmap_a, s * kMmaKStep, 0, smem_addr(&act_full[os]));
+        tma_load_2d(act_addr(os), &tmap_a, (ks0 + s) * kMmaKStep, 0, smem_addr(&act_full[os]));
         ++issued;
         if (++os == NST) {
           os = 0;
@@ -322,13 +325,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     const int64_t row = w0 + r;
     const bool valid = row < n;
     const int64_t rs_s = k / 16;
-    const uint8_t* srow = p.Ws + (valid ? row : 0) * rs_s;
+    const uint8_t* srow = p.Ws + (valid ? row : 0) * rs_s + (int64_t)ks0 * 4;  // the split's first step
     const uint32_t wdst = (uint32_t)(r >> 7) * (kWopBytes / 2) + (uint32_t)(r & 127) * 128u;
     const uint32_t swz = (uint32_t)(r & 7);
     // The row's four E4M3 scales of step s are the 4 bytes at srow + 4s. They are loaded in
     // groups of 4 steps, three groups ahead of their use, so the global-memory latency of the
     // scales (cold: they are read once per call) is off the per-step path.
-    const bool al16 = rs_s % 16 == 0;
+    const bool al16 = rs_s % 16 == 0 && ks0 % 4 == 0;
     auto load_group = [&](int gi) -> uint4 {
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       const int s0 = gi * 4;
@@ -460,16 +463,27 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (ok) {
       const float g = *p.gscale;
+      // S > 1: this split's fp32 partials D * rs[j] (exact: rs is a power of two), summed in
+      // split order by the reduce kernel; S == 1: bf16_rn(D * rs[j] * gscale)
+      float* const part = S > 1 ? p.partials + (int64_t)sp * m * n : nullptr;
       for (int h = 0; h < 2; ++h) {
         const int64_t row = w0 + h * 128 + i;
         for (int j0 = 0; j0 < N; j0 += 16) {
           float v[16];
           tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * N + j0), v);
           if (row < n) {
+            if (part == nullptr) {
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-              const int j = j0 + jj;
-              if (j < m) p.out[(int64_t)j * n + row] = f32_to_bf16_rn(__fmul_rn(__fmul_rn(v[jj], p.rs[j]), g));
+              for (int jj = 0; jj < 16; ++jj) {
+                const int j = j0 + jj;
+                if (j < m) p.out[(int64_t)j * n + row] = f32_to_bf16_rn(__fmul_rn(__fmul_rn(v[jj], p.rs[j]), g));
+              }
+            } else {
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) {
+                const int j = j0 + jj;
+                if (j < m) part[(int64_t)j * n + row] = __fmul_rn(v[jj], p.rs[j]);
+              }
             }
           }
         }
@@ -515,6 +529,8 @@ int launch_mma(const MmaArgs& a, cudaStream_t stream) {
   if (a.k % kMmaKStep != 0 || a.m_pad < 16 || a.m_pad > kMmaMaxM || a.m_pad % 16 != 0)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA path: k must be a multiple of %d and m <= %d", kMmaKStep,
                      kMmaMaxM);
+  if (a.splits < 1 || a.splits > a.k / kMmaKStep || (a.splits > 1 && !a.partials))
+    return set_error(FI_ERR_INVALID_ARG, "MMA path: %d splits for k=%lld", a.splits, (long long)a.k);
   if (a.op_stages < 2 || a.op_stages > kMmaMaxOpStages || (int64_t)a.stage_bytes != mma_stage_bytes(a.m_pad))
     return set_error(FI_ERR_INVALID_ARG, "MMA path: %d operand stages of %u bytes do not match m_pad=%d", a.op_stages,
                      a.stage_bytes, a.m_pad);
@@ -552,7 +568,7 @@ int launch_mma(const MmaArgs& a, cudaStream_t stream) {
     return set_cuda_error("act_to_f16_kernel launch");
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((a.n + kMmaTileRows - 1) / kMmaTileRows));
+  cfg.gridDim = dim3((unsigned)((a.n + kMmaTileRows - 1) / kMmaTileRows), (unsigned)a.splits);
   cfg.blockDim = dim3(kMmaThreads);
   // at most one CTA per SM: with the weights in tensor memory a CTA takes all 512 columns, and
   // a second CTA on the SM would wait in its allocation

@@ -60,11 +60,12 @@ typedef enum {
 /* ------------------------------------------------------------------------- tactics
  * A tactic is a 32-bit code built by FI_TACTIC(kind, splits, ctas_per_sm, variant):
  *   kind         FI_KIND_GEMV (streaming GEMV, 1 <= m <= 32) or FI_KIND_MMA (tcgen05
- *                tensor-core GEMM, 1 <= m <= 256, k a multiple of 64, one split);
+ *                tensor-core GEMM, 1 <= m <= 256, k a multiple of 64);
  *   splits       number of K partitions S (1..4095); 0 = device-sized ("knee") split:
  *                the smallest S that gives the device enough concurrent weight streams
  *                (PR #4038, Description, "What it does": the device-sized GEMV split).
- *                MMA: 0 or 1;
+ *                MMA: 1..k/64 splits of whole 64-k steps; 0 = the split with the fewest
+ *                waves of steps for one CTA per SM (partials and the reduce counted);
  *   ctas_per_sm  CTAs per SM the grid is sized for (PR #4038, Description, "What it
  *                does": occupancy tactics); 0 = automatic. GEMV stream pipeline: 1 = one
  *                16-warp CTA per SM, 2 = two 8-warp CTAs per SM; ring pipeline: 1..15.
@@ -108,7 +109,7 @@ typedef struct {
   int32_t grid_y;      /* CTAs along k (= splits) */
   int32_t threads;     /* threads per CTA */
   int32_t smem_bytes;  /* dynamic shared memory per CTA */
-  int64_t workspace_bytes; /* scratch: GEMV fp32 partials (0 if S == 1), MMA f16 A */
+  int64_t workspace_bytes; /* scratch: GEMV fp32 partials (0 if S == 1); MMA f16 A, then partials if S > 1 */
 } fi_tactic_info;
 
 /* ------------------------------------------------------------------ entry points */
@@ -146,7 +147,7 @@ FI_API int fi_nvfp4_pack_weights(const float* W, int64_t n, int64_t k, uint8_t* 
  * or n == 0 is a no-op; k == 0 writes zeros.
  * Workspace: a GEMV call with S > 1 needs fi_mm_workspace_bytes() bytes of device memory
  * for fp32 partials; an MMA call needs them for its f16 copy of A (each row times a power
- * of two) and the per-row scales. It uses the buffer registered with
+ * of two), the per-row scales and, when S > 1, the fp32 partials. It uses the buffer registered with
  * fi_set_workspace() for the current device (FI_ERR_WORKSPACE if that is too small); if
  * none is registered, the library allocates one with cudaMalloc (growing it when needed)
  * and keeps it until process exit, except while `stream` is capturing a CUDA graph,
@@ -179,7 +180,7 @@ FI_API int fi_mm_bf16_fp4_ex(const uint16_t* A, const uint8_t* Wq, const uint8_t
  * held until the process exits.
  * Arguments, tactics, preconditions and results are those of fi_mm_bf16_fp4.
  * Limit: the resolved tactic's fi_mm_workspace_bytes() (GEMV: 4 * splits * m * n; MMA: about
- * 2 * m * k) must not exceed FI_NOALLOC_SCRATCH_BYTES; a larger call returns
+ * 2 * m * k, plus 4 * splits * m * n when split) must not exceed FI_NOALLOC_SCRATCH_BYTES; a larger call returns
  * FI_ERR_WORKSPACE and launches nothing. Single-split GEMV tactics use no scratch.
  * Set-up: the first call on a device that reaches a launch looks up the array's device
  * address (cudaGetSymbolAddress, with that device current); make that first call before any
@@ -228,7 +229,8 @@ FI_API int64_t fi_default_tactic(int64_t m, int64_t n, int64_t k, int num_sms);
 FI_API int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, int cap);
 
 /* Workspace bytes a call with this shape and tactic needs (GEMV: 0 when S == 1; MMA: the
- * f16 activations and their row scales), or 0 for an invalid tactic. */
+ * f16 activations and their row scales, then the fp32 partials when S > 1), or 0 for an
+ * invalid tactic. */
 FI_API size_t fi_mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms);
 
 /* Register a caller-owned split-K workspace for the current device (device pointer,

@@ -82,7 +82,7 @@ def test_device_sized_split_is_m_independent():
 
 def test_default_table_is_constant_within_m_buckets():
     for n, k in [(4096, 14336), (14336, 4096), (512, 2048)]:
-        for bucket in ([1], [2, 3, 5, 8], [9, 16, 31, 32]):
+        for bucket in ([1], [2, 3, 4], [5, 8, 16, 32, 64, 256]):
             ts = {fi.default_tactic(m, n, k, B200_SMS) for m in bucket}
             assert len(ts) == 1, (n, k, bucket, ts)
 
@@ -200,9 +200,10 @@ def test_mma_tactic_resolution():
     # workspace: f16 activations [256, k] then 256 fp32 row scales
     assert info["workspace_bytes"] == 256 * 5120 * 2 + 256 * 4
     assert fi.resolve_tactic(33, 100, 64, t, B200_SMS)["workspace_bytes"] == 48 * 64 * 2 + 48 * 4
-    # the default table takes the MMA above m = 32 and the GEMV up to it
-    assert fi.resolve_tactic(33, 4096, 4096, fi.TACTIC_DEFAULT, B200_SMS)["kind"] == fi.KIND_MMA
-    assert fi.resolve_tactic(32, 4096, 4096, fi.TACTIC_DEFAULT, B200_SMS)["kind"] == fi.KIND_GEMV
+    # the default table takes the GEMV up to m = 4 and the MMA (device-sized split) above
+    assert fi.resolve_tactic(5, 4096, 4096, fi.TACTIC_DEFAULT, B200_SMS)["kind"] == fi.KIND_MMA
+    assert fi.resolve_tactic(4, 4096, 4096, fi.TACTIC_DEFAULT, B200_SMS)["kind"] == fi.KIND_GEMV
+    assert fi.resolve_tactic(32, 4096, 14336, fi.TACTIC_DEFAULT, B200_SMS)["splits"] == 9
     assert t in fi.list_tactics(64, 4096, 4096, B200_SMS)
 
 

@@ -108,3 +108,59 @@ def test_stalled_producer_reports_timeout_and_recovers():
         fi.debug_set(fi.DEBUG_WAIT_TIMEOUT_NS, 1_000_000_000)
     _gpu.assert_within_tolerance(_mm(A, dw), ref, "after recovery")
     assert fi.get_device_error() == 0
+
+
+@pytest.mark.parametrize("m,n,k,S", [(8, 1000, 2048, 3), (40, 300, 4096, 0), (1, 256, 512, 2), (128, 768, 1024, 16)])
+def test_split_k_parity(m, n, k, S):
+    """K split over grid.y: fp32 partials per split, summed in split order by the reduce kernel
+    (S = 0: the device-sized split)."""
+    A = inputs.activations(m, k, seed=m + S, outliers=True)
+    W, (Wq, Ws, g) = _gpu.weights(n, k, m + S)
+    ref = oracle.mm(A, Wq, Ws, g)
+    t = fi.make_tactic(fi.KIND_MMA, S, 0, 0)
+    _gpu.assert_within_tolerance(_mm(A, _gpu.device_weights(n, k, m + S), t), ref, f"MMA S={S} {m}x{n}x{k}")
+
+
+def test_split_k_exact_determinism_and_rows_independent_of_m():
+    n, k, S = 512, 2048, 4
+    t = fi.make_tactic(fi.KIND_MMA, S, 0, 0)
+    A, W = _exact_case(64, n, k, seed=5)
+    Wq, Ws, g = oracle.pack(W)
+    ref = oracle.mm(A, Wq, Ws, g)
+    want = np.array([[oracle.f32_to_bf16_bits(v) for v in row] for row in ref.astype(np.float32)], np.uint16)
+    dw = fi.pack_weights(torch.from_numpy(W).cuda())
+    assert np.array_equal(_mm(A, dw, t), want)
+    A2 = inputs.activations(200, k, seed=6, outliers=True)
+    dw2 = _gpu.device_weights(n, k, 6)
+    base = _mm(A2, dw2, t)
+    for _ in range(5):
+        assert np.array_equal(_mm(A2, dw2, t), base)
+    for m in (1, 17, 64, 128):
+        assert np.array_equal(_mm(A2[:m], dw2, t), base[:m]), m
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("m", [64, 256])
+def test_lm_head_default_sampled(m):
+    """The lm_head-like GEMM at full size in the launch configuration the bench times (default
+    tactic: the tensor-core path), against the oracle on every 97th column."""
+    n, k = inputs.LM_HEAD_NK
+    A = inputs.activations(m, k, seed=0)
+    W, (Wq, Ws, g) = _gpu.weights(n, k, 0, True)
+    got = _mm(A, _gpu.device_weights(n, k, 0, True), fi.TACTIC_DEFAULT)
+    cols = np.concatenate([np.arange(0, n, 97), [n - 1]])
+    ref = oracle.mm(A, Wq, Ws, g, cols=cols)
+    _gpu.assert_within_tolerance(got[:, cols], ref, f"lm_head m={m} (every 97th column)")
+
+
+@pytest.mark.parametrize("m", [8, 32])
+def test_small_batch_default_full_size_sampled(m):
+    """4096 x 14336 at m = 8 and 32 (the small-batch sweep) with the default tactic, which takes
+    the split-K tensor-core path there; every 13th column against the oracle."""
+    n, k = inputs.SMALL_BATCH_NK
+    A = inputs.activations(m, k, seed=1, outliers=True)
+    W, (Wq, Ws, g) = _gpu.weights(n, k, 1)
+    got = _mm(A, _gpu.device_weights(n, k, 1), fi.TACTIC_DEFAULT)
+    cols = np.concatenate([np.arange(0, n, 13), [n - 1]])
+    ref = oracle.mm(A, Wq, Ws, g, cols=cols)
+    _gpu.assert_within_tolerance(got[:, cols], ref, f"4096x14336 m={m}")
