@@ -154,7 +154,11 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
                          GemvGeometry* g, bool overlap) {
   const int64_t C = k / kChunkK;
   const int64_t nch = (C + S - 1) / S;  // chunks of the largest split
-  const int ctas = overlap ? 2 : (ctas_per_sm > 0 ? ctas_per_sm : (stream_wide(n, sms) ? 2 : 1));
+  // automatic CTA shape: two half-SM CTAs per SM for wide n, and at m = 1 (where the activations
+  // always fit half an SM); measured at m = 1: 4096 x 14336 8.84 us on 293 CTAs of 7 warps (R = 2)
+  // against 9.1 us on 147 CTAs of 14 warps
+  const bool wide = stream_wide(n, sms);
+  const int ctas = overlap ? 2 : (ctas_per_sm > 0 ? ctas_per_sm : (wide || m == 1 ? 2 : 1));
   if (ctas > 2) return set_error(FI_ERR_INVALID_ARG, "GEMV stream pipeline: at most 2 CTAs per SM");
   int nw = ctas == 1 ? 16 : 8;
   const int64_t budget = ctas == 1 ? kSmemBudget : kStreamHalfBudget;
@@ -162,7 +166,7 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
   const int64_t as_bytes = round_up(m * nch * 8, 128);
   const int rmax = std::min(4, gemv_rows_per_stage_max(m));  // registers: at most 4 rows per item
   int64_t r = r_req;
-  if (r == 0) r = std::min(ctas == 2 && !overlap ? 4 : 2, rmax);
+  if (r == 0) r = std::min(ctas == 2 && !overlap && wide ? 4 : 2, rmax);
   if (r < 1 || r > rmax || (r & (r - 1)) != 0)
     return set_error(FI_ERR_INVALID_ARG, "GEMV rows per item must be a power of two in 1..%d for m=%lld", rmax,
                      (long long)m);

@@ -64,7 +64,7 @@ def test_default_gemv_tactic_resolves_for_decode_shapes(n, k):
     full = 16 if info["ctas_per_sm"] == 1 else 8
     if warps < full:
         share = B200_SMS * (1 if pipe == 3 else info["ctas_per_sm"]) // info["splits"]
-        assert info["grid_x"] >= share - 1 or warps == 4, info
+        assert info["grid_x"] >= 0.95 * share or warps == 4, info  # whole groups per warp round the grid
     assert info["workspace_bytes"] == (info["splits"] * n * 4 if info["splits"] > 1 else 0)
 
 
