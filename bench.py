@@ -52,8 +52,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per launch of the GEMV kernel (dram__bytes_read.sum + dram__bytes_write.sum)
 # from one ncu capture per shape, keyed by the sha256 of the kernel source they were taken
 # on; ignored (traffic = null) when the source has changed since.
-NCU_TRAFFIC = {"source_sha256": "590fe5d56d1b360e49ebeb493d1af06ca603f71cd5ebe66af27d6a52e83206fa",
-               "bytes": {"14336x4096": 33_105_481, "4096x14336": 33_125_888}}
+NCU_TRAFFIC = {"source_sha256": "61cc4fd290e923abb59b879b18a5d30804be0c80a36418858be668314346520c",
+               "bytes": {"14336x4096": 33_104_677, "4096x14336": 33_125_120}}
 # the roofline's dominant-kernel figure: the GEMV alone (split 1, one launch per call) on the
 # two 33 MB serving shapes
 ROOFLINE_SHAPES = [(4096, 14336), (14336, 4096)]

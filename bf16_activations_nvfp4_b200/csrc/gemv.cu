@@ -4,43 +4,47 @@
 // messages: weights go from global memory straight to registers with many warps covering
 // the latency, each output row is reduced across a warp with shuffles, and a later commit
 // stages the activations in shared memory), re-designed for B200, where an m=1 GEMV has to
-// keep ~100 KB of weights in flight per SM to run at HBM speed:
+// keep ~100 KB of weights in flight per SM to run at HBM speed. Four pipelines share the
+// activation staging, the work split and the per-chunk arithmetic, so for one K split S they
+// give bitwise identical outputs:
 //
-//  * Warp specialisation. One producer warp per CTA streams weight rows HBM -> shared memory
-//    with bulk asynchronous copies (cp.async.bulk, completion counted on an mbarrier) into an
-//    NST-stage ring; 16 consumer warps decode from shared memory. In-flight bytes live in
-//    shared memory, not registers, and few large copies (a stage is ~16 KB) keep the copy
-//    engine's per-copy cost out of the way.
-//  * Programmatic dependent launch. The producer issues the first NST stages before the
-//    grid-dependency wait (weights are never written by the preceding kernel); the consumers
-//    wait, then stage the activations, so the weight stream overlaps the previous kernel's
-//    tail and the activation staging.
-//  * Work. Grid (G, S): blockIdx.y is the K split s; the G CTAs of a split own balanced,
-//    contiguous ranges of weight rows (every SM streams the same bytes, +-1 row). A ring stage
-//    holds RS consecutive rows over the split's whole k range, and consumer warp w computes
-//    stages w, w+16, w+32, ... of its CTA (every warp waits on and releases every stage, so a
-//    slot never runs more than one mbarrier phase ahead of a waiter), so a row is always
-//    computed by one warp and the activations it loads once per step serve all RS rows. With one split a stage is two bulk
-//    copies: the rows' contiguous codes and a 16-byte-aligned superset of their contiguous
-//    E4M3 scales (indexed from the remainder; where the superset would overrun the scale
-//    tensor the producer copies the scales with plain loads). With S > 1 each row's slice is
-//    copied on its own.
-//  * Arithmetic (fixed by k and S alone, hence bitwise identical for every m, RS, NST, G and
-//    CTAs per SM): A is staged as f16 with one power-of-two scale sf_a per 16-block that puts
-//    the block maximum in [2^9, 2^10) (exact for every element within 2^26 of its block
-//    maximum); codes are decoded by cvt.rn.f16x2.e2m1x2 (exact). Per 16-block, packed f16
-//    fused multiply-adds sum the even and the odd elements' products in element order (8
-//    steps each, partial sums below 2^16); the two half sums times the block's E4M3 scale go
-//    to fp32 through the mixed-precision fma.rn.f32.f16, and acc = fma(t, sf_a, acc). Lane L
-//    takes chunks L, L+32, L+64, ... of the split; the lanes combine through a fixed xor
+//  * Stream pipeline (gemv_stream_kernel, the default): every warp streams its own rows with
+//    per-thread cp.async into its own shared-memory ring; a lane copies exactly the cells it
+//    computes and waits only for its own copies (cp.async.wait_group), so there is no wait
+//    between threads. A straight-line fast path covers splits whose chunks are a multiple of
+//    64 (k = 4096, 14336 at S = 1). The overlapped variant sizes the CTAs for half an SM but
+//    launches one per SM, so the next call's CTAs are resident beside them, and prefetches
+//    each warp's weights into L2 first.
+//  * Register pipeline (gemv_reg_kernel): the pages' own design, weights straight to registers
+//    with 16-byte loads, a ring of D chunk iterations in flight per warp.
+//  * Ring pipeline (gemv_nvfp4_kernel): one producer warp per CTA streams whole rows with bulk
+//    copies (cp.async.bulk, completion counted on an mbarrier) into an NST-stage ring; 16
+//    consumer warps decode from it. Its waits are bounded (below); it also runs k = 65536 at
+//    m = 1, whose activations do not fit the other pipelines' shared memory.
+//  * Programmatic dependent launch. Weights are never written by the preceding kernel, so each
+//    pipeline issues its first weight copies before the grid-dependency wait and stages the
+//    activations after it.
+//  * Work. Grid (G, S): blockIdx.y is the K split s; the warps of a split own balanced,
+//    contiguous groups of weight rows (ring pipeline: CTAs own row ranges and warps take
+//    stages in turn), so a row is always computed by one warp and the activations it loads
+//    once per chunk serve all rows of its group.
+//  * Arithmetic (fixed by k and S alone, hence bitwise identical for every m, pipeline, rows
+//    per group, CTA shape and grid): A is staged as f16 with one power-of-two scale sf_a per
+//    16-block that puts the block maximum in [2^9, 2^10) (exact for every element within 2^26
+//    of its block maximum); codes are decoded by cvt.rn.f16x2.e2m1x2 (exact). Per 16-block,
+//    packed f16 fused multiply-adds sum the even and the odd elements' products in element
+//    order (8 steps each, partial sums below 2^16); the two half sums times the block's E4M3
+//    scale go to fp32 through the mixed-precision fma.rn.f32.f16, and acc = fma(t, sf_a, acc).
+//    Lane L takes chunks L, L+32, L+64, ... of the split; the lanes combine through a fixed xor
 //    butterfly (all lanes end with the same bits). S == 1 writes bf16_rn(acc * gscale); S > 1
 //    writes fp32 partials for the reduce kernel. The f16 half sums are what make the inner loop
 //    cheap on sm_100: the packed f16 FMA issues to the other FMA port than the e2m1 conversion,
 //    so decode and products run side by side; their rounding (one f16 rounding per step on
 //    magnitudes below 2^16) stays far below the bf16 output's own.
-//  * Bounded waits. Every mbarrier wait gives up after a time limit (%globaltimer): it sets a
-//    device error flag and a CTA-wide abort flag, the CTA finishes its control flow without
-//    computing, and the producer waits (bounded) for the copies it issued before exiting.
+//  * Bounded waits (ring pipeline). Every mbarrier wait gives up after a time limit
+//    (%globaltimer): it sets a device error flag and a CTA-wide abort flag, the CTA finishes
+//    its control flow without computing, and the producer waits (bounded) for the copies it
+//    issued before exiting.
 #include <cstdint>
 #include <cstring>
 
