@@ -64,6 +64,21 @@ int fi_mm_bf16_fp4_noalloc(const uint16_t* A, const uint8_t* Wq, const uint8_t* 
   // Empty problems, k == 0 and invalid sizes need no scratch: the regular checks answer them.
   if (m <= 0 || n <= 0 || k <= 0 || k % 32 != 0)
     return fi_mm_bf16_fp4_ex(A, Wq, Wscale, gscale, out, m, n, k, tactic, nullptr, 0, stream);
+  // The default tactic whose scratch would not fit takes, with the same kind, the largest
+  // split below its own that fits (the split changes the bits, as any split does).
+  if (tactic == FI_TACTIC_DEFAULT && fi_mm_workspace_bytes(m, n, k, tactic, 0) > kNoAllocScratchBytes) {
+    fi_tactic_info info;
+    if (fi_resolve_tactic(m, n, k, tactic, 0, &info) == FI_OK) {
+      for (int S = info.splits - 1; S >= 1; --S) {
+        const int64_t t = FI_TACTIC(info.kind, S, 0, info.kind == FI_KIND_GEMV ? (info.variant >> 4) << 4 : 0);
+        const size_t w = fi_mm_workspace_bytes(m, n, k, t, 0);
+        if (w > 0 && w <= kNoAllocScratchBytes) {
+          tactic = t;
+          break;
+        }
+      }
+    }
+  }
   // Refuse, before any launch, a call whose partials would not fit the static scratch. (An
   // invalid tactic reports 0 here and is rejected with its own message below.)
   const size_t need = fi_mm_workspace_bytes(m, n, k, tactic, 0);

@@ -180,8 +180,11 @@ FI_API int fi_mm_bf16_fp4_ex(const uint16_t* A, const uint8_t* Wq, const uint8_t
  * held until the process exits.
  * Arguments, tactics, preconditions and results are those of fi_mm_bf16_fp4.
  * Limit: the resolved tactic's fi_mm_workspace_bytes() (GEMV: 4 * splits * m * n; MMA: about
- * 2 * m * k, plus 4 * splits * m * n when split) must not exceed FI_NOALLOC_SCRATCH_BYTES; a larger call returns
- * FI_ERR_WORKSPACE and launches nothing. Single-split GEMV tactics use no scratch.
+ * 2 * m * k, plus 4 * splits * m * n when split) must not exceed FI_NOALLOC_SCRATCH_BYTES; a
+ * larger call returns FI_ERR_WORKSPACE and launches nothing. Single-split GEMV tactics use no
+ * scratch. With FI_TACTIC_DEFAULT, a default whose scratch would not fit is replaced by the
+ * same kind with the largest smaller split that fits (so its bits may differ from
+ * fi_mm_bf16_fp4's default for that shape).
  * Set-up: the first call on a device that reaches a launch looks up the array's device
  * address (cudaGetSymbolAddress, with that device current); make that first call before any
  * stream capture begins.

@@ -17,6 +17,7 @@ import pytest
 import torch
 
 import bf16_activations_nvfp4_b200 as fi
+import oracle
 from bf16_activations_nvfp4_b200 import inputs
 from tests import _gpu
 
@@ -86,3 +87,22 @@ def test_partials_beyond_the_static_scratch_are_refused():
     assert "scratch" in fi.last_error()
     torch.cuda.synchronize()
     assert bool((out == 7.0).all())  # nothing was launched
+
+
+def test_default_tactic_falls_back_to_a_split_that_fits():
+    """4096 x 14336 at m = 32: the default (the tensor-core path with 9 K splits) needs more
+    scratch than the static array holds; the allocation-free entry point takes the largest
+    smaller split that fits and stays within tolerance."""
+    m, n, k = 32, 4096, 14336
+    assert fi.workspace_bytes(m, n, k) > 4 << 20
+    A_bits = inputs.activations(m, k, seed=3)
+    W, (Wq_o, Ws_o, g_o) = _gpu.weights(n, k, 3)
+    dw = _gpu.device_weights(n, k, 3)
+    cols = np.concatenate([np.arange(0, n, 31), [n - 1]])
+    ref = oracle.mm(A_bits, Wq_o, Ws_o, g_o, cols=cols)
+    Wq, Ws, g = dw
+    out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    st = _noalloc(_gpu.dev_bf16(A_bits), Wq, Ws, g, out, fi.TACTIC_DEFAULT)
+    assert st == 0, fi.last_error()
+    torch.cuda.synchronize()
+    _gpu.assert_within_tolerance(_gpu.host_bits(out)[:, cols], ref, "no-alloc default, m=32")
