@@ -217,3 +217,34 @@ def test_mma_resolve_rejects(m, n, k, tactic, status):
     with pytest.raises(fi.FiError) as e:
         fi.resolve_tactic(m, n, k, tactic, B200_SMS)
     assert e.value.status == status
+
+
+def test_mma_device_sized_split_follows_the_wave_step_model():
+    """The MMA path's device-sized split (S = 0): one CTA per SM, so the choice is the S with the
+    fewest waves of 64-k steps (per-CTA start and epilogue, the reduce and the partials
+    counted). Small n needs a split, the lm_head-like shape does not."""
+    mma = fi.make_tactic(fi.KIND_MMA, 0, 0, 0)
+    cases = {(32, 4096, 14336): 9, (8, 4096, 14336): 9, (64, 152064, 5120): 1, (256, 152064, 5120): 1}
+    for (m, n, k), S in cases.items():
+        info = fi.resolve_tactic(m, n, k, mma, B200_SMS)
+        assert info["splits"] == S and info["grid_y"] == S, (m, n, k, info)
+        assert info["grid_x"] == -(-n // 256)
+        if S > 1:  # f16 activations, their row scales, then the partials at a 256-byte boundary
+            assert info["workspace_bytes"] >= S * m * n * 4 + 2 * 16 * k
+    # explicit splits are kept, up to k / 64 steps
+    assert fi.resolve_tactic(64, 4096, 4096, fi.make_tactic(fi.KIND_MMA, 3, 0, 0), B200_SMS)["splits"] == 3
+    with pytest.raises(fi.FiError):
+        fi.resolve_tactic(64, 4096, 128, fi.make_tactic(fi.KIND_MMA, 3, 0, 0), B200_SMS)
+
+
+def test_register_pipeline_geometry():
+    """Pipeline 4: shared memory holds only the staged activations, 1 or 2 rows per warp, and
+    the grid spreads over the SMs like the stream pipeline's."""
+    for n, k in [(10304, 2688), (4096, 14336), (512, 2048)]:
+        info = fi.resolve_tactic(1, n, k, fi.make_tactic(fi.KIND_GEMV, 1, 2, 0x40), B200_SMS)
+        assert info["variant"] >> 4 == 4 and info["variant"] & 0xF == 2
+        chunks = k // 32
+        assert info["smem_bytes"] == -(-((chunks + 31) // 32 * 2048) // 128) * 128 + -(-(chunks * 8) // 128) * 128
+        assert info["grid_x"] <= 2 * B200_SMS and info["threads"] % 32 == 0
+    with pytest.raises(fi.FiError):
+        fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, 1, 0, 0x44), B200_SMS)  # 4 rows would spill
