@@ -11,6 +11,7 @@ raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -65,6 +66,9 @@ def library_path() -> str:
 def library() -> ctypes.CDLL:
     """Load libfi_nvfp4.so (built by ``python -m bf16_activations_nvfp4_b200.build``)."""
     global _lib
+    lib = _lib
+    if lib is not None:  # loaded: no lock on the per-call path
+        return lib
     with _lock:
         if _lib is not None:
             return _lib
@@ -232,17 +236,22 @@ def mm_bf16_fp4(A: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor, gscale:
     else:
         _require(out, "out", torch.bfloat16, 2)
     lib = library()
-    with torch.cuda.device(A.device):
-        s = _stream(A.device)
+    dev = A.device
+    # the library works on the current device: switch only when A lives on another one
+    ctx = torch.cuda.device(dev) if dev.index != torch.cuda.current_device() else contextlib.nullcontext()
+    with ctx:
+        s = torch.cuda.current_stream(dev).cuda_stream
         if workspace is None:
             st = lib.fi_mm_bf16_fp4(A.data_ptr(), Wq.data_ptr(), Wscale.data_ptr(), gscale.data_ptr(),
                                     out.data_ptr(), m, n, k, tactic, s)
-            _check(st, "fi_mm_bf16_fp4")
+            if st:
+                _check(st, "fi_mm_bf16_fp4")
         else:
             st = lib.fi_mm_bf16_fp4_ex(A.data_ptr(), Wq.data_ptr(), Wscale.data_ptr(), gscale.data_ptr(),
                                        out.data_ptr(), m, n, k, tactic, workspace.data_ptr(),
                                        workspace.numel() * workspace.element_size(), s)
-            _check(st, "fi_mm_bf16_fp4_ex")
+            if st:
+                _check(st, "fi_mm_bf16_fp4_ex")
     return out
 
 
