@@ -155,10 +155,13 @@ int gemv_stream_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int 
   const int64_t C = k / kChunkK;
   const int64_t nch = (C + S - 1) / S;  // chunks of the largest split
   // automatic CTA shape: two half-SM CTAs per SM for wide n, and at m = 1 (where the activations
-  // always fit half an SM); measured at m = 1: 4096 x 14336 8.84 us on 293 CTAs of 7 warps (R = 2)
-  // against 9.1 us on 147 CTAs of 14 warps
+  // always fit half an SM) when the 2-row groups fill two CTAs of at least 4 warps on every SM;
+  // measured at m = 1: 4096 x 14336 8.78 us on 293 CTAs of 7 warps (R = 2) against 9.1 us on
+  // 147 CTAs of 14; 2048 x 7168 (1024 groups) 4.98 us on 256 CTAs of 4 warps, which leave 40
+  // SMs with one CTA, against 4.35 us on 147 CTAs of 7
   const bool wide = stream_wide(n, sms);
-  const int ctas = overlap ? 2 : (ctas_per_sm > 0 ? ctas_per_sm : (wide || m == 1 ? 2 : 1));
+  const bool fill2 = m == 1 && (n + 1) / 2 >= (int64_t)sms * 2 * 4;
+  const int ctas = overlap ? 2 : (ctas_per_sm > 0 ? ctas_per_sm : (wide || fill2 ? 2 : 1));
   if (ctas > 2) return set_error(FI_ERR_INVALID_ARG, "GEMV stream pipeline: at most 2 CTAs per SM");
   int nw = ctas == 1 ? 16 : 8;
   const int64_t budget = ctas == 1 ? kSmemBudget : kStreamHalfBudget;
