@@ -38,7 +38,7 @@ def test_parity_against_oracle(m, n, k, seed):
     _gpu.assert_within_tolerance(_mm(A, _gpu.device_weights(n, k, seed)), ref, f"MMA {m}x{n}x{k}")
 
 
-def test_default_table_takes_mma_above_m32():
+def test_default_table_takes_mma_for_larger_m():
     info = fi.resolve_tactic(64, 4096, 14336, fi.TACTIC_DEFAULT)
     assert info["kind"] == fi.KIND_MMA
     m, n, k = 64, 1000, 2048
