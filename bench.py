@@ -50,9 +50,9 @@ COLD_BYTES = 300 << 20  # per-shape footprint of the rotating weight copies
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes per launch of the GEMV kernel (dram__bytes_read.sum + dram__bytes_write.sum)
-# from one ncu capture per shape, keyed by the sha256 of the kernel source they were taken
-# on; ignored (traffic = null) when the source has changed since.
-NCU_TRAFFIC = {"source_sha256": "61cc4fd290e923abb59b879b18a5d30804be0c80a36418858be668314346520c",
+# from one ncu capture per shape, keyed by the sha256 of the kernel code they were taken on
+# (comments excluded); ignored (traffic = null) when that code has changed since.
+NCU_TRAFFIC = {"source_sha256": "57a8d32ff78458b5ee5bf631504ab7a3e47c1303506de4d74c6a0c8475536fb0",
                "bytes": {"14336x4096": 33_104_677, "4096x14336": 33_125_120}}
 # the roofline's dominant-kernel figure: the GEMV alone (split 1, one launch per call) on the
 # two 33 MB serving shapes
@@ -130,12 +130,39 @@ def run_lm_head(dev, stream, peaks) -> dict:
             "per_m": rows}
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source with its comments removed and each line's trailing blanks and the blank
+    lines dropped, so that an edit to comments alone keeps the hash; string and character
+    literals are kept as written."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (line.rstrip() for line in "".join(out).splitlines())
+    return "\n".join(line for line in lines if line)
+
+
 def _gemv_source_sha() -> str:
+    """sha256 of the GEMV kernel's code (comments excluded) in gemv.cu and common.cuh."""
     import hashlib
     h = hashlib.sha256()
     for name in ("gemv.cu", "common.cuh"):
-        with open(os.path.join(ROOT, "bf16_activations_nvfp4_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "bf16_activations_nvfp4_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

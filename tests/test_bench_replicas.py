@@ -41,3 +41,15 @@ def test_algorithmic_bytes_formula():
     # n*k/2 codes + n*k/16 scales + 2*m*k activations + 2*m*n outputs
     assert bench.algorithmic_bytes(1, 4096, 14336) == 33_067_008
     assert bench.algorithmic_bytes(1, 512, 2048) == 594_944
+
+
+def test_traffic_hash_ignores_comments_only():
+    """The stored DRAM-traffic figures are keyed by the kernel code with comments removed:
+    comment edits keep the key, a code edit (even inside a PTX string) changes it."""
+    src = ('// header\n#include "a.h"\n/* block\n comment */ int x = 1; // trailing\n'
+           'asm("mov.b32 %0, %1; // not a comment");\n')
+    stripped = bench._strip_comments(src)
+    assert stripped == '#include "a.h"\n int x = 1;\nasm("mov.b32 %0, %1; // not a comment");'
+    assert bench._strip_comments(src.replace("trailing", "other words")) == stripped
+    assert bench._strip_comments(src.replace("int x = 1", "int x = 2")) != stripped
+    assert bench._strip_comments(src.replace("%0, %1", "%1, %0")) != stripped
