@@ -303,9 +303,10 @@ static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms)
 }
 
 // GEMV variant byte: low nibble = weight rows computed together by one warp (ring pipeline:
-// rows per ring stage; stream pipeline: rows per work item; 0 = automatic); high nibble = the
-// pipeline (0 = automatic = stream, 1 = stream, 2 = ring). Both pipelines give the same bits
-// for the same S. Splits 0 = device-sized, resolved for m <= 32 so that the resolved S (and
+// rows per ring stage; the others: rows per work item; 0 = automatic); high nibble = the
+// pipeline (0 = automatic: stream, or ring when the activations do not fit; 1 = stream, 2 =
+// ring, 3 = overlapped stream, 4 = register). Every pipeline gives the same bits for the same
+// S. Splits 0 = device-sized, resolved for m <= 32 so that the resolved S (and
 // the bits) never depend on m.
 static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var,
                         int sms, fi_tactic_info* out) {
@@ -358,8 +359,9 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
   return FI_OK;
 }
 
-// MMA tactic: splits 0 or 1 (one split), CTAs per SM 0 or 1, variant 0. Needs m <= 256 and k a
-// multiple of 64; the workspace holds the f16 activations and their row scales.
+// MMA tactic: splits 1..k/64 (0 = device-sized), CTAs per SM 0 or 1, variant 0. Needs m <= 256
+// and k a multiple of 64; the workspace holds the f16 activations and their row scales, then
+// the [S, m, n] fp32 partials when S > 1.
 static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var, int sms,
                        fi_tactic_info* out) {
   if (m > kMmaMaxM)
@@ -665,9 +667,10 @@ int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, 
   clear_error();
   const int sms = sms_or_device(num_sms);
   if (sms <= 0) return set_error(FI_ERR_CUDA, "no device to query the SM count from");
-  // the split menu {1, 2, 4, 8, device-sized} on both pipelines, each with the automatic row
-  // count and with one and two rows per warp, the stream pipeline also with two CTAs per SM;
-  // entries resolving to the same launch are listed once
+  // the split menu {1, 2, 4, 8, device-sized} on the stream and ring pipelines, each with the
+  // automatic row count and with one and two rows per warp; the stream pipeline also with two
+  // CTAs per SM; the overlapped and register pipelines; the MMA. Entries resolving to the same
+  // launch are listed once
   int64_t cand[64];
   int nc = 0;
   const int splits[] = {1, 2, 4, 8, 0};
@@ -677,7 +680,7 @@ int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, 
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 2, kPipeStream << 4);
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeOverlap << 4);
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeReg << 4);
-  cand[nc++] = FI_TACTIC(FI_KIND_MMA, 1, 0, 0);
+  for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_MMA, S, 0, 0);
   fi_tactic_info seen[64];
   int nseen = 0, count = 0;
   for (int c = 0; c < nc; ++c) {

@@ -194,7 +194,7 @@ __device__ __forceinline__ float block_acc(uint32_t h, uint32_t sh, float sa, fl
 
 // One 32-k chunk of one weight row against one activation row: av the chunk's 16 staged f16
 // pairs, sa its two block scales, wf the decoded codes, sh the two E4M3 block scales as f16x2.
-// Both pipelines call this, so their bits agree.
+// Every pipeline calls this, so their bits agree.
 __device__ __forceinline__ float chunk_acc(const uint32_t (&av)[16], float2 sa, const uint32_t (&wf)[16], uint32_t sh,
                                            float acc) {
   const uint32_t h0 = hdot8(av, wf);
@@ -480,8 +480,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_nvfp4_kernel(GemvArgs p)
 //
 // The work item of a warp is (row group, chunk iteration t): chunk c = 32 t + L of the split
 // for R consecutive rows. Items run in order, each lane taking chunks L, L+32, ... of every
-// row in increasing order with the same per-chunk arithmetic as the ring pipeline, so the
-// two pipelines give bitwise identical results for the same S.
+// row in increasing order with the same per-chunk arithmetic as the other pipelines, so all
+// of them give bitwise identical results for the same S.
 //
 // A CTA is 8 warps and at most about half of an SM's shared memory and registers, so the
 // CTAs of the next programmatically dependent launch can become resident beside it and start

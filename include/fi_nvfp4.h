@@ -72,8 +72,9 @@ typedef enum {
  *                MMA: 0 or 1;
  *   variant      GEMV: low nibble = weight rows computed together by one warp (stream
  *                pipeline 1, 2 or 4; ring pipeline 1, 2, 4 or 8, at most 16 / m rounded to a
- *                power of two; 0 = automatic); high nibble = pipeline (0 = automatic =
- *                1 = per-warp asynchronous copies, 2 = producer-warp ring, 3 = per-warp
+ *                power of two; 0 = automatic); high nibble = pipeline (0 = automatic:
+ *                1, or 2 where the activations do not fit a half SM; 1 = per-warp
+ *                asynchronous copies, 2 = producer-warp ring, 3 = per-warp
  *                copies in one half-SM CTA per SM, so that consecutive calls overlap, with
  *                an L2 prefetch of weights up to 40 MB; its CTAs-per-SM field is ignored;
  *                4 = weights loaded straight to registers, 1 or 2 rows per warp). MMA: 0.
@@ -104,7 +105,7 @@ typedef struct {
   int32_t kind;        /* FI_KIND_GEMV or FI_KIND_MMA */
   int32_t splits;      /* resolved S >= 1 */
   int32_t ctas_per_sm; /* resolved co-resident CTAs per SM */
-  int32_t variant;     /* resolved variant (GEMV rows per warp) */
+  int32_t variant;     /* resolved variant (GEMV: rows per warp | pipeline << 4; MMA: 0) */
   int32_t grid_x;      /* CTAs along n */
   int32_t grid_y;      /* CTAs along k (= splits) */
   int32_t threads;     /* threads per CTA */
@@ -228,7 +229,10 @@ FI_API int fi_resolve_tactic(int64_t m, int64_t n, int64_t k, int64_t tactic, in
 FI_API int64_t fi_default_tactic(int64_t m, int64_t n, int64_t k, int num_sms);
 
 /* Enumerate the valid tactics for a shape into out[0 .. cap-1]; returns how many exist
- * (which may exceed cap), or a negative status. */
+ * (which may exceed cap), or a negative status. The menu: splits {1, 2, 4, 8, device-sized}
+ * for every GEMV pipeline (stream and ring also at one and two rows per warp, the stream
+ * pipeline also at two CTAs per SM) and for the MMA; codes resolving to the same launch are
+ * listed once, codes the shape does not support are left out. */
 FI_API int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, int cap);
 
 /* Workspace bytes a call with this shape and tactic needs (GEMV: 0 when S == 1; MMA: the

@@ -110,6 +110,17 @@ def test_list_tactics_unique_and_valid():
         fi.resolve_tactic(1, 4096, 14336, t, B200_SMS)
 
 
+def test_list_tactics_offers_the_mma_split_menu():
+    """The MMA appears with splits 1, 2, 4, 8 and device-sized, one entry per distinct launch.
+    Above m = 32 only MMA codes are listed; where k is not a multiple of 64, only GEMV codes."""
+    ts = fi.list_tactics(64, 4096, 4096, B200_SMS)
+    mma = [fi.resolve_tactic(64, 4096, 4096, t, B200_SMS) for t in ts if fi.tactic_fields(t)["kind"] == fi.KIND_MMA]
+    assert {i["splits"] for i in mma} >= {1, 2, 4, 8}
+    assert len({i["splits"] for i in mma}) == len(mma)
+    assert all(fi.tactic_fields(t)["kind"] == fi.KIND_MMA for t in ts)  # m = 64 > the GEMV's 32
+    assert all(fi.tactic_fields(t)["kind"] == fi.KIND_GEMV for t in fi.list_tactics(4, 1000, 1056, B200_SMS))
+
+
 def test_workspace_bytes():
     t = fi.make_tactic(fi.KIND_GEMV, 4, 0, 1)
     assert fi.workspace_bytes(3, 1000, 4096, t, B200_SMS) == 4 * 3 * 1000 * 4
