@@ -259,3 +259,26 @@ def test_register_pipeline_geometry():
         assert info["grid_x"] <= 2 * B200_SMS and info["threads"] % 32 == 0
     with pytest.raises(fi.FiError):
         fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, 1, 0, 0x44), B200_SMS)  # 4 rows would spill
+
+
+def test_automatic_pipeline_for_split_calls_at_m1():
+    """At m = 1 with a K split, the automatic pipeline takes the register pipeline (two CTAs per
+    SM) where k % 256 != 0 and four rows per stream item otherwise; S itself is unchanged, and
+    m > 1 keeps the stream pipeline's own row choice."""
+    for n, k in [(4096, 14336), (2048, 7168), (4096, 4096), (10304, 2688)]:
+        for S in (2, 4, 8):
+            info = fi.resolve_tactic(1, n, k, fi.make_tactic(fi.KIND_GEMV, S, 0, 0), B200_SMS)
+            assert info["splits"] == S
+            if k % 256:
+                assert (info["variant"] >> 4, info["ctas_per_sm"]) == (4, 2)
+            else:
+                assert info["variant"] == 0x14
+        # S = 1 is not affected, and the device-sized split resolves to the same S at every m
+        assert fi.resolve_tactic(1, n, k, fi.make_tactic(fi.KIND_GEMV, 1, 0, 0), B200_SMS)["variant"] >> 4 == 1
+        s1 = fi.resolve_tactic(1, n, k, fi.make_tactic(fi.KIND_GEMV, 0, 0, 0), B200_SMS)["splits"]
+        s4 = fi.resolve_tactic(4, n, k, fi.make_tactic(fi.KIND_GEMV, 0, 0, 0), B200_SMS)["splits"]
+        assert s1 == s4
+    # explicit rows or pipeline are taken as given
+    assert fi.resolve_tactic(1, 4096, 14336, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0x12), B200_SMS)["variant"] == 0x12
+    assert fi.resolve_tactic(1, 4096, 14336, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0x01), B200_SMS)["variant"] & 15 == 1
+    assert fi.resolve_tactic(2, 4096, 14336, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0), B200_SMS)["variant"] >> 4 == 1
