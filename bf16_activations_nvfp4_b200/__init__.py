@@ -198,6 +198,47 @@ def _require(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
 
 
+def _same_device(ref: torch.Tensor, **tensors) -> None:
+    d = ref.get_device()
+    for name, t in tensors.items():
+        if t is not None and t.get_device() != d:
+            raise ValueError(f"{name} is on {t.device}, the operands on {ref.device}")
+
+
+def _pack_out_check(W: torch.Tensor, out: tuple) -> tuple:
+    """The caller's (Wq, Wscale, gscale) buffers for W [n, k], checked against W's shape,
+    dtype and device (the kernel writes n*k/2, n*k/16 and 1 elements there)."""
+    n, k = W.shape
+    if len(out) != 3:
+        raise ValueError("out must be (Wq, Wscale, gscale)")
+    Wq, Ws, g = out
+    for name, t, dtype, shape in (("Wq", Wq, torch.uint8, (n, k // 2)), ("Wscale", Ws, torch.uint8, (n, k // 16)),
+                                  ("gscale", g, torch.float32, (1,))):
+        if not isinstance(t, torch.Tensor) or t.dtype != dtype or tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {shape}")
+    _same_device(W, Wq=Wq, Wscale=Ws, gscale=g)
+    return Wq, Ws, g
+
+
+def _mm_shapes(A: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor, gscale: torch.Tensor,
+               out: torch.Tensor | None) -> tuple:
+    """(m, n, k) of an mm call, after checking that the operands' shapes agree, that `out` is
+    [m, n] and that every operand is on A's device."""
+    m, k = A.shape
+    n, kq = Wq.shape
+    if kq * 2 != k or Wscale.shape != (n, k // 16):
+        raise ValueError(f"shape mismatch: A {tuple(A.shape)}, Wq {tuple(Wq.shape)}, Wscale {tuple(Wscale.shape)}")
+    if gscale.shape != (1,):
+        raise ValueError(f"gscale must hold one element, got shape {tuple(gscale.shape)}")
+    if out is not None and out.shape != (m, n):
+        raise ValueError(f"out must be [{m}, {n}], got {tuple(out.shape)}")
+    d = A.get_device()
+    if Wq.get_device() != d or Wscale.get_device() != d or gscale.get_device() != d or (
+            out is not None and out.get_device() != d):
+        _same_device(A, Wq=Wq, Wscale=Wscale, gscale=gscale, out=out)
+    return m, n, k
+
+
 def pack_weights(W: torch.Tensor, out: tuple | None = None):
     """Quantise fp32 W [n, k] (CUDA) to NVFP4 -> (Wq uint8 [n, k/2], Wscale uint8 [n, k/16],
     gscale fp32 [1]), all on W's device."""
@@ -208,7 +249,7 @@ def pack_weights(W: torch.Tensor, out: tuple | None = None):
         Ws = torch.empty((n, k // 16), dtype=torch.uint8, device=W.device)
         g = torch.empty(1, dtype=torch.float32, device=W.device)
     else:
-        Wq, Ws, g = out
+        Wq, Ws, g = _pack_out_check(W, out)
     with torch.cuda.device(W.device):
         _check(library().fi_nvfp4_pack_weights(W.data_ptr(), n, k, Wq.data_ptr(), Ws.data_ptr(),
                                                g.data_ptr(), _stream(W.device)), "fi_nvfp4_pack_weights")
@@ -227,14 +268,15 @@ def mm_bf16_fp4(A: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor, gscale:
     _require(Wq, "Wq", torch.uint8, 2)
     _require(Wscale, "Wscale", torch.uint8, 2)
     _require(gscale, "gscale", torch.float32, 1)
-    m, k = A.shape
-    n = Wq.shape[0]
-    if Wq.shape[1] * 2 != k or Wscale.shape != (n, k // 16):
-        raise ValueError(f"shape mismatch: A {tuple(A.shape)}, Wq {tuple(Wq.shape)}, Wscale {tuple(Wscale.shape)}")
+    if out is not None:
+        _require(out, "out", torch.bfloat16, 2)
+    if workspace is not None:
+        if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        _same_device(A, workspace=workspace)
+    m, n, k = _mm_shapes(A, Wq, Wscale, gscale, out)
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=A.device)
-    else:
-        _require(out, "out", torch.bfloat16, 2)
     lib = library()
     dev = A.device
     # the library works on the current device: switch only when A lives on another one
@@ -260,8 +302,15 @@ def splitk_reduce(partials: torch.Tensor, gscale: torch.Tensor, out: torch.Tenso
     _require(partials, "partials", torch.float32, 3)
     _require(gscale, "gscale", torch.float32, 1)
     S, m, n = partials.shape
+    if gscale.numel() != 1:
+        raise ValueError(f"gscale must hold one element, got {gscale.numel()}")
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=partials.device)
+    else:
+        _require(out, "out", torch.bfloat16, 2)
+        if tuple(out.shape) != (m, n):
+            raise ValueError(f"out must be [{m}, {n}], got {tuple(out.shape)}")
+    _same_device(partials, gscale=gscale, out=out)
     with torch.cuda.device(partials.device):
         _check(library().fi_splitk_reduce(partials.data_ptr(), S, m, n, gscale.data_ptr(), out.data_ptr(),
                                           _stream(partials.device)), "fi_splitk_reduce")

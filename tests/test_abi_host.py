@@ -282,3 +282,48 @@ def test_automatic_pipeline_for_split_calls_at_m1():
     assert fi.resolve_tactic(1, 4096, 14336, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0x12), B200_SMS)["variant"] == 0x12
     assert fi.resolve_tactic(1, 4096, 14336, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0x01), B200_SMS)["variant"] & 15 == 1
     assert fi.resolve_tactic(2, 4096, 14336, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0), B200_SMS)["variant"] >> 4 == 1
+
+
+class _OnDevice:
+    """Shape and device stand-in for a tensor on another GPU (no GPU needed)."""
+
+    def __init__(self, t, index):
+        self.shape, self._index = t.shape, index
+        self.device = f"cuda:{index}"
+
+    def get_device(self):
+        return self._index
+
+
+def test_binding_checks_shapes_and_devices_before_any_launch():
+    """The Python binding refuses operands the kernels would read or write out of bounds:
+    `out` must be [m, n], Wscale [n, k/16], gscale one element, and every operand on A's
+    device; pack_weights' `out` buffers must match W."""
+    import torch
+    m, n, k = 2, 64, 128
+    A = torch.empty((m, k), dtype=torch.bfloat16)
+    Wq = torch.empty((n, k // 2), dtype=torch.uint8)
+    Ws = torch.empty((n, k // 16), dtype=torch.uint8)
+    g = torch.empty(1)
+    out = torch.empty((m, n), dtype=torch.bfloat16)
+    assert fi._mm_shapes(A, Wq, Ws, g, out) == (m, n, k)
+    assert fi._mm_shapes(A, Wq, Ws, g, None) == (m, n, k)
+    for bad in (torch.empty((m, n - 1), dtype=torch.bfloat16), torch.empty((m + 1, n), dtype=torch.bfloat16)):
+        with pytest.raises(ValueError, match="out must be"):
+            fi._mm_shapes(A, Wq, Ws, g, bad)
+    with pytest.raises(ValueError, match="shape mismatch"):
+        fi._mm_shapes(A, Wq, torch.empty((n, k // 32), dtype=torch.uint8), g, out)
+    with pytest.raises(ValueError, match="shape mismatch"):
+        fi._mm_shapes(A, torch.empty((n, k), dtype=torch.uint8), Ws, g, out)
+    with pytest.raises(ValueError, match="gscale"):
+        fi._mm_shapes(A, Wq, Ws, torch.empty(2), out)
+    with pytest.raises(ValueError, match="is on cuda:1"):
+        fi._mm_shapes(_OnDevice(A, 0), _OnDevice(Wq, 1), _OnDevice(Ws, 0), _OnDevice(g, 0), None)
+    with pytest.raises(ValueError, match="out is on cuda:1"):
+        fi._mm_shapes(_OnDevice(A, 0), _OnDevice(Wq, 0), _OnDevice(Ws, 0), _OnDevice(g, 0), _OnDevice(out, 1))
+    W = torch.empty((n, k))
+    assert fi._pack_out_check(W, (Wq, Ws, g)) == (Wq, Ws, g)
+    for bad in [(Wq, Ws), (Wq[:, :-1], Ws, g), (Wq, Ws.to(torch.int8), g), (Wq, Ws, torch.empty(2)),
+                (Wq, Ws, torch.empty(1, dtype=torch.float64))]:
+        with pytest.raises(ValueError):
+            fi._pack_out_check(W, bad)
