@@ -406,7 +406,7 @@ def run_fi(args, rank: int, world: int) -> dict | None:
             "m": M, "calls_per_step": len(calls),
             "tactics": "GEMV at split-K S in {1,2,4,8,device-sized} for every shape",
             "weights": "N(0,0.02) -> NVFP4 (library pack)", "activations": "N(0,1) -> bf16", "seed": 0,
-            "l2": "inputs larger than L2: every call reads its own weight copy, >= 300 MB of copies per shape",
+            "l2": "inputs larger than L2: the 25 calls of a step read 25 distinct weight copies (about 500 MB); per-call graphs rotate over >= 300 MB of copies per shape",
             "timing": "CUDA-graph replays (calls chained with programmatic dependent launch), CUDA events",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         },
