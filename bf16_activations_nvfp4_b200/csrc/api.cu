@@ -340,13 +340,17 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
   } else {
     int rc = FI_ERR_UNSUPPORTED_SHAPE;
     // the automatic pipeline at m = 1 with a K split: each warp's share of a split is short, and
-    // more weight bytes per warp item pay. Where k % 256 != 0 the register pipeline (two CTAs
-    // per SM unless asked otherwise), else the stream pipeline with four rows per item. Measured
-    // on B200 at S in {2, 4, 8} on the five serving shapes: 3-22% less time per call than two
-    // rows per stream item, never more than 1% slower. Same bits: only the pipeline changes.
-    if (pipe_auto && m == 1 && S > 1 && rsel == 0) {
-      rc = (k % 256 != 0) ? geometry_for(kPipeReg, m, n, k, S, 0, ctas ? ctas : 2, sms, &g)
-                          : geometry_for(kPipeStream, m, n, k, S, 4, ctas, sms, &g);
+    // more weight bytes per warp item pay. Where k % 256 != 0 the register pipeline (two rows,
+    // two CTAs per SM unless asked otherwise), else the stream pipeline with four rows per item;
+    // only where those row groups, over all splits, still give every SM at least 4 warps (as on
+    // the serving shapes, n >= 2048, that the measurement covers). Measured on B200 at S in
+    // {2, 4, 8}: 3-22% less time per call than two rows per stream item, never more than 1%
+    // slower. Same bits: only the pipeline changes.
+    const bool reg_rule = k % 256 != 0;
+    const int64_t rule_warps = (n + (reg_rule ? 1 : 3)) / (reg_rule ? 2 : 4) * S;
+    if (pipe_auto && m == 1 && S > 1 && rsel == 0 && rule_warps >= 4 * (int64_t)sms) {
+      rc = reg_rule ? geometry_for(kPipeReg, m, n, k, S, 0, ctas ? ctas : 2, sms, &g)
+                    : geometry_for(kPipeStream, m, n, k, S, 4, ctas, sms, &g);
       if (rc != FI_OK) clear_error();
     }
     if (rc != FI_OK) rc = geometry_for(pipe, m, n, k, S, rsel, ctas, sms, &g);

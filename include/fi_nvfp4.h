@@ -75,7 +75,8 @@ typedef enum {
  *                power of two; 0 = automatic); high nibble = pipeline (0 = automatic:
  *                1, or 2 where the activations do not fit a half SM; at m = 1 with S > 1
  *                and automatic rows, 4 with two CTAs per SM where k % 256 != 0, else 1 with
- *                4 rows per item; 1 = per-warp
+ *                4 rows per item, where those row groups still give every SM 4 warps;
+ *                1 = per-warp
  *                asynchronous copies, 2 = producer-warp ring, 3 = per-warp
  *                copies in one half-SM CTA per SM, so that consecutive calls overlap, with
  *                an L2 prefetch of weights up to 40 MB; its CTAs-per-SM field is ignored;

@@ -278,6 +278,12 @@ def test_automatic_pipeline_for_split_calls_at_m1():
         s1 = fi.resolve_tactic(1, n, k, fi.make_tactic(fi.KIND_GEMV, 0, 0, 0), B200_SMS)["splits"]
         s4 = fi.resolve_tactic(4, n, k, fi.make_tactic(fi.KIND_GEMV, 0, 0, 0), B200_SMS)["splits"]
         assert s1 == s4
+    # where those row groups would leave SMs with fewer than 4 warps, the stream pipeline keeps
+    # its own row choice (n = 300: 75 four-row groups per split)
+    for S in (2, 4):
+        info = fi.resolve_tactic(1, 300, 4096, fi.make_tactic(fi.KIND_GEMV, S, 0, 0), B200_SMS)
+        assert info["variant"] >> 4 == 1 and info["variant"] & 15 != 4
+    assert fi.resolve_tactic(1, 129, 2688, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0), B200_SMS)["variant"] >> 4 == 1
     # explicit rows or pipeline are taken as given
     assert fi.resolve_tactic(1, 4096, 14336, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0x12), B200_SMS)["variant"] == 0x12
     assert fi.resolve_tactic(1, 4096, 14336, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0x01), B200_SMS)["variant"] & 15 == 1

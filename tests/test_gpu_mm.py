@@ -171,6 +171,23 @@ def test_pipelines_give_identical_bits():
                 assert np.array_equal(stream, other), (m, n, k, S, hex(var))
 
 
+@pytest.mark.parametrize("n,k", [(1000, 2688), (777, 1056), (300, 4096), (2048, 7168)])
+def test_automatic_pipeline_of_split_calls_at_m1(n, k):
+    """At m = 1 with S > 1 the automatic pipeline may be the register pipeline with two CTAs
+    per SM (k % 256 != 0) or the stream pipeline with four rows per item: within tolerance of
+    the oracle and bitwise equal to the stream pipeline with two rows per item at the same S."""
+    A = inputs.activations(1, k, seed=31, outliers=True)
+    W, (Wq, Ws, g) = _gpu.weights(n, k, 4, True)
+    ref = oracle.mm(A, Wq, Ws, g)
+    dw = _gpu.device_weights(n, k, 4, True)
+    for S in (2, 3, 8, 0):
+        t = fi.make_tactic(GEMV, S, 0, 0)
+        auto = _mm(A, dw, t)
+        _gpu.assert_within_tolerance(auto, ref, f"n={n} k={k} S={S}")
+        S_res = fi.resolve_tactic(1, n, k, t)["splits"]
+        assert np.array_equal(auto, _mm(A, dw, fi.make_tactic(GEMV, S_res, 0, 0x12))), (n, k, S)
+
+
 def test_multi_slab_rows_and_many_splits():
     """k = 65536 needs several ring stages per row (slabs); narrow n and ragged shapes."""
     for m, n, k, S in [(1, 8, 65536, 1), (2, 33, 16384, 5), (3, 17, 32768, 2)]:
