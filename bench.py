@@ -399,7 +399,7 @@ def run_fi(args, rank: int, world: int) -> dict | None:
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 x e2m1 (f16 half-block sums, f32 accumulate)",
+        "dtype": "bf16 x e2m1 (exact products, f32 accumulate)",
         "data": "synthetic",
         "config": {
             "workload": "serving-class decode GEMV, m=1, n x k in " + ", ".join(f"{n}x{k}" for n, k in SHAPES),

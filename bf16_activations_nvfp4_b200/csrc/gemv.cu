@@ -31,16 +31,12 @@
 //  * Arithmetic (fixed by k and S alone, hence bitwise identical for every m, pipeline, rows
 //    per group, CTA shape and grid): A is staged as f16 with one power-of-two scale sf_a per
 //    16-block that puts the block maximum in [2^9, 2^10) (exact for every element within 2^26
-//    of its block maximum); codes are decoded by cvt.rn.f16x2.e2m1x2 (exact). Per 16-block,
-//    packed f16 fused multiply-adds sum the even and the odd elements' products in element
-//    order (8 steps each, partial sums below 2^16); the two half sums times the block's E4M3
-//    scale go to fp32 through the mixed-precision fma.rn.f32.f16, and acc = fma(t, sf_a, acc).
-//    Lane L takes chunks L, L+32, L+64, ... of the split; the lanes combine through a fixed xor
-//    butterfly (all lanes end with the same bits). S == 1 writes bf16_rn(acc * gscale); S > 1
-//    writes fp32 partials for the reduce kernel. The f16 half sums are what make the inner loop
-//    cheap on sm_100: the packed f16 FMA issues to the other FMA port than the e2m1 conversion,
-//    so decode and products run side by side; their rounding (one f16 rounding per step on
-//    magnitudes below 2^16) stays far below the bf16 output's own.
+//    of its block maximum); codes are decoded by cvt.rn.f16x2.e2m1x2 (exact). Per 16-block, the
+//    16 products (each exact in fp32) are summed in fp32 in element order by the
+//    mixed-precision fma.rn.f32.f16, and acc = fma(t, sw * sf_a, acc) with sw the block's E4M3
+//    scale. Lane L takes chunks L, L+32, L+64, ... of the split; the lanes combine through a
+//    fixed xor butterfly (all lanes end with the same bits). S == 1 writes bf16_rn(acc *
+//    gscale); S > 1 writes fp32 partials for the reduce kernel.
 //  * Bounded waits (ring pipeline). Every mbarrier wait gives up after a time limit
 //    (%globaltimer): it sets a device error flag and a CTA-wide abort flag, the CTA finishes
 //    its control flow without computing, and the producer waits (bounded) for the copies it
@@ -159,48 +155,36 @@ __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A
   }
 }
 
-// The 8 f16 pairs of one 16-block multiplied lane-wise and summed in element order in packed
-// f16: the low half sums the block's even elements, the high half its odd ones, one fused
-// multiply-add (one rounding) per step. The activations are staged below 2^10 and |e2m1| <= 6,
-// so every partial sum stays below 8 * 6 * 2^10 < 2^16: no overflow.
-__device__ __forceinline__ uint32_t hdot8(const uint32_t* a, const uint32_t* w) {
-  uint32_t h;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h) : "r"(a[0]), "r"(w[0]));
-#pragma unroll
-  for (int i = 1; i < 8; ++i) asm("fma.rn.f16x2 %0, %1, %2, %0;" : "+r"(h) : "r"(a[i]), "r"(w[i]));
-  return h;
-}
-
-// acc + (h.lo * sw + h.hi * sw) * sa for one 16-block: its two f16 half sums times the block's
-// E4M3 weight scale sw (an f16: the low half of sh for HALF 0, the high half for HALF 1) in
-// fp32 (the first product exact, the second added with one rounding), then times the
-// activation block's power-of-two scale sa and added to acc (one rounding).
-template <int HALF>
-__device__ __forceinline__ float block_acc(uint32_t h, uint32_t sh, float sa, float acc) {
+// The 16 products of one 16-block summed in fp32, in element order: a and w hold the block's
+// 8 f16 pairs (element 2j in the low half of word j). Each product of two f16 values is exact
+// in fp32, and the mixed-precision fma.rn.f32.f16 adds it to the running fp32 sum with one
+// round-to-nearest-even, so this is the block's dot product accumulated in fp32.
+__device__ __forceinline__ float block_dot(const uint32_t* a, const uint32_t* w) {
   float t;
-  if constexpr (HALF == 0) {
-    asm("{\n .reg .b16 hl, hh, sl, su;\n mov.b32 {hl, hh}, %1;\n mov.b32 {sl, su}, %2;\n"
-        " fma.rn.f32.f16 %0, hl, sl, 0f00000000;\n fma.rn.f32.f16 %0, hh, sl, %0;\n}"
-        : "=f"(t)
-        : "r"(h), "r"(sh));
-  } else {
-    asm("{\n .reg .b16 hl, hh, sl, su;\n mov.b32 {hl, hh}, %1;\n mov.b32 {sl, su}, %2;\n"
-        " fma.rn.f32.f16 %0, hl, su, 0f00000000;\n fma.rn.f32.f16 %0, hh, su, %0;\n}"
-        : "=f"(t)
-        : "r"(h), "r"(sh));
-  }
-  return fmaf(t, sa, acc);
+  asm("{\n .reg .b16 al, ah, wl, wh;\n mov.b32 {al, ah}, %1;\n mov.b32 {wl, wh}, %2;\n"
+      " fma.rn.f32.f16 %0, al, wl, 0f00000000;\n fma.rn.f32.f16 %0, ah, wh, %0;\n}"
+      : "=f"(t)
+      : "r"(a[0]), "r"(w[0]));
+#pragma unroll
+  for (int i = 1; i < 8; ++i)
+    asm("{\n .reg .b16 al, ah, wl, wh;\n mov.b32 {al, ah}, %1;\n mov.b32 {wl, wh}, %2;\n"
+        " fma.rn.f32.f16 %0, al, wl, %0;\n fma.rn.f32.f16 %0, ah, wh, %0;\n}"
+        : "+f"(t)
+        : "r"(a[i]), "r"(w[i]));
+  return t;
 }
 
 // One 32-k chunk of one weight row against one activation row: av the chunk's 16 staged f16
-// pairs, sa its two block scales, wf the decoded codes, sh the two E4M3 block scales as f16x2.
-// Every pipeline calls this, so their bits agree.
+// pairs, sa its two activation block scales (powers of two), wf the decoded codes, sh the two
+// E4M3 block scales as f16x2. Per block, acc = fma(t, sw * sa, acc) with t the block's fp32 dot
+// product (sw * sa is exact: sa is a power of two). Every pipeline calls this, so their bits
+// agree.
 __device__ __forceinline__ float chunk_acc(const uint32_t (&av)[16], float2 sa, const uint32_t (&wf)[16], uint32_t sh,
                                            float acc) {
-  const uint32_t h0 = hdot8(av, wf);
-  const uint32_t h1 = hdot8(av + 8, wf + 8);
-  acc = block_acc<0>(h0, sh, sa.x, acc);
-  return block_acc<1>(h1, sh, sa.y, acc);
+  const float t0 = block_dot(av, wf);
+  const float t1 = block_dot(av + 8, wf + 8);
+  acc = fmaf(t0, __fmul_rn(f16_lo_to_f32(sh), sa.x), acc);
+  return fmaf(t1, __fmul_rn(f16_hi_to_f32(sh), sa.y), acc);
 }
 
 // Decode one 16-byte code quad (32 E2M1 codes) into 16 f16x2 words.

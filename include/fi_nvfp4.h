@@ -83,10 +83,11 @@ typedef enum {
  *                4 = weights loaded straight to registers, 1 or 2 rows per warp). MMA: 0.
  * Only `kind` and the resolved S change the arithmetic: two tactics with the same kind
  * and S give bitwise identical outputs (whatever their pipeline, rows or CTAs), and for a
- * fixed tactic every output row is bitwise independent of m. GEMV and MMA results differ
- * in their last bits: the MMA forms exact f16 products and accumulates in fp32; the GEMV sums
- * the even and the odd elements of each 16-block in f16 (8 fused steps each, every partial
- * below 2^16) before fp32 accumulation; both errors stay below the bf16 output's rounding.
+ * fixed tactic every output row is bitwise independent of m. Both kinds form every product
+ * exactly and accumulate in fp32; GEMV and MMA results differ in their last bits because
+ * they group and order the fp32 additions differently (the GEMV sums each 16-block's products
+ * in element order, then adds the block sum times its scale; the MMA accumulates 64-k steps
+ * of pre-scaled weights in the tensor core).
  * FI_TACTIC_DEFAULT (-1) selects from the built-in per-shape
  * table (PR #4038, Description, "What it does": the untuned m=1 route to the GEMV); the
  * table's choice of kind and S depends on m, so the default is batch-invariant only
@@ -135,8 +136,8 @@ FI_API int fi_nvfp4_pack_weights(const float* W, int64_t n, int64_t k, uint8_t* 
                           uint8_t* Wscale, float* gscale, fi_stream_t stream);
 
 /*
- * out[m, n] = bf16_rn(gscale * sum_k A[m, k] * e2m1(Wq) * e4m3(Wscale)), fp32 accumulation of
- * the per-block sums (see the tactic notes above for the arithmetic inside a block)
+ * out[m, n] = bf16_rn(gscale * sum_k A[m, k] * e2m1(Wq) * e4m3(Wscale)), with exact products
+ * and fp32 accumulation (see the tactic notes above for the order of the additions)
  * (PR #4038, Description).
  *   A       device bf16 bits [m, k], 16-byte aligned.
  *   Wq, Wscale, gscale  NVFP4 weights as produced by fi_nvfp4_pack_weights; Wq and Wscale
