@@ -57,6 +57,8 @@ def _load():
         lib.orc_e4m3_encode.restype = ctypes.c_uint32
         lib.orc_e2m1_encode.argtypes = [ctypes.c_float]
         lib.orc_e2m1_encode.restype = ctypes.c_uint32
+        lib.orc_f32_to_f16.argtypes = [ctypes.c_float]
+        lib.orc_f32_to_f16.restype = ctypes.c_uint16
         lib.orc_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.orc_f32_to_bf16.restype = ctypes.c_uint16
         lib.orc_global_scale.argtypes = [f32p, i64]
@@ -67,7 +69,7 @@ def _load():
         lib.orc_dequant_row.restype = None
         lib.orc_mm.argtypes = [u16p, u8p, u8p, ctypes.c_float, i64, i64, i64, i64p, i64, f64p]
         lib.orc_mm.restype = ctypes.c_int
-        lib.orc_splitk_reduce.argtypes = [f32p, i64, i64, ctypes.c_float, u16p]
+        lib.orc_splitk_reduce.argtypes = [f32p, i64, i64, ctypes.c_float, ctypes.c_int, u16p]
         lib.orc_splitk_reduce.restype = None
         lib.orc_num_threads.argtypes = []
         lib.orc_num_threads.restype = ctypes.c_int
@@ -107,6 +109,18 @@ def e2m1_encode(x: float) -> int:
 def f32_to_bf16_bits(x: float) -> int:
     """fp32 -> bf16 bit pattern, round to nearest even."""
     return _load().orc_f32_to_bf16(float(np.float32(x)))
+
+
+def f32_to_f16_bits(x: float) -> int:
+    """fp32 -> IEEE binary16 bit pattern, round to nearest even, overflow to +-inf."""
+    return _load().orc_f32_to_f16(float(np.float32(x)))
+
+
+def round_out(v: np.ndarray, out_dtype: str = "bf16") -> np.ndarray:
+    """fp32 values -> output bits (uint16) of out_dtype ("bf16" or "f16"), round to nearest even."""
+    f = f32_to_f16_bits if out_dtype == "f16" else f32_to_bf16_bits
+    v = np.asarray(v, np.float32)
+    return np.array([f(x) for x in v.ravel()], np.uint16).reshape(v.shape)
 
 
 # ---------------------------------------------------------------------- quantise
@@ -181,17 +195,20 @@ def mm(A_bits: np.ndarray, Wq: np.ndarray, Wscale: np.ndarray, gscale, cols=None
     return ref
 
 
-def splitk_reduce(partials: np.ndarray, gscale) -> np.ndarray:
-    """bf16 bits of bf16_rn(gscale * (((p0 + p1) + p2) + ...)), all in fp32.
+def splitk_reduce(partials: np.ndarray, gscale, out_dtype: str = "bf16") -> np.ndarray:
+    """Bits of round(gscale * (((p0 + p1) + p2) + ...)), all in fp32, rounded to nearest even
+    into out_dtype ("bf16", or "f16" for the optional fp16 output).
 
     partials is float32 [S, m, n]; returns uint16 [m, n].
     """
+    if out_dtype not in ("bf16", "f16"):
+        raise ValueError("out_dtype must be 'bf16' or 'f16'")
     partials = np.ascontiguousarray(partials, dtype=np.float32)
     S = partials.shape[0]
     mn = partials[0].size
     out = np.zeros(partials.shape[1:], np.uint16)
     _load().orc_splitk_reduce(_ptr(partials, ctypes.c_float), S, mn, float(np.float32(gscale)),
-                              _ptr(out, ctypes.c_uint16))
+                              1 if out_dtype == "f16" else 0, _ptr(out, ctypes.c_uint16))
     return out
 
 

@@ -116,6 +116,33 @@ uint16_t orc_f32_to_bf16(float f) {
   return (uint16_t)((u + 0x7fffu + lsb) >> 16);
 }
 
+/* fp32 -> IEEE binary16 bits, round to nearest, ties to even (the optional f16 output of
+ * PR #4038's commit covering fp16 output through the GEMV path). Written from the format
+ * definition: the quantum of x's binade is 2^(e-10) for normal results (e >= -14) and 2^-24
+ * below; x / quantum is exact in double, nearbyint rounds it half-to-even (the oracle is built
+ * with the default rounding mode), and a result of 65536 or more is an overflow to +-inf. */
+uint16_t orc_f32_to_f16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  const uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)(sign | 0x7e00u); /* NaN */
+  const double x = fabs((double)f);
+  if (x == 0.0) return sign;
+  if (isinf(x)) return (uint16_t)(sign | 0x7c00u);
+  int e2 = 0;
+  frexp(x, &e2);           /* x = mant * 2^e2, mant in [0.5, 1): floor(log2 x) = e2 - 1 */
+  int e = e2 - 1;
+  const double q = e < -14 ? ldexp(1.0, -24) : ldexp(1.0, e - 10);
+  const double nq = nearbyint(x / q);
+  const double v = nq * q;
+  if (v >= 65536.0) return (uint16_t)(sign | 0x7c00u);
+  if (v < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)(v / ldexp(1.0, -24))); /* subnormal */
+  frexp(v, &e2);
+  e = e2 - 1;              /* the rounded value may have moved up one binade */
+  const uint32_t mant = (uint32_t)(v / ldexp(1.0, e - 10)) - 1024u;
+  return (uint16_t)(sign | (uint32_t)(e + 15) << 10 | mant);
+}
+
 /* --------------------------------------------------------------------- quantise */
 
 /* Global scale: one fp32 division of the tensor amax by 448 * 6 = 2688 (exact in fp32). */
@@ -217,15 +244,16 @@ int orc_mm(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, float gs
 /* ------------------------------------------------------------ split-K reduce */
 
 /* The fixed-order split-K reduction as a plain definition: for each output element,
- * s = ((p_0 + p_1) + p_2) + ... in fp32, then out = bf16_rn(s * gscale) with the
- * product in fp32. partials is [S, m*n] fp32, out is bf16 bits [m*n]. */
-void orc_splitk_reduce(const float* partials, int64_t S, int64_t mn, float gscale,
+ * s = ((p_0 + p_1) + p_2) + ... in fp32, then out = bf16_rn(s * gscale) (f16 == 0) or
+ * f16_rn(s * gscale) (f16 != 0) with the product in fp32. partials is [S, m*n] fp32, out is
+ * the output's bits [m*n]. */
+void orc_splitk_reduce(const float* partials, int64_t S, int64_t mn, float gscale, int f16,
                        uint16_t* out) {
   for (int64_t e = 0; e < mn; ++e) {
     float s = partials[e];
     for (int64_t p = 1; p < S; ++p) s = s + partials[p * mn + e];
     const float v = s * gscale;
-    out[e] = orc_f32_to_bf16(v);
+    out[e] = f16 ? orc_f32_to_f16(v) : orc_f32_to_bf16(v);
   }
 }
 

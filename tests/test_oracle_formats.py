@@ -141,3 +141,56 @@ def test_bf16_rounding_matches_torch():
     ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     got = np.array([oracle.f32_to_bf16_bits(float(v)) for v in x], np.uint16)
     assert np.array_equal(got, ref)
+
+
+def _f16_table():
+    """Every finite IEEE binary16 value (as float64) with its bit pattern, decoded from the format
+    definition: sign, 5-bit exponent (bias 15), 10-bit mantissa; exponent 0 is subnormal."""
+    bits = np.arange(0, 0x7c00, dtype=np.uint32)
+    e = (bits >> 10) & 0x1f
+    m = bits & 0x3ff
+    val = np.where(e == 0, m * 2.0 ** -24, (1024 + m) * 2.0 ** (e.astype(np.int64) - 25))
+    return val, bits
+
+
+def test_f16_rounding_matches_torch_and_overflows_to_inf():
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal(50000) * np.exp2(rng.integers(-30, 18, 50000))).astype(np.float32)
+    edge = np.array([65504, 65519.99, 65520, 65536, 1e30, -1e30, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26,
+                     2.0 ** -14 - 2.0 ** -25, 0.0, -0.0, np.inf, -np.inf], np.float32)
+    x = np.concatenate([x, edge])
+    got = oracle.round_out(x, "f16")
+    want = torch.from_numpy(x).to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+    assert oracle.f32_to_f16_bits(65520.0) == 0x7c00 and oracle.f32_to_f16_bits(-65520.0) == 0xfc00
+    assert oracle.f32_to_f16_bits(65519.0) == 0x7bff
+
+
+def test_f16_rounding_is_the_nearest_value_ties_to_even_by_brute_force():
+    """Argmin over all finite f16 values (ties to the even mantissa) on random fp32 inputs and on
+    every exact midpoint between neighbouring f16 values below 2^-10, plus a sample above."""
+    val, bits = _f16_table()
+    rng = np.random.default_rng(6)
+    x = np.abs(rng.standard_normal(3000) * np.exp2(rng.integers(-26, 15, 3000))).astype(np.float32)
+    mids = ((val[:-1] + val[1:]) / 2)
+    x = np.concatenate([x, mids[val[1:] < 2.0 ** -10].astype(np.float32), mids[::97].astype(np.float32)])
+    x = x[x.astype(np.float64) < 65504.0]  # finite results only; overflow is pinned above
+    for v in x:
+        d = np.abs(val - float(v))
+        cand = np.flatnonzero(d == d.min())
+        best = cand[0] if len(cand) == 1 else cand[(bits[cand] & 1) == 0][0]
+        assert oracle.f32_to_f16_bits(float(v)) == bits[best], (float(v), hex(bits[best]))
+        assert oracle.f32_to_f16_bits(-float(v)) == (bits[best] | 0x8000 if val[best] != 0 else 0x8000)
+
+
+def test_splitk_reduce_f16_output_definition():
+    """out = f16_rn(((p0 + p1) + p2) * g), the fp32 sum in split order: 2^24 + 1 - 2^24 in that
+    order is 0, a product past 65520 is +inf, and a representable result is exact."""
+    p = np.array([[[2.0 ** 24, 3.0, 1.0, 65000.0]], [[1.0, 5.0, 2.0, 500.0]],
+                  [[-(2.0 ** 24), 0.5, 65503.0, 20.0]]], np.float32)
+    got = oracle.splitk_reduce(p, np.float32(1.0), "f16")
+    assert got[0, 0] == 0x0000  # (2^24 + 1) rounds to 2^24 in fp32, minus 2^24 = 0
+    assert got[0, 1] == 0x4840  # 8.5 = 1.0625 * 2^3
+    assert got[0, 2] == 0x7bff  # 65506 < 65520: rounds to 65504, the largest finite f16
+    assert got[0, 3] == 0x7c00  # 65520 and above: +inf
+    assert np.array_equal(oracle.splitk_reduce(p, np.float32(1.0)), oracle.splitk_reduce(p, np.float32(1.0), "bf16"))
