@@ -386,7 +386,10 @@ def run_fi(args, rank: int, world: int) -> dict | None:
     keys = [key(c["shape"]) for c in on]
     if NCU_TRAFFIC["source_sha256"] == _gemv_source_sha() and all(k_ in NCU_TRAFFIC["bytes"] for k_ in keys):
         traffic = round(statistics.fmean(NCU_TRAFFIC["bytes"][k_] for k_ in keys))
-    roof_kernel = "gemv_stream_kernel, split 1, one launch per call, on " + ", ".join(sorted(set(keys)))
+    kernels = {1: "gemv_stream_kernel", 2: "gemv_nvfp4_kernel", 3: "gemv_stream_kernel", 4: "gemv_reg_kernel",
+               5: "gemv_lean_kernel"}
+    roof_names = sorted({kernels.get(c["info"]["variant"] >> 4, "gemv") for c in on})
+    roof_kernel = "/".join(roof_names) + ", split 1, one launch per call, on " + ", ".join(sorted(set(keys)))
     def_bytes = sum(shapes[d["shape"]]["bytes"] for d in defaults)
     return {
         "metric": METRIC,
@@ -433,8 +436,9 @@ def run_fi(args, rank: int, world: int) -> dict | None:
 
 def run_extra_shapes(dev, stream, peaks) -> dict:
     """Default-tactic µs per call, cold L2 (each call reads its own weight copy, copies >= 300
-    MB per shape), PDL-chained graph replays: the narrow-n decode grid at m = 1 and the
-    small-batch sweep of 4096 x 14336 at m in {1, 2, 4, 8, 16, 32}."""
+    MB per shape), PDL-chained graph replays: the narrow-n decode grid at m = 1, the
+    small-batch sweep of 4096 x 14336 at m in {1, 2, 4, 8, 16, 32}, and the second workload,
+    the Qwen3.6-27B-shaped decode GEMMs at m = 1 (34816 x 5120, 5120 x 17408, 248320 x 5120)."""
     import torch
 
     import bf16_activations_nvfp4_b200 as fi
@@ -477,7 +481,8 @@ def run_extra_shapes(dev, stream, peaks) -> dict:
 
     narrow = [time_case(1, n, k) for n, k in inputs.NARROW_N]
     small = [time_case(m, *inputs.SMALL_BATCH_NK) for m in inputs.SMALL_BATCH_M]
-    return {"narrow_n": narrow, "small_batch": small,
+    qwen = [time_case(1, n, k) for n, k in inputs.QWEN36_27B_DECODE]
+    return {"narrow_n": narrow, "small_batch": small, "qwen36_27b_m1": qwen,
             "method": "default tactic, PDL-chained CUDA-graph replays over >= 300 MB of weight copies (cold L2)"}
 
 
@@ -571,21 +576,55 @@ def _oracle_packed():
     return packed
 
 
+def _host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def oracle_sample(target_s: float) -> dict:
-    """Time the CPU oracle's product (dequantise + fp64 dot) on the same five shapes."""
+    """The CPU oracle on the same five m = 1 shapes, once with 1 thread and once with every
+    host core (os.sched_getaffinity), pack (fp32 quantiser) and matmul (fp64 dequantise + dot)
+    timed separately per shape. `value` is the all-cores matmul rate in the metric's unit (GB/s
+    of algorithmic bytes); passes repeat until about target_s seconds of matmul time per thread
+    count, each shape's pack is timed once per thread count."""
     import oracle
-    packed = _oracle_packed()
-    reps, elapsed, nbytes = 0, 0.0, 0
-    while elapsed < target_s and reps < 200:
-        for A, Wq, Ws, g, b in packed:
+    from bf16_activations_nvfp4_b200 import inputs
+    cores = _host_cores()
+    data = [(n, k, inputs.weights(n, k, seed=0), inputs.activations(M, k, seed=0), algorithmic_bytes(M, n, k))
+            for n, k in SHAPES]
+    per_shape = {f"{n}x{k}": {"n": n, "k": k} for n, k, *_ in data}
+    rates = {}
+    for label, threads in (("1_thread", 1), ("all_cores", cores)):
+        oracle.set_num_threads(threads)
+        packed = []
+        for n, k, W, A, b in data:
             t0 = time.perf_counter()
-            oracle.mm(A, Wq, Ws, g)
-            elapsed += time.perf_counter() - t0
-            nbytes += b
-        reps += 1
-    return {"value": round(nbytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle", "reps": reps, "seconds": round(elapsed, 2),
-            "sample": f"{reps} full passes over the five m=1 products (pack excluded)"}
+            Wq, Ws, g = oracle.pack(W)
+            per_shape[f"{n}x{k}"][f"pack_ms_{label}"] = round((time.perf_counter() - t0) * 1e3, 2)
+            packed.append((n, k, A, Wq, Ws, g, b))
+        reps, elapsed, nbytes = 0, 0.0, 0
+        mm_s = {f"{n}x{k}": [] for n, k, *_ in data}
+        while elapsed < target_s / 2 and reps < 200:
+            for n, k, A, Wq, Ws, g, b in packed:
+                t0 = time.perf_counter()
+                oracle.mm(A, Wq, Ws, g)
+                dt = time.perf_counter() - t0
+                mm_s[f"{n}x{k}"].append(dt)
+                elapsed += dt
+                nbytes += b
+            reps += 1
+        for key, ts in mm_s.items():
+            per_shape[key][f"matmul_ms_{label}"] = round(statistics.median(ts) * 1e3, 3)
+        rates[label] = {"value": round(nbytes / elapsed / 1e9, 4), "unit": "GB/s", "threads": threads,
+                        "reps": reps, "matmul_seconds": round(elapsed, 2)}
+    oracle.set_num_threads(cores)
+    return {"value": rates["all_cores"]["value"], "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "one_thread": rates["1_thread"], "all_cores": rates["all_cores"],
+            "per_shape": list(per_shape.values()),
+            "sample": f"{rates['all_cores']['reps']} full passes over the five m=1 products at {cores} threads "
+                      f"({rates['1_thread']['reps']} at 1 thread); pack timed once per shape and thread count"}
 
 
 REFERENCE_BUDGET_S = 120.0  # whole --impl reference run, all steps

@@ -31,6 +31,8 @@ _LIB_NAME = "libfi_nvfp4.so"
 KIND_GEMV = 0
 KIND_MMA = 1
 TACTIC_DEFAULT = -1
+# output element types of fi_mm_bf16_fp4_out / fi_splitk_reduce_out
+_DTYPES = {torch.bfloat16: 0, torch.float16: 1}
 
 _STATUS = {0: "FI_OK", -1: "FI_ERR_INVALID_ARG", -2: "FI_ERR_UNSUPPORTED_SHAPE",
            -3: "FI_ERR_UNSUPPORTED_ARCH", -4: "FI_ERR_WORKSPACE", -5: "FI_ERR_CUDA"}
@@ -84,6 +86,8 @@ def library() -> ctypes.CDLL:
         lib.fi_mm_bf16_fp4_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp]
         lib.fi_mm_bf16_fp4_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
         lib.fi_splitk_reduce.argtypes = [vp, i64, i64, i64, vp, vp, vp]
+        lib.fi_mm_bf16_fp4_out.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i64, vp, sz, vp]
+        lib.fi_splitk_reduce_out.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_int, vp]
         lib.fi_resolve_tactic.argtypes = [i64, i64, i64, i64, ctypes.c_int, ctypes.POINTER(TacticInfo)]
         lib.fi_default_tactic.argtypes = [i64, i64, i64, ctypes.c_int]
         lib.fi_default_tactic.restype = i64
@@ -97,7 +101,7 @@ def library() -> ctypes.CDLL:
         lib.fi_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         lib.fi_debug_set.argtypes = [ctypes.c_int, i64]
         for name in ("fi_nvfp4_pack_weights", "fi_mm_bf16_fp4", "fi_mm_bf16_fp4_ex", "fi_mm_bf16_fp4_noalloc",
-                     "fi_splitk_reduce",
+                     "fi_splitk_reduce", "fi_mm_bf16_fp4_out", "fi_splitk_reduce_out",
                      "fi_resolve_tactic", "fi_list_tactics", "fi_set_workspace", "fi_version",
                      "fi_get_device_error", "fi_debug_set"):
             getattr(lib, name).restype = ctypes.c_int
@@ -256,34 +260,51 @@ def pack_weights(W: torch.Tensor, out: tuple | None = None):
     return Wq, Ws, g
 
 
+def _out_dtype(out: torch.Tensor | None, out_dtype: torch.dtype | None) -> torch.dtype:
+    dtype = out.dtype if out is not None else (out_dtype or torch.bfloat16)
+    if dtype not in _DTYPES or (out_dtype is not None and out_dtype != dtype):
+        raise ValueError(f"the output is bf16 or f16 (out_dtype {out_dtype}, out {None if out is None else out.dtype})")
+    return dtype
+
+
 def mm_bf16_fp4(A: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor, gscale: torch.Tensor,
                 tactic: int = TACTIC_DEFAULT, out: torch.Tensor | None = None,
-                workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """out[m, n] = A[m, k] . dequant(W)^T, bf16 out (CUDA tensors on one device).
+                workspace: torch.Tensor | None = None, out_dtype: torch.dtype | None = None) -> torch.Tensor:
+    """out[m, n] = A[m, k] . dequant(W)^T (CUDA tensors on one device), bf16 out unless
+    out_dtype (or the dtype of `out`) is torch.float16.
 
     `workspace` (optional CUDA tensor) is passed to fi_mm_bf16_fp4_ex; without it the call
-    uses the per-device workspace of fi_mm_bf16_fp4.
+    uses the per-device workspace of fi_mm_bf16_fp4. An f16 output goes through
+    fi_mm_bf16_fp4_out.
     """
     _require(A, "A", torch.bfloat16, 2)
     _require(Wq, "Wq", torch.uint8, 2)
     _require(Wscale, "Wscale", torch.uint8, 2)
     _require(gscale, "gscale", torch.float32, 1)
+    dtype = _out_dtype(out, out_dtype)
     if out is not None:
-        _require(out, "out", torch.bfloat16, 2)
+        _require(out, "out", dtype, 2)
     if workspace is not None:
         if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda or not workspace.is_contiguous():
             raise ValueError("workspace must be a contiguous CUDA tensor")
         _same_device(A, workspace=workspace)
     m, n, k = _mm_shapes(A, Wq, Wscale, gscale, out)
     if out is None:
-        out = torch.empty((m, n), dtype=torch.bfloat16, device=A.device)
+        out = torch.empty((m, n), dtype=dtype, device=A.device)
     lib = library()
     dev = A.device
     # the library works on the current device: switch only when A lives on another one
     ctx = torch.cuda.device(dev) if dev.index != torch.cuda.current_device() else contextlib.nullcontext()
     with ctx:
         s = torch.cuda.current_stream(dev).cuda_stream
-        if workspace is None:
+        if dtype != torch.bfloat16:
+            ws_ptr, ws_bytes = (0, 0) if workspace is None else (workspace.data_ptr(),
+                                                                  workspace.numel() * workspace.element_size())
+            st = lib.fi_mm_bf16_fp4_out(A.data_ptr(), Wq.data_ptr(), Wscale.data_ptr(), gscale.data_ptr(),
+                                        out.data_ptr(), _DTYPES[dtype], m, n, k, tactic, ws_ptr or None, ws_bytes, s)
+            if st:
+                _check(st, "fi_mm_bf16_fp4_out")
+        elif workspace is None:
             st = lib.fi_mm_bf16_fp4(A.data_ptr(), Wq.data_ptr(), Wscale.data_ptr(), gscale.data_ptr(),
                                     out.data_ptr(), m, n, k, tactic, s)
             if st:
@@ -297,21 +318,24 @@ def mm_bf16_fp4(A: torch.Tensor, Wq: torch.Tensor, Wscale: torch.Tensor, gscale:
     return out
 
 
-def splitk_reduce(partials: torch.Tensor, gscale: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
-    """bf16_rn(gscale * fixed-order sum over dim 0) of fp32 partials [S, m, n]."""
+def splitk_reduce(partials: torch.Tensor, gscale: torch.Tensor, out: torch.Tensor | None = None,
+                  out_dtype: torch.dtype | None = None) -> torch.Tensor:
+    """round(gscale * fixed-order sum over dim 0) of fp32 partials [S, m, n] to bf16 (default)
+    or f16 (out_dtype, or the dtype of `out`)."""
     _require(partials, "partials", torch.float32, 3)
     _require(gscale, "gscale", torch.float32, 1)
     S, m, n = partials.shape
     if gscale.numel() != 1:
         raise ValueError(f"gscale must hold one element, got {gscale.numel()}")
+    dtype = _out_dtype(out, out_dtype)
     if out is None:
-        out = torch.empty((m, n), dtype=torch.bfloat16, device=partials.device)
+        out = torch.empty((m, n), dtype=dtype, device=partials.device)
     else:
-        _require(out, "out", torch.bfloat16, 2)
+        _require(out, "out", dtype, 2)
         if tuple(out.shape) != (m, n):
             raise ValueError(f"out must be [{m}, {n}], got {tuple(out.shape)}")
     _same_device(partials, gscale=gscale, out=out)
     with torch.cuda.device(partials.device):
-        _check(library().fi_splitk_reduce(partials.data_ptr(), S, m, n, gscale.data_ptr(), out.data_ptr(),
-                                          _stream(partials.device)), "fi_splitk_reduce")
+        _check(library().fi_splitk_reduce_out(partials.data_ptr(), S, m, n, gscale.data_ptr(), out.data_ptr(),
+                                              _DTYPES[dtype], _stream(partials.device)), "fi_splitk_reduce_out")
     return out

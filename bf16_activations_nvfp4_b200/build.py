@@ -37,7 +37,7 @@ def _nvcc() -> str:
 
 def _deps() -> list[str]:
     return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
-        glob.glob(os.path.join(INCLUDE, "*.h"))
+        glob.glob(os.path.join(CSRC, "*.inc")) + glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
 def _stale(target: str, sources: list[str]) -> bool:

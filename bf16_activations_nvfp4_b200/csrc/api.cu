@@ -245,9 +245,63 @@ static int gemv_reg_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, 
   return FI_OK;
 }
 
+// Lean stream pipeline (m = 1 only): the stream pipeline's CTA shapes and row groups, with
+// per-warp rings of NS slots of R rows x kLeanIters chunk iterations (codes and scales, 576
+// bytes per row and iteration); a row group's last item may hold a single iteration. Needs
+// k % 256 == 0 and every split a whole number of 32-chunk iterations ((k/32) % (32 S) == 0).
+static int gemv_lean_geometry(int64_t m, int64_t n, int64_t k, int S, int r_req, int ctas_per_sm, int sms,
+                              GemvGeometry* g) {
+  if (m != 1)
+    return set_error(FI_ERR_UNSUPPORTED_SHAPE, "GEMV lean pipeline: m = 1 only (got m=%lld)", (long long)m);
+  const int64_t C = k / kChunkK;
+  if (k % 256 != 0 || C % (32 * (int64_t)S) != 0)
+    return set_error(FI_ERR_UNSUPPORTED_SHAPE,
+                     "GEMV lean pipeline: needs k %% 256 == 0 and k/32 a multiple of 32 * splits (k=%lld, splits=%d)",
+                     (long long)k, S);
+  const int64_t nch = C / S;
+  const bool wide = stream_wide(n, sms);
+  const bool fill2 = (n + 1) / 2 >= (int64_t)sms * 2 * 4;
+  const int ctas = ctas_per_sm > 0 ? ctas_per_sm : (wide || fill2 ? 2 : 1);
+  if (ctas > 2) return set_error(FI_ERR_INVALID_ARG, "GEMV lean pipeline: at most 2 CTAs per SM");
+  int nw = ctas == 1 ? 16 : 8;
+  const int64_t budget = ctas == 1 ? kSmemBudget : kStreamHalfBudget;
+  const int64_t a_bytes = round_up(((nch + 31) / 32) * 2048, 128);
+  const int64_t as_bytes = round_up(nch * 8, 128);
+  int64_t r = r_req;
+  if (r == 0) r = ctas == 2 && wide ? 4 : 2;
+  if (r != 1 && r != 2 && r != 4)
+    return set_error(FI_ERR_INVALID_ARG, "GEMV lean pipeline: 1, 2 or 4 rows per item (got %lld)", (long long)r);
+  const int64_t slot = (int64_t)kLeanIters * r * 576;
+  const int64_t groups = (n + r - 1) / r;
+  const int64_t gx_cap = std::max<int64_t>(1, (int64_t)sms * ctas / S);
+  if ((groups + nw - 1) / nw < gx_cap) nw = (int)std::max<int64_t>(4, (groups + gx_cap - 1) / gx_cap);
+  const int64_t fixed = a_bytes + as_bytes;
+  int ns = 4;
+  if (fixed + (int64_t)nw * ns * slot > budget) ns = 2;
+  if (fixed + (int64_t)nw * ns * slot > budget)
+    return set_error(FI_ERR_UNSUPPORTED_SHAPE,
+                     "GEMV lean pipeline: %lld k per split leave no room for the weight slots; use more splits",
+                     (long long)(nch * kChunkK));
+  g->pipeline = kPipeLean;
+  g->threads = nw * 32;
+  g->S = S;
+  g->RS = (int)r;
+  g->stages = ns;
+  g->ctas_per_sm = ctas;
+  g->grid_x = (int)std::max<int64_t>(1, std::min<int64_t>(gx_cap, (groups + nw - 1) / nw));
+  g->grid_y = S;
+  g->stage_bytes = slot;
+  g->off_as = a_bytes;
+  g->off_bar = fixed;
+  g->off_ring = fixed;
+  g->smem_bytes = fixed + (int64_t)nw * ns * slot;
+  return FI_OK;
+}
+
 static int geometry_for(int pipe, int64_t m, int64_t n, int64_t k, int S, int r, int ctas, int sms, GemvGeometry* g) {
   if (pipe == kPipeRing) return gemv_geometry(m, n, k, S, r, ctas, sms, g);
   if (pipe == kPipeReg) return gemv_reg_geometry(m, n, k, S, r, ctas, sms, g);
+  if (pipe == kPipeLean) return gemv_lean_geometry(m, n, k, S, r, ctas, sms, g);
   return gemv_stream_geometry(m, n, k, S, r, ctas, sms, g, pipe == kPipeOverlap);
 }
 
@@ -258,7 +312,7 @@ static int gemv_knee(int pipe, int64_t n, int64_t k, int sms, int64_t m_fit, int
   const int64_t C = k / kChunkK;
   const int64_t maxS = std::max<int64_t>(1, std::min<int64_t>(C, 4095));
   for (int64_t S = 1; S <= maxS; ++S) {
-    GemvGeometry g;
+    GemvGeometry g{};
     if (geometry_for(pipe, m_fit, n, k, (int)S, rs, ctas, sms, &g) != FI_OK) continue;
     // enough: the splits' warps cover at least 40% of the SMs' warp slots (16 per SM; the ring
     // pipeline's CTAs always have 16 consumer warps). Measured on B200: idle warp slots cost
@@ -279,9 +333,28 @@ static int gemv_knee(int pipe, int64_t n, int64_t k, int sms, int64_t m_fit, int
 
 static int resolve(int64_t m, int64_t n, int64_t k, int64_t tactic, int num_sms, fi_tactic_info* out);
 
+// The measured table (generated by the package's cold-L2 tuner, tune.py): per (n, k, SM count)
+// and bucket of m, the tactic that was fastest on this GPU model. Shapes and devices it does not
+// list take the built-in rules below.
+struct TunedTactic {
+  int64_t n, k;
+  int32_t m_lo, m_hi, sms;
+  int64_t tactic;
+  double us;  // measured mean us per call (documentation only)
+};
+#include "tactic_table.inc"
+
+static int64_t tuned_tactic(int64_t m, int64_t n, int64_t k, int sms) {
+  for (const TunedTactic& e : kTunedTactics)
+    if (e.n == n && e.k == k && e.sms == sms && m >= e.m_lo && m <= e.m_hi) return e.tactic;
+  return -1;
+}
+
 // The built-in table. m = 1, 2..4 and 5..256 are separate buckets: the tactic (and so the bits
 // of a row) is the same for every m inside a bucket.
 static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms) {
+  const int64_t tuned = tuned_tactic(m, n, k, num_sms);
+  if (tuned >= 0) return tuned;
   if (m <= kDefaultGemvMaxM) {
     const int64_t m_fit = m <= 1 ? 1 : kDefaultGemvMaxM;
     // stream pipeline with its automatic CTA shape and rows per item (see gemv_stream_geometry);
@@ -292,8 +365,12 @@ static int64_t default_tactic_impl(int64_t m, int64_t n, int64_t k, int num_sms)
     // Where k % 256 != 0 the stream pipeline takes its general path (4-byte scale words, lane
     // predicates): there the register pipeline with two CTAs per SM was faster (10304 x 2688:
     // 6.60 against 7.46 us).
+    // At m = 1 with k a multiple of 2048, the lean stream pipeline (measured on B200, cold L2,
+    // PDL-chained graphs: 4096 x 14336 9.45-9.97 against 9.65-10.0 us, 14336 x 4096 9.26-9.37
+    // against 9.4-9.6 us on different boxes).
     const bool small = n * (k / 2 + k / 16) <= ((int64_t)12 << 20);
-    const int pipe = small ? kPipeOverlap : (k % 256 != 0 ? kPipeReg : kPipeStream);
+    const bool lean = m <= 1 && k % (kChunkK * 32 * kLeanIters) == 0;
+    const int pipe = small ? kPipeOverlap : (k % 256 != 0 ? kPipeReg : (lean ? kPipeLean : kPipeStream));
     const int ctas = pipe == kPipeReg ? 2 : 0;
     int S = 1;
     if (gemv_knee(pipe, n, k, num_sms, m_fit, 0, ctas, &S) != FI_OK) S = 1;
@@ -318,17 +395,18 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
   const int rsel = var & 0xF;
   const bool pipe_auto = (var >> 4) == kPipeAuto;
   int pipe = pipe_auto ? kPipeStream : var >> 4;
-  if (var < 0 || pipe > kPipeReg || rsel > 8)
+  if (var < 0 || pipe > kPipeLean || rsel > 8)
     return set_error(FI_ERR_INVALID_ARG,
-                     "GEMV variant 0x%x: rows must be 0, 1, 2, 4 or 8 and the pipeline 0 to 4", var);
+                     "GEMV variant 0x%x: rows must be 0, 1, 2, 4 or 8 and the pipeline 0 to 5", var);
   int S = S_req;
   if (S == 0) {
-    const int rc = gemv_knee(pipe, n, k, sms, kGemvMaxM, 0, ctas, &S);
+    // the lean pipeline takes m = 1 only, so its split is sized for one activation row
+    const int rc = gemv_knee(pipe, n, k, sms, pipe == kPipeLean ? 1 : kGemvMaxM, 0, ctas, &S);
     if (rc != FI_OK) return rc;
   } else if (C > 0 && S > C) {
     return set_error(FI_ERR_INVALID_ARG, "splits=%lld exceeds k/32=%lld", (long long)S, (long long)C);
   }
-  GemvGeometry g;
+  GemvGeometry g{};
   if (C == 0) {  // k == 0: nothing to stream; the caller writes zeros
     memset(&g, 0, sizeof(g));
     g.pipeline = pipe;
@@ -348,7 +426,14 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
     // slower. Same bits: only the pipeline changes.
     const bool reg_rule = k % 256 != 0;
     const int64_t rule_warps = (n + (reg_rule ? 1 : 3)) / (reg_rule ? 2 : 4) * S;
-    if (pipe_auto && m == 1 && S > 1 && rsel == 0 && rule_warps >= 4 * (int64_t)sms) {
+    // at m = 1 the automatic pipeline is the lean stream pipeline wherever its whole items fit
+    // the split (measured on B200 at S = 1: 4096 x 14336 9.45 against 10.0 us, 14336 x 4096
+    // 9.26 against 9.6 us); the bits are those of any other pipeline at the same S
+    if (pipe_auto && m == 1) {
+      rc = geometry_for(kPipeLean, m, n, k, S, rsel, ctas, sms, &g);
+      if (rc != FI_OK) clear_error();
+    }
+    if (rc != FI_OK && pipe_auto && m == 1 && S > 1 && rsel == 0 && rule_warps >= 4 * (int64_t)sms) {
       rc = reg_rule ? geometry_for(kPipeReg, m, n, k, S, 0, ctas ? ctas : 2, sms, &g)
                     : geometry_for(kPipeStream, m, n, k, S, 4, ctas, sms, &g);
       if (rc != FI_OK) clear_error();
@@ -396,12 +481,15 @@ static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req,
     // sms) waves of ceil(KS / S) steps plus about 4 steps of per-CTA start and epilogue. A
     // split adds 3 steps for the reduce launch and the partials' write and read (2 S m n 4
     // bytes at about 4 MB per step, a step being about 0.6 us measured on B200). Take the S
-    // (1..16) of least cost.
+    // (1..16) of least cost. The partials are costed at m = kMmaMaxM whatever the call's m, so
+    // that S (and with it a row's bits) depends on (n, k, SMs) alone: the device-sized code is
+    // batch-invariant like every other tactic code.
     S = 1;
     double best = -1.0;
+    const double m_cost = (double)kMmaMaxM;
     for (int64_t c = 1; c <= std::min<int64_t>(16, std::max<int64_t>(1, KS)); ++c) {
       const double cost = (double)((tiles * c + sms - 1) / sms) * (double)((KS + c - 1) / c + 4) +
-                          (c > 1 ? 3.0 + 2.0 * (double)c * (double)m * (double)n * 4.0 / 4.0e6 : 0.0);
+                          (c > 1 ? 3.0 + 2.0 * (double)c * m_cost * (double)n * 4.0 / 4.0e6 : 0.0);
       if (best < 0 || cost < best) {
         best = cost;
         S = c;
@@ -503,9 +591,12 @@ std::atomic<uint64_t> g_wait_timeout_ns{1000000000ull};
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, const float* gscale,
-                  uint16_t* out, int64_t m, int64_t n, int64_t k, int64_t tactic, void* workspace,
+                  uint16_t* out, int out_dtype, int64_t m, int64_t n, int64_t k, int64_t tactic, void* workspace,
                   size_t workspace_bytes, bool use_registered, cudaStream_t stream) {
   clear_error();
+  if (out_dtype != FI_DTYPE_BF16 && out_dtype != FI_DTYPE_F16)
+    return set_error(FI_ERR_INVALID_ARG, "out_dtype %d is neither FI_DTYPE_BF16 nor FI_DTYPE_F16", out_dtype);
+  const bool out_f16 = out_dtype == FI_DTYPE_F16;
   if (m < 0 || n < 0 || k < 0) return set_error(FI_ERR_INVALID_ARG, "negative size");
   if (k % 32 != 0) return set_error(FI_ERR_UNSUPPORTED_SHAPE, "k=%lld is not a multiple of 32", (long long)k);
   if (m == 0 || n == 0) return FI_OK;
@@ -545,7 +636,7 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     }
   }
   if (info.kind == FI_KIND_GEMV) {
-    GemvGeometry g;
+    GemvGeometry g{};
     rc = geometry_for(info.variant >> 4, m, n, k, info.splits, info.variant & 0xF, info.ctas_per_sm, sms, &g);
     if (rc != FI_OK) return rc;
     GemvArgs a;
@@ -555,6 +646,7 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.Ws = Wscale;
     a.gscale = gscale;
     a.out = out;
+    a.out_f16 = out_f16 ? 1 : 0;
     a.partials = partials;
     a.m = m;
     a.n = n;
@@ -590,6 +682,7 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.Ws = Wscale;
     a.gscale = gscale;
     a.out = out;
+    a.out_f16 = out_f16 ? 1 : 0;
     uint8_t* ws = reinterpret_cast<uint8_t*>(partials);
     a.a16 = reinterpret_cast<uint16_t*>(ws);
     a.rs = reinterpret_cast<float*>(ws + mma_rs_offset(m, k));
@@ -608,10 +701,11 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.timeout_ns = g_wait_timeout_ns;
     rc = launch_mma(a, stream);
     if (rc != FI_OK) return rc;
-    if (info.splits > 1) return launch_splitk_reduce(a.partials, info.splits, m, n, gscale, out, true, stream);
+    if (info.splits > 1)
+      return launch_splitk_reduce(a.partials, info.splits, m, n, gscale, out, out_f16, true, stream);
     return FI_OK;
   }
-  if (info.splits > 1) return launch_splitk_reduce(partials, info.splits, m, n, gscale, out, true, stream);
+  if (info.splits > 1) return launch_splitk_reduce(partials, info.splits, m, n, gscale, out, out_f16, true, stream);
   return FI_OK;
 }
 
@@ -637,20 +731,34 @@ int fi_nvfp4_pack_weights(const float* W, int64_t n, int64_t k, uint8_t* Wq, uin
 
 int fi_mm_bf16_fp4(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, const float* gscale,
                    uint16_t* out, int64_t m, int64_t n, int64_t k, int64_t tactic, fi_stream_t stream) {
-  return mm_run(A, Wq, Wscale, gscale, out, m, n, k, tactic, nullptr, 0, true,
+  return mm_run(A, Wq, Wscale, gscale, out, FI_DTYPE_BF16, m, n, k, tactic, nullptr, 0, true,
                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fi_mm_bf16_fp4_ex(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, const float* gscale,
                       uint16_t* out, int64_t m, int64_t n, int64_t k, int64_t tactic, void* workspace,
                       size_t workspace_bytes, fi_stream_t stream) {
-  return mm_run(A, Wq, Wscale, gscale, out, m, n, k, tactic, workspace, workspace_bytes, false,
+  return mm_run(A, Wq, Wscale, gscale, out, FI_DTYPE_BF16, m, n, k, tactic, workspace, workspace_bytes, false,
                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fi_mm_bf16_fp4_out(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, const float* gscale,
+                       uint16_t* out, int out_dtype, int64_t m, int64_t n, int64_t k, int64_t tactic,
+                       void* workspace, size_t workspace_bytes, fi_stream_t stream) {
+  return mm_run(A, Wq, Wscale, gscale, out, out_dtype, m, n, k, tactic, workspace, workspace_bytes,
+                workspace == nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fi_splitk_reduce(const float* partials, int64_t splits, int64_t m, int64_t n, const float* gscale,
                      uint16_t* out, fi_stream_t stream) {
+  return fi_splitk_reduce_out(partials, splits, m, n, gscale, out, FI_DTYPE_BF16, stream);
+}
+
+int fi_splitk_reduce_out(const float* partials, int64_t splits, int64_t m, int64_t n, const float* gscale,
+                         uint16_t* out, int out_dtype, fi_stream_t stream) {
   clear_error();
+  if (out_dtype != FI_DTYPE_BF16 && out_dtype != FI_DTYPE_F16)
+    return set_error(FI_ERR_INVALID_ARG, "out_dtype %d is neither FI_DTYPE_BF16 nor FI_DTYPE_F16", out_dtype);
   if (m < 0 || n < 0) return set_error(FI_ERR_INVALID_ARG, "negative size");
   if (splits < 1 || splits > 4095) return set_error(FI_ERR_INVALID_ARG, "splits must be in [1, 4095]");
   if (m == 0 || n == 0) return FI_OK;
@@ -659,7 +767,7 @@ int fi_splitk_reduce(const float* partials, int64_t splits, int64_t m, int64_t n
     return set_error(FI_ERR_INVALID_ARG, "partials must be 16-byte, out 2-byte aligned");
   const int rc = check_arch();
   if (rc != FI_OK) return rc;
-  return launch_splitk_reduce(partials, (int)splits, m, n, gscale, out, false,
+  return launch_splitk_reduce(partials, (int)splits, m, n, gscale, out, out_dtype == FI_DTYPE_F16, false,
                               reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -695,6 +803,7 @@ int fi_list_tactics(int64_t m, int64_t n, int64_t k, int num_sms, int64_t* out, 
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 2, kPipeStream << 4);
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeOverlap << 4);
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeReg << 4);
+  for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_GEMV, S, 0, kPipeLean << 4);
   for (int S : splits) cand[nc++] = FI_TACTIC(FI_KIND_MMA, S, 0, 0);
   fi_tactic_info seen[64];
   int nseen = 0, count = 0;

@@ -112,7 +112,7 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
   return r;
 }
 
-// ------------------------------------------------------------------- bf16 output
+// ------------------------------------------------------------------- output rounding
 
 __device__ __forceinline__ uint16_t f32_to_bf16_rn(float x) {
   unsigned short r;
@@ -121,6 +121,16 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float x) {
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+// fp32 -> IEEE binary16 bits, round to nearest even (the optional f16 output).
+__device__ __forceinline__ uint16_t f32_to_f16_rn(float x) {
+  unsigned short r;
+  asm("cvt.rn.f16.f32 %0, %1;" : "=h"(r) : "f"(x));
+  return r;
+}
+
+// The output element's bits: bf16 (f16 == false) or f16, round to nearest even.
+__device__ __forceinline__ uint16_t f32_to_out(float x, bool f16) { return f16 ? f32_to_f16_rn(x) : f32_to_bf16_rn(x); }
 
 // ---------------------------------------------------- programmatic dependent launch
 

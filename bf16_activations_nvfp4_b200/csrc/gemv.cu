@@ -32,9 +32,9 @@
 //    per group, CTA shape and grid): A is staged as f16 with one power-of-two scale sf_a per
 //    16-block that puts the block maximum in [2^9, 2^10) (exact for every element within 2^26
 //    of its block maximum); codes are decoded by cvt.rn.f16x2.e2m1x2 (exact). Per 16-block, the
-//    16 products (each exact in fp32) are summed in fp32 in element order by the
-//    mixed-precision fma.rn.f32.f16, and acc = fma(t, sw * sf_a, acc) with sw the block's E4M3
-//    scale. Lane L takes chunks L, L+32, L+64, ... of the split; the lanes combine through a
+//    16 products (each exact in fp32) are summed in fp32 by the mixed-precision fma.rn.f32.f16,
+//    the even and the odd elements in two chains in element order, t = even + odd, and
+//    acc = fma(t, sw * sf_a, acc) with sw the block's E4M3 scale. Lane L takes chunks L, L+32, L+64, ... of the split; the lanes combine through a
 //    fixed xor butterfly (all lanes end with the same bits). S == 1 writes bf16_rn(acc *
 //    gscale); S > 1 writes fp32 partials for the reduce kernel.
 //  * Bounded waits (ring pipeline). Every mbarrier wait gives up after a time limit
@@ -126,16 +126,17 @@ __device__ __forceinline__ void stage_block(const uint4 v0, const uint4 v1, int 
 // contiguous bytes per quad. Values are f16 scaled by a power of two per 16-block that puts
 // the block maximum in [2^9, 2^10); As[r][b] holds the inverse scale. A thread loads up to four
 // of its blocks before converting any, so their global-memory latencies overlap.
+template <int U = 4>
 __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A, int64_t k, int m,
                                                   int64_t kbase, int nch, uint4* Ah4, float* As, int tid,
                                                   int nthreads) {
   const int GA = (nch + 31) / 32;
   const int blocks_per_row = nch * 2;
   const int nblk = m * blocks_per_row;
-  for (int b0 = tid; b0 < nblk; b0 += 4 * nthreads) {
-    uint4 v[4][2];
+  for (int b0 = tid; b0 < nblk; b0 += U * nthreads) {
+    uint4 v[U][2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int bi = b0 + u * nthreads;
       if (bi < nblk) {
         const int r = bi / blocks_per_row;
@@ -145,7 +146,7 @@ __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int bi = b0 + u * nthreads;
       if (bi < nblk) {
         const int r = bi / blocks_per_row;
@@ -155,23 +156,24 @@ __device__ __forceinline__ void stage_activations(const uint16_t* __restrict__ A
   }
 }
 
-// The 16 products of one 16-block summed in fp32, in element order: a and w hold the block's
-// 8 f16 pairs (element 2j in the low half of word j). Each product of two f16 values is exact
-// in fp32, and the mixed-precision fma.rn.f32.f16 adds it to the running fp32 sum with one
-// round-to-nearest-even, so this is the block's dot product accumulated in fp32.
+// The 16 products of one 16-block summed in fp32: a and w hold the block's 8 f16 pairs
+// (element 2j in the low half of word j). Each product of two f16 values is exact in fp32; the
+// mixed-precision fma.rn.f32.f16 adds it to a running fp32 sum with one round-to-nearest-even.
+// The even elements and the odd elements are summed in two chains, each in element order
+// (two chains halve the dependent-latency path), and the block's sum is even + odd.
 __device__ __forceinline__ float block_dot(const uint32_t* a, const uint32_t* w) {
-  float t;
-  asm("{\n .reg .b16 al, ah, wl, wh;\n mov.b32 {al, ah}, %1;\n mov.b32 {wl, wh}, %2;\n"
-      " fma.rn.f32.f16 %0, al, wl, 0f00000000;\n fma.rn.f32.f16 %0, ah, wh, %0;\n}"
-      : "=f"(t)
+  float te, to;
+  asm("{\n .reg .b16 al, ah, wl, wh;\n mov.b32 {al, ah}, %2;\n mov.b32 {wl, wh}, %3;\n"
+      " fma.rn.f32.f16 %0, al, wl, 0f00000000;\n fma.rn.f32.f16 %1, ah, wh, 0f00000000;\n}"
+      : "=f"(te), "=f"(to)
       : "r"(a[0]), "r"(w[0]));
 #pragma unroll
   for (int i = 1; i < 8; ++i)
-    asm("{\n .reg .b16 al, ah, wl, wh;\n mov.b32 {al, ah}, %1;\n mov.b32 {wl, wh}, %2;\n"
-        " fma.rn.f32.f16 %0, al, wl, %0;\n fma.rn.f32.f16 %0, ah, wh, %0;\n}"
-        : "+f"(t)
+    asm("{\n .reg .b16 al, ah, wl, wh;\n mov.b32 {al, ah}, %2;\n mov.b32 {wl, wh}, %3;\n"
+        " fma.rn.f32.f16 %0, al, wl, %0;\n fma.rn.f32.f16 %1, ah, wh, %1;\n}"
+        : "+f"(te), "+f"(to)
         : "r"(a[i]), "r"(w[i]));
-  return t;
+  return __fadd_rn(te, to);
 }
 
 // One 32-k chunk of one weight row against one activation row: av the chunk's 16 staged f16
@@ -254,7 +256,8 @@ __device__ __forceinline__ void stage_rows(uint32_t code0, int cstride, uint32_t
 }
 
 // Combine the lanes of acc (fixed xor butterfly: every lane ends with the same bits) and
-// write rows j0 .. j0+rows-1: bf16_rn(acc * g) when S == 1, else the fp32 partial of split s.
+// write rows j0 .. j0+rows-1: round(acc * g) to the output type (bf16, or f16) when S == 1,
+// else the fp32 partial of split s.
 template <int MT, int NR>
 __device__ __forceinline__ void finish_rows(float (&acc)[NR][MT], const GemvArgs& p, int64_t j0, int rows, int m,
                                             int S, int s, float g, int lane, bool write) {
@@ -275,7 +278,7 @@ __device__ __forceinline__ void finish_rows(float (&acc)[NR][MT], const GemvArgs
       if (i < rows && r < m && lane == ((i * MT + r) & 31)) {
         const int64_t j = j0 + i;
         if (S == 1)
-          p.out[(int64_t)r * p.n + j] = f32_to_bf16_rn(acc[i][r] * g);
+          p.out[(int64_t)r * p.n + j] = f32_to_out(acc[i][r] * g, p.out_f16 != 0);
         else
           p.partials[((int64_t)s * m + r) * p.n + j] = acc[i][r];
       }
@@ -846,6 +849,140 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_stream_kernel(GemvA
 }
 
 // ---------------------------------------------------------------------------------------
+// Lean stream pipeline (pipeline 5, m = 1). The stream pipeline's per-lane asynchronous
+// copies, cut to what decode needs: one activation row, k % 256 == 0, and splits of whole 32-k
+// chunk iterations. A slot holds R rows x TI chunk iterations: row i's cells of iteration ti
+// at (i * TI + ti) * 512 (lane L's at + 16 L) and its scales at R * TI * 512 + (i * TI + ti) * 64
+// (lane L's two bytes at + 2 L); a row group's last item may hold fewer iterations. The item
+// loop is unrolled over the NS slots of the warp's ring, so every shared-memory address of the
+// inner loop is a per-item base plus a compile-time offset, and the copy cursor is one pointer
+// per tensor. The activations of the split are staged once per CTA; grid.y is the K split, as in
+// the other pipelines.
+template <int R, int NS>
+__global__ void __launch_bounds__(kStreamMaxThreads, 1) gemv_lean_kernel(GemvArgs p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int TI = kLeanIters;
+  constexpr uint32_t kCodes = (uint32_t)(R * TI * 512), kSlot = kCodes + (uint32_t)(R * TI * 64);
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int NW = (int)(blockDim.x >> 5);
+  const int64_t n = p.n, k = p.k;
+  const int S = p.splits;
+  const int s = blockIdx.y;
+
+  const int64_t C = k / kChunkK;
+  const int64_t c0 = (int64_t)s * C / S;
+  const int nch = (int)((int64_t)(s + 1) * C / S - c0);  // a multiple of 32
+  const int T = nch / 32;                               // chunk iterations of a row
+  const int TT = (T + TI - 1) / TI;                     // items of a row group
+
+  const int64_t GW = (int64_t)gridDim.x * NW;
+  const int64_t gw = (int64_t)blockIdx.x * NW + warp;
+  const int64_t ngr = (n + R - 1) / R;
+  const int64_t g_lo = gw * ngr / GW, g_hi = (gw + 1) * ngr / GW;
+  const int64_t r_lo = g_lo * R, r_hi = min(n, g_hi * R);
+  const int Q = (int)(g_hi - g_lo) * TT;
+
+  const int64_t rs_q = k / 2, rs_s = k / 16;
+  const uint32_t ring = smem_addr(smem + p.off_ring) + (uint32_t)warp * NS * kSlot;
+  const uint32_t my_code = ring + (uint32_t)lane * 16;
+  // scale pieces: lane L < 4 * TI * R copies bytes [16 (L % 4TI), +16) of row L / 4TI's item
+  // range (TI * 64 bytes) to kCodes + 16 L of the slot; the piece belongs to iteration (L % 4TI) / 4
+  const bool s_lane = lane < 4 * TI * R;
+  const int i_l = lane / (4 * TI), ti_l = (lane % (4 * TI)) / 4;
+  const uint32_t my_s16 = ring + kCodes + (uint32_t)lane * 16;
+
+  // ---- copy cursor: code cell of row 0 for this lane, this lane's scale piece, rows present
+  const uint8_t* gq = p.Wq + r_lo * rs_q + (c0 + lane) * 16;
+  const uint8_t* gs = p.Ws + (r_lo + (s_lane ? i_l : 0)) * rs_s + c0 * 2 + (lane % (4 * TI)) * 16;
+  // from the end of a group's last item to the next group's first (every item advances the
+  // cursor by TI iterations, a short last item included)
+  const int64_t dq = (int64_t)R * rs_q - (int64_t)TT * TI * 512;
+  const int64_t ds = (int64_t)R * rs_s - (int64_t)TT * TI * 64;
+  int rows_i = (int)min((int64_t)R, r_hi - r_lo);  // rows of the group being copied
+  int itt = 0, iq = 0;
+  auto issue = [&](uint32_t off) {
+    if (iq < Q) {
+      const int tin = min(TI, T - itt * TI);  // iterations of this item
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+        if (i < rows_i)
+#pragma unroll
+          for (int ti = 0; ti < TI; ++ti)
+            if (ti < tin) cp_async_16(my_code + off + (uint32_t)((i * TI + ti) * 512), gq + i * rs_q + ti * 512);
+      if (s_lane && i_l < rows_i && ti_l < tin) cp_async_16(my_s16 + off, gs);
+      gq += TI * 512;
+      gs += TI * 64;
+      if (++itt == TT) {
+        itt = 0;
+        gq += dq;
+        gs += ds;
+        rows_i = (int)min((int64_t)R, r_hi - (r_lo + (int64_t)(iq / TT + 1) * R));
+      }
+      ++iq;
+    }
+    cp_async_commit();
+  };
+  pdl_launch_dependents();
+#pragma unroll
+  for (int u = 0; u < NS; ++u) issue((uint32_t)u * kSlot);
+
+  pdl_wait();
+  {  // the split's activations (one activation row), staged once per CTA
+    const int GA = (nch + 31) / 32;
+    uint4* Ah4 = reinterpret_cast<uint4*>(smem);
+    float* As = reinterpret_cast<float*>(smem + p.off_as);
+    const uint16_t* src = p.A + c0 * kChunkK;
+    for (int b = tid; b < 2 * nch; b += (int)blockDim.x) {
+      const uint4 v0 = ldg_v4(src + b * 16), v1 = ldg_v4(src + b * 16 + 8);
+      stage_block(v0, v1, 0, b, GA, 2 * nch, Ah4, As);
+    }
+  }
+  __syncthreads();
+  const float g = (S == 1) ? *p.gscale : 1.0f;
+
+  const uint32_t a_lane = smem_addr(smem) + (uint32_t)lane * 16;
+  const uint32_t as_lane = smem_addr(smem + p.off_as) + (uint32_t)lane * 8;
+  const uint32_t sc_lane = ring + kCodes + (uint32_t)lane * 2;
+  const uint32_t zoff[R] = {};
+  float acc[R][1];
+#pragma unroll
+  for (int i = 0; i < R; ++i) acc[i][0] = 0.0f;
+  int64_t j0 = r_lo;
+  int ctt = 0;
+  uint32_t ac = a_lane, asc = as_lane;
+  for (int q0 = 0; q0 < Q; q0 += NS) {
+#pragma unroll
+    for (int u = 0; u < NS; ++u) {
+      if (q0 + u < Q) {
+        cp_async_wait<NS - 1>();  // this lane's copies of item q0 + u have landed
+        const int tin = min(TI, T - ctt * TI);
+#pragma unroll
+        for (int ti = 0; ti < TI; ++ti)
+          if (ti < tin)
+            item_rows<1, R, TI * 512, TI * 64>(my_code + (uint32_t)(u * kSlot + ti * 512),
+                                               sc_lane + (uint32_t)(u * kSlot + ti * 64), zoff,
+                                               ac + (uint32_t)ti * 2048, asc + (uint32_t)ti * 256, 0, 0, 1, acc);
+        issue((uint32_t)u * kSlot);  // refill the slot just read with item q0 + u + NS
+        ac += TI * 2048;
+        asc += TI * 256;
+        if (++ctt == TT) {
+          finish_rows<1, R>(acc, p, j0, (int)min((int64_t)R, r_hi - j0), 1, S, s, g, lane, true);
+#pragma unroll
+          for (int i = 0; i < R; ++i) acc[i][0] = 0.0f;
+          ctt = 0;
+          ac = a_lane;
+          asc = as_lane;
+          j0 += R;
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------------------
 // Register pipeline (pipeline 4): the weights go from global memory straight to registers
 // with 16-byte loads, as in the pages' streaming GEMV; nothing is copied to shared memory but
 // the staged activations. Each warp keeps the loads of its next D chunk iterations in flight
@@ -1084,8 +1221,38 @@ int launch_reg(const GemvArgs& a, cudaStream_t stream) {
   return FI_OK;
 }
 
+template <int R>
+int launch_lean(const GemvArgs& a, cudaStream_t stream) {
+  auto kern = a.stages == 4 ? gemv_lean_kernel<R, 4> : gemv_lean_kernel<R, 2>;
+  static int configured[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return set_cuda_error("cudaGetDevice");
+  if (!(configured[dev] & (a.stages == 4 ? 1 : 2))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget) != cudaSuccess)
+      return set_cuda_error("cudaFuncSetAttribute(gemv lean smem)");
+    configured[dev] |= a.stages == 4 ? 1 : 2;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.grid_x, (unsigned)a.splits);
+  cfg.blockDim = dim3((unsigned)a.threads);
+  cfg.dynamicSmemBytes = (size_t)a.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return set_cuda_error("gemv lean kernel launch");
+  return FI_OK;
+}
+
 template <int MT, int R>
 int launch_stream_ns(const GemvArgs& a, cudaStream_t stream) {
+  if (a.pipeline == kPipeLean) {
+    if constexpr (MT == 1) return launch_lean<R>(a, stream);
+    return set_error(FI_ERR_INVALID_ARG, "GEMV lean pipeline: m = 1 only");
+  }
   if (a.pipeline == kPipeReg) {
     if constexpr (R <= 2) return launch_reg<MT, R>(a, stream);  // R = 4 would spill the register ring
     return set_error(FI_ERR_INVALID_ARG, "GEMV register pipeline: at most 2 rows per warp");

@@ -40,8 +40,9 @@ constexpr int kStreamIters = 2;                            // chunk iterations p
 constexpr int kStreamCellBytes = 32 * 16 + 32 * 4;         // one iteration of one row: code cells + scale words
 constexpr int kStreamHalfBudget = 228 * 1024 / 2 - 1024;   // dynamic shared memory per CTA, two CTAs per SM
 // pipelines (the high nibble of the GEMV tactic variant)
-constexpr int kPipeAuto = 0, kPipeStream = 1, kPipeRing = 2, kPipeOverlap = 3, kPipeReg = 4;
-constexpr int kRegDepth = 4;  // register pipeline: chunk iterations in flight per warp
+constexpr int kPipeAuto = 0, kPipeStream = 1, kPipeRing = 2, kPipeOverlap = 3, kPipeReg = 4, kPipeLean = 5;
+constexpr int kRegDepth = 4;   // register pipeline: chunk iterations in flight per warp
+constexpr int kLeanIters = 2;  // lean stream pipeline: chunk iterations per work item
 
 // Activation rows the GEMV kernel instance for m is compiled for (1, 2, 4, ..., 32).
 inline int gemv_mt(int64_t m) {
@@ -65,7 +66,7 @@ int gemv_rows_per_stage_max(int64_t m);
 // Launch geometry of the GEMV for one shape and tactic (computed on the host).
 struct GemvGeometry {
   int pipeline;  // kPipeStream or kPipeRing
-  int S, RS, stages, ctas_per_sm, grid_x, threads;
+  int S, RS, stages, ctas_per_sm, grid_x, grid_y, threads;
   int64_t stage_bytes, off_as, off_bar, off_ring, smem_bytes;
 };
 // Returns FI_OK and fills g, or FI_ERR_UNSUPPORTED_SHAPE when the activations of m rows over
@@ -83,6 +84,7 @@ struct GemvArgs {
   const uint8_t* Ws;
   const float* gscale;
   uint16_t* out;       // used when splits == 1
+  int out_f16;         // out holds f16 (1) or bf16 (0)
   float* partials;     // [splits, m, n] when splits > 1
   int64_t m, n, k;
   int pipeline;        // kPipeStream or kPipeRing
@@ -131,6 +133,7 @@ struct MmaArgs {
   const uint8_t* Ws;
   const float* gscale;
   uint16_t* out;
+  int out_f16;    // out holds f16 (1) or bf16 (0)
   uint16_t* a16;  // workspace: f16 activations [m_pad, k]
   float* rs;      // workspace: per-row inverse scales [m_pad]
   int64_t m, n, k;
@@ -149,7 +152,7 @@ unsigned* device_error_word();
 
 // ---------------------------------------------------------------------- reduce
 int launch_splitk_reduce(const float* partials, int splits, int64_t m, int64_t n,
-                         const float* gscale, uint16_t* out, bool pdl, cudaStream_t stream);
+                         const float* gscale, uint16_t* out, bool out_f16, bool pdl, cudaStream_t stream);
 
 // ------------------------------------------------------------------------ pack
 int launch_pack(const float* W, int64_t n, int64_t k, uint8_t* Wq, uint8_t* Wscale,

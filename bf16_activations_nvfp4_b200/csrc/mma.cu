@@ -21,8 +21,8 @@
 //      warps 1, 23 the MMAs, one thread each, one M = 128 half of the tile each (warp 1 also
 //                  allocates TMEM): per 64-k step 4 K=16 steps, N = m_pad, accumulating in
 //                  TMEM; tcgen05.commit frees the stage once both halves have read it;
-//      warps 19-22 epilogue: tcgen05.ld of the accumulator, out[j][i] = bf16_rn(D[i][j] *
-//                  rs[j] * gscale).
+//      warps 19-22 epilogue: tcgen05.ld of the accumulator, out[j][i] = round(D[i][j] *
+//                  rs[j] * gscale) to bf16 (or f16).
 //  * The weight tile is decoded once per call (the activations, m_pad <= 256 rows, are one MMA
 //    N tile), so the decode work is one cvt and one f16 multiply per two codes.
 //  * Every wait is bounded (see sync.cuh); on a timeout the roles stop, the MMA issuer and the
@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     if (ok) {
       const float g = *p.gscale;
       // S > 1: this split's fp32 partials D * rs[j] (exact: rs is a power of two), summed in
-      // split order by the reduce kernel; S == 1: bf16_rn(D * rs[j] * gscale)
+      // split order by the reduce kernel; S == 1: round(D * rs[j] * gscale) to the output type
       float* const part = S > 1 ? p.partials + (int64_t)sp * m * n : nullptr;
       for (int h = 0; h < 2; ++h) {
         const int64_t row = w0 + h * 128 + i;
@@ -476,7 +476,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
 #pragma unroll
               for (int jj = 0; jj < 16; ++jj) {
                 const int j = j0 + jj;
-                if (j < m) p.out[(int64_t)j * n + row] = f32_to_bf16_rn(__fmul_rn(__fmul_rn(v[jj], p.rs[j]), g));
+                if (j < m)
+                  p.out[(int64_t)j * n + row] = f32_to_out(__fmul_rn(__fmul_rn(v[jj], p.rs[j]), g), p.out_f16 != 0);
               }
             } else {
 #pragma unroll

@@ -66,15 +66,23 @@ int fi_mm_bf16_fp4_noalloc(const uint16_t* A, const uint8_t* Wq, const uint8_t* 
     return fi_mm_bf16_fp4_ex(A, Wq, Wscale, gscale, out, m, n, k, tactic, nullptr, 0, stream);
   // The default tactic whose scratch would not fit takes, with the same kind, the largest
   // split below its own that fits (the split changes the bits, as any split does).
+  // Validity comes from fi_resolve_tactic: a single-split GEMV is valid with no scratch at all.
+  // A GEMV keeps the default's pipeline where that fits the smaller split, else takes the
+  // automatic pipeline (which falls back to the producer-warp ring when the activations of a
+  // longer split do not fit the other pipelines' shared memory); the bits depend on S only.
   if (tactic == FI_TACTIC_DEFAULT && fi_mm_workspace_bytes(m, n, k, tactic, 0) > kNoAllocScratchBytes) {
     fi_tactic_info info;
     if (fi_resolve_tactic(m, n, k, tactic, 0, &info) == FI_OK) {
-      for (int S = info.splits - 1; S >= 1; --S) {
-        const int64_t t = FI_TACTIC(info.kind, S, 0, info.kind == FI_KIND_GEMV ? (info.variant >> 4) << 4 : 0);
-        const size_t w = fi_mm_workspace_bytes(m, n, k, t, 0);
-        if (w > 0 && w <= kNoAllocScratchBytes) {
-          tactic = t;
-          break;
+      for (int S = info.splits - 1; S >= 1 && tactic == FI_TACTIC_DEFAULT; --S) {
+        const int pipe_bits = info.kind == FI_KIND_GEMV ? (info.variant >> 4) << 4 : 0;
+        for (int v : {pipe_bits, 0}) {
+          const int64_t t = FI_TACTIC(info.kind, S, 0, v);
+          fi_tactic_info ti;
+          if (fi_resolve_tactic(m, n, k, t, 0, &ti) == FI_OK &&
+              (size_t)ti.workspace_bytes <= kNoAllocScratchBytes) {
+            tactic = t;
+            break;
+          }
         }
       }
     }

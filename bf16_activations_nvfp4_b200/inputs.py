@@ -64,3 +64,6 @@ SMALL_BATCH_M = [1, 2, 4, 8, 16, 32]
 SMALL_BATCH_NK = (4096, 14336)
 LM_HEAD_NK = (152064, 5120)
 LM_HEAD_M = [1, 64, 256]
+# second workload: the Qwen3.6-27B-shaped decode GEMMs at m = 1 of PR #4038's table of them
+# (fused gate/up 34816 x 5120, down 5120 x 17408, lm_head 248320 x 5120); synthetic weights
+QWEN36_27B_DECODE = [(34816, 5120), (5120, 17408), (248320, 5120)]

@@ -80,7 +80,14 @@ typedef enum {
  *                asynchronous copies, 2 = producer-warp ring, 3 = per-warp
  *                copies in one half-SM CTA per SM, so that consecutive calls overlap, with
  *                an L2 prefetch of weights up to 40 MB; its CTAs-per-SM field is ignored;
- *                4 = weights loaded straight to registers, 1 or 2 rows per warp). MMA: 0.
+ *                4 = weights loaded straight to registers, 1 or 2 rows per warp;
+ *                5 = the lean form of 1 for m = 1: k % 256 == 0 and every split's k/32 chunks
+ *                a multiple of 32, 1, 2 or 4 rows per item). MMA: 0. At m = 1 the automatic
+ *                pipeline is 5 wherever it applies.
+ *                The default table: for the shapes the library's cold-L2 tuner measured (the
+ *                generated csrc/tactic_table.inc, per SM count and bucket of m), its pick;
+ *                otherwise at m = 1, 3 for weights up to 12 MB, else 4 where k % 256 != 0, 5
+ *                where k % 2048 == 0, 1 otherwise.
  * Only `kind` and the resolved S change the arithmetic: two tactics with the same kind
  * and S give bitwise identical outputs (whatever their pipeline, rows or CTAs), and for a
  * fixed tactic every output row is bitwise independent of m. Both kinds form every product
@@ -116,6 +123,10 @@ typedef struct {
   int32_t smem_bytes;  /* dynamic shared memory per CTA */
   int64_t workspace_bytes; /* scratch: GEMV fp32 partials (0 if S == 1); MMA f16 A, then partials if S > 1 */
 } fi_tactic_info;
+
+/* Output element types (the op writes bf16 by default; PR #4038's commits add an fp16 output
+ * through the GEMV path, covered by its test of fp16 GEMV output). */
+typedef enum { FI_DTYPE_BF16 = 0, FI_DTYPE_F16 = 1 } fi_dtype;
 
 /* ------------------------------------------------------------------ entry points */
 
@@ -174,6 +185,24 @@ FI_API int fi_mm_bf16_fp4_ex(const uint16_t* A, const uint8_t* Wq, const uint8_t
                       fi_stream_t stream);
 
 /*
+ * fi_mm_bf16_fp4 with a choice of output type (PR #4038, the commit that covers fp16 output
+ * through the GEMV path): out_dtype FI_DTYPE_BF16 writes bf16 bits as fi_mm_bf16_fp4 does,
+ * FI_DTYPE_F16 writes IEEE binary16 bits, rounded to nearest even from the same fp32 value
+ * (magnitudes of 65520 and more become +-inf). Every tactic and kind supports both; the fp32
+ * arithmetic before the final rounding is the same, so the two outputs of one tactic are the
+ * two roundings of one fp32 result.
+ *   out        device [m, n] of 16-bit elements, 2-byte aligned.
+ *   workspace  NULL: the per-device workspace of fi_mm_bf16_fp4 (registered or allocated, with
+ *              its rules under stream capture); otherwise as fi_mm_bf16_fp4_ex.
+ * Other arguments, preconditions and errors are those of fi_mm_bf16_fp4 / fi_mm_bf16_fp4_ex;
+ * an out_dtype other than the two above returns FI_ERR_INVALID_ARG.
+ */
+FI_API int fi_mm_bf16_fp4_out(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale,
+                       const float* gscale, uint16_t* out, int out_dtype, int64_t m, int64_t n,
+                       int64_t k, int64_t tactic, void* workspace, size_t workspace_bytes,
+                       fi_stream_t stream);
+
+/*
  * fi_mm_bf16_fp4 without any device allocation. The paper has no counterpart: this entry
  * point exists for users of this library who may not allocate GPU memory at call time, such
  * as an operator plugin inside a serving engine that has already reserved the device's memory
@@ -188,8 +217,9 @@ FI_API int fi_mm_bf16_fp4_ex(const uint16_t* A, const uint8_t* Wq, const uint8_t
  * 2 * m * k, plus 4 * splits * m * n when split) must not exceed FI_NOALLOC_SCRATCH_BYTES; a
  * larger call returns FI_ERR_WORKSPACE and launches nothing. Single-split GEMV tactics use no
  * scratch. With FI_TACTIC_DEFAULT, a default whose scratch would not fit is replaced by the
- * same kind with the largest smaller split that fits (so its bits may differ from
- * fi_mm_bf16_fp4's default for that shape).
+ * same kind with the largest smaller split that fits (for a GEMV, with the default's pipeline
+ * where that resolves at the smaller split, else the automatic one; a single split needs no
+ * scratch), so its bits may differ from fi_mm_bf16_fp4's default for that shape.
  * Set-up: the first call on a device that reaches a launch looks up the array's device
  * address (cudaGetSymbolAddress, with that device current); make that first call before any
  * stream capture begins.
@@ -217,6 +247,12 @@ FI_API int fi_mm_bf16_fp4_noalloc(const uint16_t* A, const uint8_t* Wq, const ui
  */
 FI_API int fi_splitk_reduce(const float* partials, int64_t splits, int64_t m, int64_t n,
                      const float* gscale, uint16_t* out, fi_stream_t stream);
+
+/* fi_splitk_reduce with a choice of output type: out = round(s * gscale[0]) to bf16
+ * (FI_DTYPE_BF16) or to IEEE binary16 (FI_DTYPE_F16, round to nearest even, +-inf from 65520
+ * on); FI_ERR_INVALID_ARG for any other out_dtype. */
+FI_API int fi_splitk_reduce_out(const float* partials, int64_t splits, int64_t m, int64_t n,
+                         const float* gscale, uint16_t* out, int out_dtype, fi_stream_t stream);
 
 /* --------------------------------------------------------------- host helpers
  * These run on the host only and never launch work. `num_sms` <= 0 means "query the

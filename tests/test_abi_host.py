@@ -49,19 +49,20 @@ def test_default_gemv_tactic_resolves_for_decode_shapes(n, k):
     assert 1 <= info["splits"] <= k // 32
     # one persistent wave: the grid never asks for more CTAs than the SMs hold
     assert info["grid_x"] * info["grid_y"] <= B200_SMS * info["ctas_per_sm"]
-    # the default runs the per-warp async-copy pipeline: one CTA of up to 16 warps per SM, or
-    # two of up to 8 warps within half an SM each; weights of at most 12 MB take the overlapped
-    # variant (one half-SM CTA per SM). Fewer warps only where the row groups would otherwise
+    # the default runs the per-warp async-copy pipeline (its lean form where k % 2048 == 0): one
+    # CTA of up to 16 warps per SM, or two of up to 8 warps within half an SM each; weights of at
+    # most 12 MB take the overlapped variant (one half-SM CTA per SM). Fewer warps only where the row groups would otherwise
     # leave SMs idle, and then the grid spans every SM of the split's share
     pipe = info["variant"] >> 4
     small = n * (k // 2 + k // 16) <= 12 << 20
-    assert pipe == (3 if small else (4 if k % 256 else 1))
+    assert pipe == (3 if small else (4 if k % 256 else (5 if k % 2048 == 0 else 1)))
     warps = info["threads"] // 32
+    wide = 16
     if info["ctas_per_sm"] == 1:
-        assert 4 <= warps <= 16 and 0 < info["smem_bytes"] <= 227 * 1024 - 1024
+        assert 4 <= warps <= wide and 0 < info["smem_bytes"] <= 227 * 1024 - 1024
     else:
-        assert 4 <= warps <= 8 and 0 < info["smem_bytes"] <= 228 * 1024 // 2 - 1024
-    full = 16 if info["ctas_per_sm"] == 1 else 8
+        assert 4 <= warps <= wide // 2 and 0 < info["smem_bytes"] <= 228 * 1024 // 2 - 1024
+    full = wide if info["ctas_per_sm"] == 1 else wide // 2
     if warps < full:
         share = B200_SMS * (1 if pipe == 3 else info["ctas_per_sm"]) // info["splits"]
         assert info["grid_x"] >= 0.95 * share or warps == 4, info  # whole groups per warp round the grid
@@ -139,7 +140,11 @@ def test_workspace_bytes():
     (32, 64, 14336, fi.make_tactic(0, 1, 0, 1), -2),      # A slice does not fit shared memory
     (32, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),       # one row per stage above m = 8
     (5, 64, 4096, fi.make_tactic(0, 1, 0, 4), -1),        # two rows per stage above m = 4
-    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x52), -1),     # pipeline 5
+    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x62), -1),     # pipeline 6
+    (1, 64, 2688, fi.make_tactic(0, 1, 0, 0x52), -2),     # the lean pipeline needs k % 256 == 0
+    (1, 64, 4096, fi.make_tactic(0, 3, 0, 0x52), -2),     # ... and splits of whole 64-chunk items
+    (2, 64, 4096, fi.make_tactic(0, 1, 0, 0x52), -2),     # the lean pipeline takes m = 1 only
+    (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x58), -1),     # lean pipeline: 1, 2 or 4 rows per item
     (1, 64, 4096, fi.make_tactic(0, 1, 0, 0x19), -1),     # rows 9 on the stream pipeline
     (1, 8, 65536, fi.make_tactic(0, 1, 0, 0x22), -2),     # ring: two 36 KB rows per stage do not fit twice
     (1, 8, 65536, fi.make_tactic(0, 1, 2, 0x11), -2),     # stream, half-SM CTAs: 128 KB of activations
@@ -248,6 +253,16 @@ def test_mma_device_sized_split_follows_the_wave_step_model():
         fi.resolve_tactic(64, 4096, 128, fi.make_tactic(fi.KIND_MMA, 3, 0, 0), B200_SMS)
 
 
+@pytest.mark.parametrize("n,k", [(4096, 14336), (14336, 4096), (2048, 7168), (4096, 4096), (152064, 5120),
+                                 (512, 2048), (1000, 2688 + 64), (129, 1088)])
+def test_mma_device_sized_split_does_not_depend_on_m(n, k):
+    """A row's bits depend on the kind and the resolved S; the device-sized MMA split must
+    therefore resolve to one S for every m (1..256), so that the code is batch-invariant."""
+    mma = fi.make_tactic(fi.KIND_MMA, 0, 0, 0)
+    splits = {fi.resolve_tactic(m, n, k, mma, B200_SMS)["splits"] for m in (1, 2, 5, 8, 16, 17, 32, 64, 100, 256)}
+    assert len(splits) == 1, (n, k, splits)
+
+
 def test_register_pipeline_geometry():
     """Pipeline 4: shared memory holds only the staged activations, 1 or 2 rows per warp, and
     the grid spreads over the SMs like the stream pipeline's."""
@@ -261,28 +276,38 @@ def test_register_pipeline_geometry():
         fi.resolve_tactic(1, 4096, 4096, fi.make_tactic(fi.KIND_GEMV, 1, 0, 0x44), B200_SMS)  # 4 rows would spill
 
 
+def _lean_fits(k, S):
+    """The lean pipeline takes splits of whole 32-chunk iterations: k % 256 == 0, (k / 32) % (32 S) == 0."""
+    return k % 256 == 0 and (k // 32) % (32 * S) == 0
+
+
 def test_automatic_pipeline_for_split_calls_at_m1():
-    """At m = 1 with a K split, the automatic pipeline takes the register pipeline (two CTAs per
-    SM) where k % 256 != 0 and four rows per stream item otherwise; S itself is unchanged, and
-    m > 1 keeps the stream pipeline's own row choice."""
+    """At m = 1 the automatic pipeline is the lean stream pipeline where its whole items fit the
+    split; otherwise, with a K split, the register pipeline (two CTAs per SM) where k % 256 != 0
+    and four rows per stream item elsewhere; S itself is unchanged, and m > 1 keeps the stream
+    pipeline's own row choice."""
     for n, k in [(4096, 14336), (2048, 7168), (4096, 4096), (10304, 2688)]:
         for S in (2, 4, 8):
             info = fi.resolve_tactic(1, n, k, fi.make_tactic(fi.KIND_GEMV, S, 0, 0), B200_SMS)
             assert info["splits"] == S
-            if k % 256:
+            if _lean_fits(k, S):
+                assert info["variant"] >> 4 == 5
+            elif k % 256:
                 assert (info["variant"] >> 4, info["ctas_per_sm"]) == (4, 2)
             else:
                 assert info["variant"] == 0x14
-        # S = 1 is not affected, and the device-sized split resolves to the same S at every m
-        assert fi.resolve_tactic(1, n, k, fi.make_tactic(fi.KIND_GEMV, 1, 0, 0), B200_SMS)["variant"] >> 4 == 1
+        # S = 1: the lean pipeline where it fits, else the stream pipeline; the device-sized split
+        # resolves to the same S at every m
+        v1 = fi.resolve_tactic(1, n, k, fi.make_tactic(fi.KIND_GEMV, 1, 0, 0), B200_SMS)["variant"] >> 4
+        assert v1 == (5 if _lean_fits(k, 1) else 1)
         s1 = fi.resolve_tactic(1, n, k, fi.make_tactic(fi.KIND_GEMV, 0, 0, 0), B200_SMS)["splits"]
         s4 = fi.resolve_tactic(4, n, k, fi.make_tactic(fi.KIND_GEMV, 0, 0, 0), B200_SMS)["splits"]
         assert s1 == s4
     # where those row groups would leave SMs with fewer than 4 warps, the stream pipeline keeps
-    # its own row choice (n = 300: 75 four-row groups per split)
-    for S in (2, 4):
-        info = fi.resolve_tactic(1, 300, 4096, fi.make_tactic(fi.KIND_GEMV, S, 0, 0), B200_SMS)
-        assert info["variant"] >> 4 == 1 and info["variant"] & 15 != 4
+    # its own row choice (n = 280: 70 four-row groups per split, 560 warps over 8 splits; S = 8
+    # has no whole lean iterations at k = 4096)
+    info = fi.resolve_tactic(1, 280, 4096, fi.make_tactic(fi.KIND_GEMV, 8, 0, 0), B200_SMS)
+    assert info["variant"] >> 4 == 1 and info["variant"] & 15 != 4
     assert fi.resolve_tactic(1, 129, 2688, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0), B200_SMS)["variant"] >> 4 == 1
     # explicit rows or pipeline are taken as given
     assert fi.resolve_tactic(1, 4096, 14336, fi.make_tactic(fi.KIND_GEMV, 2, 0, 0x12), B200_SMS)["variant"] == 0x12
@@ -333,3 +358,25 @@ def test_binding_checks_shapes_and_devices_before_any_launch():
                 (Wq, Ws, torch.empty(1, dtype=torch.float64))]:
         with pytest.raises(ValueError):
             fi._pack_out_check(W, bad)
+
+
+def _tuned_entries():
+    """The rows of the generated default-tactic table (csrc/tactic_table.inc)."""
+    import os
+    import re
+    path = os.path.join(os.path.dirname(fi.__file__), "csrc", "tactic_table.inc")
+    text = open(path).read()
+    rows = re.findall(r"\{(\d+), (\d+), (\d+), (\d+), (\d+), (0x[0-9a-f]+), ([0-9.]+)\}", text)
+    return [tuple(int(v, 0) for v in r[:6]) for r in rows if int(r[0]) > 0]
+
+
+def test_tuned_table_picks_are_the_defaults_and_valid_for_their_whole_bucket():
+    """Every generated entry is what the default resolves to for its (n, k, SMs) at every m of its
+    bucket, it resolves at every such m, and its K split does not change inside the bucket (so
+    the default stays batch-invariant within it)."""
+    for n, k, m_lo, m_hi, sms, t in _tuned_entries():
+        splits = set()
+        for m in sorted({m_lo, (m_lo + m_hi) // 2, m_hi} | set(range(m_lo, min(m_hi, m_lo + 4) + 1))):
+            assert fi.default_tactic(m, n, k, sms) == t, (n, k, m)
+            splits.add(fi.resolve_tactic(m, n, k, t, sms)["splits"])
+        assert len(splits) == 1, (n, k, m_lo, m_hi, splits)

@@ -150,10 +150,12 @@ def test_rows_per_stage_and_occupancy_do_not_change_bits():
 
 
 def test_pipelines_give_identical_bits():
-    """The per-warp async-copy pipeline, the producer-warp ring, the overlapped variant and the
-    register pipeline run the same per-chunk arithmetic in the same order, so for one S their
-    outputs are bitwise equal."""
-    for m, n, k in [(1, 2048, 7168), (3, 1000, 4096), (8, 515, 2688), (32, 300, 2048)]:
+    """The per-warp async-copy pipeline, the producer-warp ring, the overlapped variant, the
+    register pipeline and the lean stream pipeline run the same per-chunk arithmetic in the
+    same order, so for one S their outputs are bitwise equal."""
+    # (1, 20000, 2048): several row groups per warp
+    for m, n, k in [(1, 2048, 7168), (3, 1000, 4096), (8, 515, 2688), (32, 300, 2048), (1, 333, 4096), (1, 97, 8192),
+                    (1, 20000, 2048)]:
         A = inputs.activations(m, k, seed=21, outliers=True)
         dw = _gpu.device_weights(n, k, 2)
         for S in (1, 2, 5):
@@ -162,11 +164,13 @@ def test_pipelines_give_identical_bits():
             except fi.FiError as e:  # activations of this split do not fit half an SM
                 assert e.status == -2
                 continue
-            for var in (0x20, 0x30, 0x40, 0x41):
+            for var in (0x20, 0x30, 0x40, 0x41, 0x50, 0x51, 0x52, 0x54):
                 try:
                     other = _mm(A, dw, fi.make_tactic(GEMV, S, 0, var))
-                except fi.FiError as e:  # the overlapped variant's half SM cannot hold these activations
-                    assert e.status == -2 and var == 0x30, (m, n, k, S, hex(var))
+                except fi.FiError as e:
+                    # the overlapped variant's half SM cannot hold these activations; the lean
+                    # pipeline takes m = 1 with k % 256 == 0 and splits of whole items only
+                    assert e.status == -2 and (var == 0x30 or var >> 4 == 5), (m, n, k, S, hex(var))
                     continue
                 assert np.array_equal(stream, other), (m, n, k, S, hex(var))
 
@@ -244,6 +248,23 @@ def test_lm_head_m1_sampled():
     cols = np.concatenate([np.arange(0, n, 97), [n - 1]])
     ref = oracle.mm(A, Wq, Ws, g, cols=cols)
     _gpu.assert_within_tolerance(got[:, cols], ref, "lm_head m=1 (every 97th column)")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("n,k", inputs.QWEN36_27B_DECODE)
+def test_qwen36_27b_decode_shapes_default_sampled(n, k):
+    """The second workload (PR #4038's Qwen3.6-27B-NVFP4 decode GEMMs at m = 1, synthetic weights):
+    the default tactic and two split tactics at full size, every 61st output column (and the
+    last) against the oracle."""
+    A = inputs.activations(1, k, seed=2)
+    W, (Wq, Ws, g) = _gpu.weights(n, k, 2)
+    dw = fi.pack_weights(torch.from_numpy(W).cuda())
+    cols = np.concatenate([np.arange(0, n, 61), [n - 1]])
+    ref = oracle.mm(A, Wq, Ws, g, cols=cols)
+    for t in (fi.TACTIC_DEFAULT, fi.make_tactic(GEMV, 2, 0, 0), fi.make_tactic(GEMV, 0, 0, 0)):
+        _gpu.assert_within_tolerance(_mm(A, dw, t)[:, cols], ref, f"{n}x{k} {t}")
+    del dw
+    torch.cuda.empty_cache()
 
 
 # ------------------------------------------------------------------- split-K reduce

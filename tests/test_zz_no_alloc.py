@@ -6,8 +6,9 @@ split-K workspace, and may own no buffer to lend it either. fi_mm_bf16_fp4_noall
 split-K partials in a static device array of the library instead. These tests call it
 through the C ABI and hold it to the allocating entry point, fi_mm_bf16_fp4: two split-K
 calls in a row (the second with another shape, over the partials the first one left
-behind) must both agree within the parity tolerance used by the other GPU tests, and a call
-whose partials would not fit the array must be refused before anything is launched.
+behind) must give exactly the bits of the allocating call with the same tactic (both run the
+same kernels; only where the partials live differs), and a call whose partials would not fit
+the array must be refused before anything is launched.
 
 This file sorts last so that a run which stops at the first failure has run every other
 test first; it passes on its own in a fresh process as well.
@@ -57,8 +58,7 @@ def test_two_calls_in_a_row_match_the_allocating_entry_point(splits):
         assert st == 0, fi.last_error()
         ref = _allocating(A, Wq, Ws, g, tactic)
         torch.cuda.synchronize()
-        _gpu.assert_within_tolerance(_gpu.host_bits(out), _gpu.bits_to_f64(_gpu.host_bits(ref)),
-                                     f"no-alloc vs allocating, m={m} n={n} k={k} S={splits}")
+        assert np.array_equal(_gpu.host_bits(out), _gpu.host_bits(ref)), f"m={m} n={n} k={k} S={splits}"
 
 
 def test_single_split_needs_no_scratch():
@@ -70,7 +70,7 @@ def test_single_split_needs_no_scratch():
     assert _noalloc(A, Wq, Ws, g, out, tactic) == 0, fi.last_error()
     ref = _allocating(A, Wq, Ws, g, tactic)
     torch.cuda.synchronize()
-    _gpu.assert_within_tolerance(_gpu.host_bits(out), _gpu.bits_to_f64(_gpu.host_bits(ref)), "single split")
+    assert np.array_equal(_gpu.host_bits(out), _gpu.host_bits(ref)), "single split"
 
 
 def test_partials_beyond_the_static_scratch_are_refused():
@@ -106,3 +106,29 @@ def test_default_tactic_falls_back_to_a_split_that_fits():
     assert st == 0, fi.last_error()
     torch.cuda.synchronize()
     _gpu.assert_within_tolerance(_gpu.host_bits(out)[:, cols], ref, "no-alloc default, m=32")
+
+
+def test_default_falls_back_to_a_single_split_gemv():
+    """lm_head-like 152064 x 5120 at m = 4: the default (GEMV with two K splits) needs about
+    4.9 MB of partials; the only smaller split, S = 1, needs no scratch at all and must be the
+    one taken. Its bits equal the allocating call's with that tactic, and it stays within
+    tolerance of the oracle on sampled columns."""
+    m, n, k = 4, 152064, 5120
+    info = fi.resolve_tactic(m, n, k, fi.TACTIC_DEFAULT)
+    assert info["kind"] == fi.KIND_GEMV and info["splits"] > 1 and info["workspace_bytes"] > SCRATCH_BYTES
+    fallback = fi.make_tactic(fi.KIND_GEMV, 1, 0, 0)  # the automatic pipeline: any S = 1 GEMV gives these bits
+    fb = fi.resolve_tactic(m, n, k, fallback)
+    assert fb["splits"] == 1 and fb["workspace_bytes"] == 0
+    A_bits = inputs.activations(m, k, seed=4)
+    W, (Wq_o, Ws_o, g_o) = _gpu.weights(n, k, 0, True)
+    Wq, Ws, g = _gpu.device_weights(n, k, 0, True)
+    A = _gpu.dev_bf16(A_bits)
+    out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    st = _noalloc(A, Wq, Ws, g, out, fi.TACTIC_DEFAULT)
+    assert st == 0, fi.last_error()
+    ref = _allocating(A, Wq, Ws, g, fallback)
+    torch.cuda.synchronize()
+    got = _gpu.host_bits(out)
+    assert np.array_equal(got, _gpu.host_bits(ref))
+    cols = np.concatenate([np.arange(0, n, 499), [n - 1]])
+    _gpu.assert_within_tolerance(got[:, cols], oracle.mm(A_bits, Wq_o, Ws_o, g_o, cols=cols), "no-alloc m=4 lm_head")
