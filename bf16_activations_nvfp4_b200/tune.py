@@ -48,7 +48,7 @@ def default_shapes():
 
 def time_tactic(fi, torch, stream, A, copies, g, out, tactic, ws) -> float:
     """Median µs per call of `tactic` over PDL-chained graph replays, every call on its own weight copy."""
-    nrep = max(2, 2 * len(copies))
+    nrep = max(2, len(copies))  # one pass over the copies: every call on weights not in L2
     with torch.cuda.stream(stream):
         fi.mm_bf16_fp4(A, copies[0][0], copies[0][1], g, tactic=tactic, out=out, workspace=ws)
         torch.cuda.synchronize()
