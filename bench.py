@@ -52,8 +52,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per launch of the GEMV kernel (dram__bytes_read.sum + dram__bytes_write.sum)
 # from one ncu capture per shape, keyed by the sha256 of the kernel code they were taken on
 # (comments excluded); ignored (traffic = null) when that code has changed since.
-NCU_TRAFFIC = {"source_sha256": "57a8d32ff78458b5ee5bf631504ab7a3e47c1303506de4d74c6a0c8475536fb0",
-               "bytes": {"14336x4096": 33_104_677, "4096x14336": 33_125_120}}
+NCU_TRAFFIC = {"source_sha256": "a99dfc7674f8a00b7d7729ba7f7462fd7a114e51eaa244746630eceda2b810b4",
+               "bytes": {"4096x14336": 33_109_760, "14336x4096": 33_083_648}}
 # the roofline's dominant-kernel figure: the GEMV alone (split 1, one launch per call) on the
 # two 33 MB serving shapes
 ROOFLINE_SHAPES = [(4096, 14336), (14336, 4096)]
@@ -355,6 +355,33 @@ def run_fi(args, rank: int, world: int) -> dict | None:
     torch.cuda.synchronize(dev)
     e2e_us = x0.elapsed_time(x1) * 1e3
 
+    # host cost per call on the 4096 x 14336 default: the public op (binding + C ABI) and the bare
+    # C-ABI call with its arguments prepared once, each issued back to back without synchronising
+    # (the launch queue absorbs them); the GPU work is the same in both
+    host_us = {}
+    with torch.cuda.stream(stream):
+        hi = next((i for i, sh in enumerate(shapes) if (sh["n"], sh["k"]) == (4096, 14336)), 0)
+        sh = shapes[hi]
+        Wq, Ws = sh["copies"][0]
+        t_def = fi.default_tactic(M, sh["n"], sh["k"])
+        reps = 200
+        for label in ("public_op", "c_abi"):
+            torch.cuda.synchronize(dev)
+            if label == "public_op":
+                t0 = time.perf_counter()
+                for _ in range(reps):
+                    fi.mm_bf16_fp4(sh["A"], Wq, Ws, sh["g"], tactic=t_def, out=sh["out"])
+                t1 = time.perf_counter()
+            else:
+                lib = fi.library()
+                cargs = (sh["A"].data_ptr(), Wq.data_ptr(), Ws.data_ptr(), sh["g"].data_ptr(), sh["out"].data_ptr(),
+                         M, sh["n"], sh["k"], t_def, stream.cuda_stream)
+                t0 = time.perf_counter()
+                for _ in range(reps):
+                    lib.fi_mm_bf16_fp4(*cargs)
+                t1 = time.perf_counter()
+            host_us[label] = round((t1 - t0) / reps * 1e6, 2)
+        torch.cuda.synchronize(dev)
     total_us, e2e_us = max_over_ranks([total_us, e2e_us], world, dev)
     step_bytes = sum(shapes[c["shape"]]["bytes"] for c in calls)
     value = replica_value(step_bytes, args.steps, world, total_us)
@@ -420,7 +447,9 @@ def run_fi(args, rank: int, world: int) -> dict | None:
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": sum(2 * M * shapes[c["shape"]]["k"] for c in calls),
                 "d2h_bytes_per_step": sum(2 * M * shapes[c["shape"]]["n"] for c in calls),
-                "how": "eager public-op calls; per call a pinned H2D copy of A, the op, a D2H copy of out"},
+                "how": "eager public-op calls; per call a pinned H2D copy of A, the op, a D2H copy of out",
+                "host_us_per_call": dict(host_us, shape="4096x14336 default tactic",
+                                         how="200 calls issued back to back, host wall time per call")},
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,

@@ -459,9 +459,17 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
   return FI_OK;
 }
 
-// MMA tactic: splits 1..k/64 (0 = device-sized), CTAs per SM 0 or 1, variant 0. Needs m <= 256
-// and k a multiple of 64; the workspace holds the f16 activations and their row scales, then
-// the [S, m, n] fp32 partials when S > 1.
+// MMA tactic: splits 1..k/64 (0 = device-sized), CTAs per SM 0 or 1, variant 0 (automatic), 1
+// (activations converted by a prepass kernel into the workspace) or 2 (converted by the kernel
+// into shared memory, "resident"; only where the split's slice fits, m <= 128). Every CTA then
+// converts its split's slice while its decode warps start on the weights; that saves the
+// prepass launch (about 3 us in a chained sequence of calls on B200) but costs the CTA time in
+// proportion to m_pad x its steps, once per wave. Measured on B200 (4096 x 4096 at m = 8, S = 8:
+// 10.1 against 11.4 us; 4096 x 14336 at m = 32, S = 8: 28.4 against 24.4 us), so automatic
+// takes it only for one-wave grids (tiles x S <= SMs) with m_pad = 16 and at most 16 steps per
+// split. Needs m <= 256 and k a multiple of 64; the workspace holds the f16
+// activations and their (row, split) scales in prepass mode, then the [S, m, n] fp32 partials
+// when S > 1. Both modes give the same bits.
 static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var, int sms,
                        fi_tactic_info* out) {
   if (m > kMmaMaxM)
@@ -469,8 +477,8 @@ static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req,
   if (k % kMmaKStep != 0)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA tactics need k to be a multiple of %d (got k=%lld)", kMmaKStep,
                      (long long)k);
-  if (ctas_req > 1 || var != 0)
-    return set_error(FI_ERR_INVALID_ARG, "MMA tactics take CTAs per SM 0/1 and variant 0");
+  if (ctas_req > 1 || var > 2)
+    return set_error(FI_ERR_INVALID_ARG, "MMA tactics take CTAs per SM 0/1 and variant 0, 1 or 2");
   const int64_t tiles = std::max<int64_t>(1, (n + kMmaTileRows - 1) / kMmaTileRows);
   const int64_t KS = k / kMmaKStep;
   int64_t S = S_req;
@@ -497,15 +505,28 @@ static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req,
     }
   }
   if (S < 1) S = 1;
+  const int m_pad = mma_m_pad(std::max<int64_t>(m, 1));
+  const bool fits = mma_act_resident(m_pad, k, (int)S);
+  if (var == 2 && !fits)
+    return set_error(FI_ERR_UNSUPPORTED_SHAPE,
+                     "MMA resident activations: m=%lld rows of %lld k over %lld splits do not fit shared memory",
+                     (long long)m, (long long)k, (long long)S);
+  const int64_t steps = (KS + S - 1) / S;
+  const bool resident = var == 2 || (var == 0 && fits && tiles * S <= sms && m_pad == 16 && steps <= 16);
   out->kind = FI_KIND_MMA;
   out->splits = (int32_t)S;
   out->ctas_per_sm = 1;
-  out->variant = 0;
+  out->variant = resident ? 2 : 1;
   out->grid_x = (int32_t)tiles;
   out->grid_y = (int32_t)S;
   out->threads = kMmaThreads;
-  out->smem_bytes = (int32_t)mma_smem_bytes(mma_m_pad(m));
-  out->workspace_bytes = (m > 0 && k > 0) ? (S > 1 ? mma_partials_offset(m, k) + S * m * n * 4 : mma_workspace_bytes(m, k)) : 0;
+  out->smem_bytes = (int32_t)(resident ? mma_resident_smem_bytes(m_pad, k, (int)S) : mma_smem_bytes(m_pad));
+  if (m <= 0 || k <= 0)
+    out->workspace_bytes = 0;
+  else if (resident)
+    out->workspace_bytes = S > 1 ? S * m * n * 4 : 0;
+  else
+    out->workspace_bytes = S > 1 ? mma_partials_offset(m, k, S) + S * m * n * 4 : mma_workspace_bytes(m, k, S);
   return FI_OK;
 }
 
@@ -684,16 +705,26 @@ static int mm_run(const uint16_t* A, const uint8_t* Wq, const uint8_t* Wscale, c
     a.out = out;
     a.out_f16 = out_f16 ? 1 : 0;
     uint8_t* ws = reinterpret_cast<uint8_t*>(partials);
-    a.a16 = reinterpret_cast<uint16_t*>(ws);
-    a.rs = reinterpret_cast<float*>(ws + mma_rs_offset(m, k));
     a.m = m;
     a.n = n;
     a.k = k;
     a.m_pad = mma_m_pad(m);
     a.splits = info.splits;
-    a.partials = reinterpret_cast<float*>(ws + mma_partials_offset(m, k));
-    a.op_stages = mma_op_stages(a.m_pad);
-    a.stage_bytes = (uint32_t)mma_stage_bytes(a.m_pad);
+    a.act_resident = info.variant == 2 ? 1 : 0;
+    if (a.act_resident) {
+      // the kernel converts the activations into shared memory: the workspace is the partials
+      a.partials = reinterpret_cast<float*>(ws);
+      a.op_stages = kMmaMaxOpStages;
+      a.stage_bytes = 0;
+      a.act_bytes = (uint32_t)mma_resident_act_bytes(a.m_pad, k, info.splits);
+      a.act_extra_bytes = (uint32_t)mma_resident_extra_bytes(a.m_pad);
+    } else {
+      a.a16 = reinterpret_cast<uint16_t*>(ws);
+      a.rs = reinterpret_cast<float*>(ws + mma_rs_offset(m, k));
+      a.partials = reinterpret_cast<float*>(ws + mma_partials_offset(m, k, info.splits));
+      a.op_stages = mma_op_stages(a.m_pad);
+      a.stage_bytes = (uint32_t)mma_stage_bytes(a.m_pad);
+    }
     a.debug_stall = g_debug_stall_launches > 0 ? 1 : 0;
     if (g_debug_stall_launches > 0) --g_debug_stall_launches;
     a.err = device_error_word();

@@ -104,18 +104,25 @@ int launch_gemv(const GemvArgs& a, cudaStream_t stream);
 int gemv_read_error(unsigned* bits);
 
 // ------------------------------------------------------------------------- MMA
-// Tensor-core path: one CTA per kMmaTileRows weight rows, 64 k per pipeline step, activations
-// converted to f16 (times a per-row power of two) in the workspace: a16 [m_pad, k] then
-// rs [m_pad] fp32 at the next 256-byte boundary.
+// Tensor-core path: one CTA per kMmaTileRows weight rows, 64 k per pipeline step. The
+// activations are converted to f16 times a power of two per (row, K split): either by a prepass
+// kernel into the workspace (a16 [m_pad, k], then rs [splits, m_pad] fp32 at the next 256-byte
+// boundary, then the split-K partials) or, when the split's slice fits shared memory next to the
+// raw-code ring ("resident" mode, m_pad <= kMmaTmemMaxM), by the kernel's decode warps into
+// shared memory, in which case the workspace holds only the partials.
 constexpr int kMmaTileRows = 256;
 constexpr int kMmaKStep = 64;
 constexpr int kMmaMaxM = 256;
 constexpr int kMmaThreads = 24 * 32;
 inline int mma_m_pad(int64_t m) { return (int)((m + 15) / 16 * 16); }
 inline int64_t mma_rs_offset(int64_t m, int64_t k) { return round_up((int64_t)mma_m_pad(m) * k * 2, 256); }
-inline int64_t mma_workspace_bytes(int64_t m, int64_t k) { return mma_rs_offset(m, k) + (int64_t)mma_m_pad(m) * 4; }
+inline int64_t mma_workspace_bytes(int64_t m, int64_t k, int64_t splits) {
+  return mma_rs_offset(m, k) + (int64_t)mma_m_pad(m) * 4 * splits;
+}
 // split-K partials [splits, m, n] fp32 follow the activations at the next 256-byte boundary
-inline int64_t mma_partials_offset(int64_t m, int64_t k) { return round_up(mma_workspace_bytes(m, k), 256); }
+inline int64_t mma_partials_offset(int64_t m, int64_t k, int64_t splits) {
+  return round_up(mma_workspace_bytes(m, k, splits), 256);
+}
 // operand stages (decoded weights + activation tile of one 64-k step): as many as fit, 2..4
 constexpr int kMmaMaxOpStages = 4;
 // m_pad <= kMmaTmemMaxM: the decoded weights live in tensor memory, a stage is the activation
@@ -126,6 +133,13 @@ inline int64_t mma_stage_bytes(int m_pad) {
 }
 int mma_op_stages(int m_pad);
 int64_t mma_smem_bytes(int m_pad);
+// Resident mode: the bytes of a split's activation slice (steps x m_pad x 128, the largest split
+// of `splits` over k/64 steps) and of the row scales after it; the mode is taken when
+// m_pad <= kMmaTmemMaxM and it fits shared memory next to the raw-code ring.
+int64_t mma_resident_act_bytes(int m_pad, int64_t k, int splits);
+inline int64_t mma_resident_extra_bytes(int m_pad) { return round_up((int64_t)m_pad * 4, 16); }
+bool mma_act_resident(int m_pad, int64_t k, int splits);
+int64_t mma_resident_smem_bytes(int m_pad, int64_t k, int splits);
 
 struct MmaArgs {
   const uint16_t* A;
@@ -141,7 +155,10 @@ struct MmaArgs {
   int splits;           // K splits (grid.y); > 1 writes fp32 partials [splits, m, n] to `partials`
   float* partials;
   int op_stages;        // operand stages in shared memory (mma_op_stages)
-  uint32_t stage_bytes; // bytes of one operand stage (mma_stage_bytes)
+  uint32_t stage_bytes; // bytes of one operand stage (mma_stage_bytes; 0 in resident mode)
+  int act_resident;     // the decode warps convert the split's activations into shared memory
+  uint32_t act_bytes;   // resident mode: bytes of the activation slice (mma_resident_act_bytes)
+  uint32_t act_extra_bytes;  // resident mode: row scales (mma_resident_extra_bytes)
   int debug_stall;      // test hook: the producer issues nothing (the waits time out)
   unsigned* err;        // the device error word
   uint64_t timeout_ns;  // limit of every mbarrier wait

@@ -6,15 +6,20 @@
 //  * Operands. tcgen05.mma kind::f16 needs both operands of one 16-bit type. The weights are
 //    decoded to f16 (every E2M1 value times its E4M3 block scale is exact in f16: at most 6
 //    significant bits, magnitudes 2^-10 .. 2688); the activations are converted once per call
-//    by act_to_f16_kernel to f16 times a per-row power of two that puts the row maximum in
-//    [2^14, 2^15) (exact for every element within 2^29 of its row maximum), so the tensor core
-//    accumulates sum_k W'[i][k] * A'[j][k] in fp32 and one per-row factor undoes the scale.
+//    to f16 times a power of two per (row, K split) that puts the maximum of the row's split
+//    range in [2^14, 2^15) (exact for every element within 2^29 of that maximum), so the tensor
+//    core accumulates sum_k W'[i][k] * A'[j][k] in fp32 and one factor per (row, split) undoes
+//    the scale. The conversion runs in act_to_f16_kernel into the workspace, or, when the
+//    split's slice fits shared memory (m_pad <= 128), in otherwise idle warps at kernel start
+//    ("resident" activations: no second launch and no per-step activation copies); both use
+//    the same arithmetic and give the same bits.
 //  * Roles (one CTA per 256 weight rows, 24 warps):
 //      warp 0      TMA producer of the raw codes of the tile (256 rows x 32 bytes per 64-k step)
 //                  into a 4-stage ring, issued before the grid-dependency wait (weights never
 //                  depend on the preceding kernel);
 //      warp 18     TMA producer of the f16 activation tiles (m_pad rows x 64 k, 128-byte
 //                  swizzled) into the operand stages (2 to 4, as many as shared memory holds);
+//                  with resident activations it converts them instead, with warps 19-22;
 //      warps 2-17  decode: two threads per weight row (32 k each), codes -> f16 (cvt.rn.f16x2.e2m1x2) times
 //                  the block scale (exact f16 multiply), stored in the 128-byte-swizzled
 //                  K-major layout the MMA reads; the block scales are loaded 8-11 steps ahead;
@@ -22,7 +27,8 @@
 //                  allocates TMEM): per 64-k step 4 K=16 steps, N = m_pad, accumulating in
 //                  TMEM; tcgen05.commit frees the stage once both halves have read it;
 //      warps 19-22 epilogue: tcgen05.ld of the accumulator, out[j][i] = round(D[i][j] *
-//                  rs[j] * gscale) to bf16 (or f16).
+//                  rs[j] * gscale) to bf16 (or f16); with resident activations they first
+//                  convert them (warp 18 too), while the decode warps start on the weights.
 //  * The weight tile is decoded once per call (the activations, m_pad <= 256 rows, are one MMA
 //    N tile), so the decode work is one cvt and one f16 multiply per two codes.
 //  * Every wait is bounded (see sync.cuh); on a timeout the roles stop, the MMA issuer and the
@@ -50,6 +56,9 @@ constexpr int kWarpTma = 0, kWarpMma = 1, kWarpDq0 = 2, kDqWarps = 16, kWarpAct 
 static_assert((kWarpMma2 + 1) * 32 == kMmaThreads, "warp roles cover the CTA");
 static_assert(kWarpDq0 + kDqWarps == kWarpAct && kWarpAct + 1 == kWarpEpi0 && kDqWarps * 32 == 2 * kMmaTileRows,
               "two decode threads per tile row");
+// resident activations: converted by the activation producer and epilogue warps (18-22)
+constexpr int kConvWarps = kEpiWarps + 1;
+static_assert(kWarpAct + kConvWarps == kWarpMma2, "converting warps: 18 .. 22");
 constexpr int kRawStages = 4;
 constexpr uint32_t kRawBytes = kMmaTileRows * 32;  // 256 rows x 32 code bytes
 constexpr uint32_t kWopBytes = kMmaTileRows * 128;  // 256 rows x 64 f16, 128-byte swizzled
@@ -151,29 +160,55 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
 
 }  // namespace
 
-// A[m, k] bf16 -> a16[m_pad, k] f16 scaled by a per-row power of two (row maximum in
-// [2^14, 2^15)); rs[row] = the inverse scale. Rows m .. m_pad-1 are zero.
+// The activation conversion shared by the prepass kernel and the kernel's resident mode, so
+// that both give the same bits. Per (activation row, K split): the largest biased exponent of
+// the row's bf16 values over the split's k range sets a power of two that puts the maximum in
+// [2^14, 2^15); every value times it is rounded to f16, and the epilogue multiplies by the
+// inverse (exact).
+__device__ __forceinline__ uint32_t bf16x8_max_exp(const uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t e = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) e = max(e, max((w[q] >> 7) & 0xFFu, (w[q] >> 23) & 0xFFu));
+  return e;
+}
+
+__device__ __forceinline__ int act_shift(uint32_t e_max) {
+  const int sh = 141 - (int)e_max;  // biased exponent E of the maximum -> [2^14, 2^15)
+  return sh < -126 ? -126 : (sh > 126 ? 126 : sh);
+}
+
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, float up) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t h[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    h[q] = f32x2_to_f16x2(__uint_as_float(w[q] << 16) * up, __uint_as_float(w[q] & 0xFFFF0000u) * up);
+  return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+// A[m, k] bf16 -> a16[m_pad, k] f16, block (row, split) over the split's k range (64-k steps
+// [s KS/S, (s+1) KS/S)), scaled by the per-(row, split) power of two above; rs[split][row] =
+// the inverse scale. Rows m .. m_pad-1 are zero.
 __global__ void __launch_bounds__(256) act_to_f16_kernel(const uint16_t* __restrict__ A, int64_t m, int64_t k,
                                                          uint16_t* __restrict__ a16, float* __restrict__ rs) {
   pdl_launch_dependents();
   pdl_wait();
   const int64_t row = blockIdx.x;
+  const int m_pad = (int)gridDim.x, S = (int)gridDim.y, sp = (int)blockIdx.y;
+  const int64_t KS_all = k / kMmaKStep;
+  const int64_t kb = sp * KS_all / S * kMmaKStep, ke = (sp + 1) * KS_all / S * kMmaKStep;
   const int tid = threadIdx.x;
-  uint4* dst = reinterpret_cast<uint4*>(a16 + row * k);
-  const int64_t n8 = k / 8;  // 16-byte groups of the row
+  uint4* dst = reinterpret_cast<uint4*>(a16 + row * k + kb);
+  const int64_t n8 = (ke - kb) / 8;  // 16-byte groups of the row's split range
   if (row >= m) {
     for (int64_t i = tid; i < n8; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
-    if (tid == 0) rs[row] = 0.0f;
+    if (tid == 0) rs[(int64_t)sp * m_pad + row] = 0.0f;
     return;
   }
-  const uint4* src = reinterpret_cast<const uint4*>(A + row * k);
+  const uint4* src = reinterpret_cast<const uint4*>(A + row * k + kb);
   uint32_t e = 0;
-  for (int64_t i = tid; i < n8; i += blockDim.x) {
-    const uint4 v = ldg_v4(src + i);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) e = max(e, max((w[q] >> 7) & 0xFFu, (w[q] >> 23) & 0xFFu));
-  }
+  for (int64_t i = tid; i < n8; i += blockDim.x) e = max(e, bf16x8_max_exp(ldg_v4(src + i)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
   __shared__ uint32_t red[8];
@@ -182,19 +217,10 @@ __global__ void __launch_bounds__(256) act_to_f16_kernel(const uint16_t* __restr
   e = 0;
 #pragma unroll
   for (int w = 0; w < 8; ++w) e = max(e, red[w]);
-  int sh = 141 - (int)e;  // biased exponent E of the row maximum -> [2^14, 2^15)
-  sh = sh < -126 ? -126 : (sh > 126 ? 126 : sh);
+  const int sh = act_shift(e);
   const float up = __uint_as_float((uint32_t)(sh + 127) << 23);
-  for (int64_t i = tid; i < n8; i += blockDim.x) {
-    const uint4 v = ldg_v4(src + i);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t h[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      h[q] = f32x2_to_f16x2(__uint_as_float(w[q] << 16) * up, __uint_as_float(w[q] & 0xFFFF0000u) * up);
-    dst[i] = make_uint4(h[0], h[1], h[2], h[3]);
-  }
-  if (tid == 0) rs[row] = __uint_as_float((uint32_t)(127 - sh) << 23);
+  for (int64_t i = tid; i < n8; i += blockDim.x) dst[i] = bf16x8_to_f16x8(ldg_v4(src + i), up);
+  if (tid == 0) rs[(int64_t)sp * m_pad + row] = __uint_as_float((uint32_t)(127 - sh) << 23);
 }
 
 // TA: the decoded weights go to tensor memory (tcgen05.st) and the MMAs read A from there
@@ -214,7 +240,14 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   const uint32_t raw_s = smem_addr(smem_raw);
   const uint32_t base = (raw_s + 1023u) & ~1023u;
   uint8_t* const basep = smem_raw + (base - raw_s);
-  uint64_t* const bars = reinterpret_cast<uint64_t*>(basep + kRawStages * kRawBytes + (uint32_t)NST * stage_bytes);
+  // resident activations (p.act_resident): the split's whole f16 activation slice, one
+  // 128-byte-swizzled tile of m_pad rows x 64 k per step, then the per-row inverse scales
+  const bool resident = p.act_resident != 0;
+  const uint32_t act_res = base + kRawStages * kRawBytes + (uint32_t)NST * stage_bytes;
+  float* const rs_res = reinterpret_cast<float*>(basep + kRawStages * kRawBytes + (uint32_t)NST * stage_bytes +
+                                                 p.act_bytes);
+  uint64_t* const bars = reinterpret_cast<uint64_t*>(basep + kRawStages * kRawBytes + (uint32_t)NST * stage_bytes +
+                                                     p.act_bytes + p.act_extra_bytes);
   uint64_t* const raw_full = bars;
   uint64_t* const raw_empty = bars + kRawStages;
   uint64_t* const act_full = bars + 2 * kRawStages;
@@ -245,7 +278,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       mbar_init(&raw_empty[i], kDqWarps);
     }
     for (int i = 0; i < NST; ++i) {
-      mbar_init(&act_full[i], 1);
+      // resident mode: act_full[0] completes once, when the converting warps are done, and
+      // act_full[1] once, when the copies of the split's bf16 activations have landed
+      mbar_init(&act_full[i], resident && i == 0 ? kConvWarps : 1);
       mbar_init(&op_full[i], kDqWarps);
       mbar_init(&op_empty[i], 2);  // both MMA issuers commit
     }
@@ -265,6 +300,59 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = tmem_slot;
   pdl_launch_dependents();
+
+  if (resident && warp >= kWarpAct && warp < kWarpAct + kConvWarps) {
+    // ----------------------------------------------------------- resident activations
+    // The activation producer and epilogue warps (idle until the accumulator is complete)
+    // convert the split's activations while the decode warps start on the weights. Each warp
+    // owns whole rows (no atomics, no barrier between warps): A over k [64 ks0, 64 (ks0 + KS))
+    // lands as bf16 in the swizzled tiles the MMA reads (one 128-byte-swizzled tile of N rows x
+    // 64 k per step, one TMA copy each, all in flight at once; rows m..N-1 zero), then each
+    // row's largest exponent over the split (a warp reduction), then the in-place conversion
+    // to f16 with the per-(row, split) scale (the prepass kernel's arithmetic). A is written
+    // by the preceding kernel.
+    pdl_wait();
+    const int cw = warp - kWarpAct;   // 0 .. kConvWarps - 1: this warp converts rows cw, cw + 5, ...
+    const int per_row = KS * 8;       // 16-byte pieces of a row's split range
+    if (cw == 0 && lane == 0) {
+      // the split's bf16 tiles, one TMA copy per step (rows m..N-1 read as zeros)
+      mbar_arrive_expect_tx(&act_full[1], (uint32_t)KS * (uint32_t)(N * 128));
+      for (int s = 0; s < KS; ++s)
+        tma_load_2d(act_res + (uint32_t)s * (uint32_t)(N * 128), &tmap_a, (ks0 + s) * kMmaKStep, 0,
+                    smem_addr(&act_full[1]));
+    }
+    auto piece_addr = [&](int j, int c) {
+      const int st = c >> 3, cc = c & 7;  // step, 16-byte chunk within the row's 128 bytes
+      return act_res + (uint32_t)st * (uint32_t)(N * 128) + (uint32_t)(j >> 3) * 1024u + (uint32_t)(j & 7) * 128u +
+             ((uint32_t)(cc ^ (j & 7)) << 4);
+    };
+    // every copy must land before the conversion reads it or the CTA exits, abort or not
+    drain_wait(&act_full[1], 0u, p.timeout_ns, p.err);
+    for (int j = cw; j < N; j += kConvWarps) {
+      if (j >= m) {
+        if (lane == 0) rs_res[j] = 0.0f;
+        continue;
+      }
+      uint32_t e = 0;
+#pragma unroll 4
+      for (int c = lane; c < per_row; c += 32) e = max(e, bf16x8_max_exp(lds_v4m(piece_addr(j, c))));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
+      const int sh = act_shift(e);
+      const float up = __uint_as_float((uint32_t)(sh + 127) << 23);
+#pragma unroll 4
+      for (int c = lane; c < per_row; c += 32) {
+        const uint32_t a = piece_addr(j, c);
+        const uint4 h = bf16x8_to_f16x8(lds_v4m(a), up);
+        sts_v4(a, h.x, h.y, h.z, h.w);
+      }
+      if (lane == 0) rs_res[j] = __uint_as_float((uint32_t)(127 - sh) << 23);
+    }
+    // make the generic-proxy stores visible to the tensor core (async proxy)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&act_full[0]);
+  }
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------------------ producers
@@ -295,7 +383,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   } else if (warp == kWarpAct) {
     // --------------------------------------------------------------- activation producer
     // one thread streams the f16 activation tiles, gated by the MMAs freeing operand stages
-    if (lane == 0 && !p.debug_stall) {
+    if (lane == 0 && !p.debug_stall && !resident) {
       pdl_wait();  // the activations come from the conversion kernel launched just before
       int issued = 0, os = 0;
       uint32_t ph = 0;  // phase of op_empty[os] to wait for once every stage has been used
@@ -420,17 +508,21 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       const uint32_t a_first = (wop_addr(0) >> 4) & 0x3FFFu, a_stride = stage_bytes >> 4;
       constexpr uint32_t kHalf = kWopBytes / 2 / 16, kAct = kWopBytes / 16;  // in 16-byte units
       uint32_t a_lo = a_first;
+      // resident mode: step s's activation tile at act_res + s * N * 128 (in 16-byte units)
+      uint32_t b_res = (act_res >> 4) & 0x3FFFu;
+      const uint32_t b_res_step = (uint32_t)N * 8u;
       int os = 0;
       uint32_t par = 0;  // phase of act_full[os] and op_full[os] for step s
-      for (int s = 0; s < KS; ++s) {
-        if (!mbar_wait_bounded(&act_full[os], par, &abort_flag, p.timeout_ns, p.err, 4u)) break;
+      bool go = !resident || mbar_wait_bounded(&act_full[0], 0u, &abort_flag, p.timeout_ns, p.err, 4u);
+      for (int s = 0; s < KS && go; ++s) {
+        if (!resident && !mbar_wait_bounded(&act_full[os], par, &abort_flag, p.timeout_ns, p.err, 4u)) break;
         if (!mbar_wait_bounded(&op_full[os], par, &abort_flag, p.timeout_ns, p.err, 4u)) break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t acc0 = s != 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kMmaKStep / 16; ++kk) {
           if constexpr (TA) {
-            const uint64_t bdesc = desc_fixed | (uint64_t)(a_lo + (uint32_t)kk * 2u);
+            const uint64_t bdesc = desc_fixed | (uint64_t)((resident ? b_res : a_lo) + (uint32_t)kk * 2u);
             umma_f16_ta(tmem + (uint32_t)(h * N), tmem + a_col(os, h) + (uint32_t)kk * 8u, bdesc, idesc,
                         kk != 0 ? 1u : acc0);
           } else {
@@ -441,6 +533,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         }
         umma_commit(&op_empty[os]);  // frees the stage when these MMAs have read it
         a_lo += a_stride;
+        b_res += b_res_step;
         if (++os == NST) {
           os = 0;
           par ^= 1u;
@@ -458,8 +551,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int i = q * 32 + lane;
     // warp-uniform: the TMEM loads below are collective over the warp
+    // resident mode: the row scales come from the converting warps (wait for all of them)
     const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(tmem_full, 0, &abort_flag, p.timeout_ns, p.err, 16u) &&
+                                                (!resident || mbar_wait_bounded(&act_full[0], 0u, &abort_flag,
+                                                                                p.timeout_ns, p.err, 16u)) &&
                                                 !abort_flag);
+    const float* const rsp = resident ? rs_res : p.rs + (int64_t)sp * N;  // this split's inverse row scales
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (ok) {
       const float g = *p.gscale;
@@ -477,13 +574,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
               for (int jj = 0; jj < 16; ++jj) {
                 const int j = j0 + jj;
                 if (j < m)
-                  p.out[(int64_t)j * n + row] = f32_to_out(__fmul_rn(__fmul_rn(v[jj], p.rs[j]), g), p.out_f16 != 0);
+                  p.out[(int64_t)j * n + row] = f32_to_out(__fmul_rn(__fmul_rn(v[jj], rsp[j]), g), p.out_f16 != 0);
               }
             } else {
 #pragma unroll
               for (int jj = 0; jj < 16; ++jj) {
                 const int j = j0 + jj;
-                if (j < m) part[(int64_t)j * n + row] = __fmul_rn(v[jj], p.rs[j]);
+                if (j < m) part[(int64_t)j * n + row] = __fmul_rn(v[jj], rsp[j]);
               }
             }
           }
@@ -526,20 +623,53 @@ int64_t mma_smem_bytes(int m_pad) {
          kNumBars * 8;
 }
 
+int64_t mma_resident_act_bytes(int m_pad, int64_t k, int splits) {
+  const int64_t KS_all = k / kMmaKStep;
+  const int64_t ks_max = splits > 0 ? (KS_all + splits - 1) / splits : KS_all;  // the largest split
+  return ks_max * (int64_t)m_pad * 128;
+}
+
+int64_t mma_resident_smem_bytes(int m_pad, int64_t k, int splits) {
+  return 1024 + (int64_t)kRawStages * kRawBytes + mma_resident_act_bytes(m_pad, k, splits) +
+         mma_resident_extra_bytes(m_pad) + kNumBars * 8;
+}
+
+bool mma_act_resident(int m_pad, int64_t k, int splits) {
+  return m_pad <= kMmaTmemMaxM && k >= kMmaKStep && mma_resident_smem_bytes(m_pad, k, splits) <= kSmemBudget;
+}
+
 int launch_mma(const MmaArgs& a, cudaStream_t stream) {
   if (a.k % kMmaKStep != 0 || a.m_pad < 16 || a.m_pad > kMmaMaxM || a.m_pad % 16 != 0)
     return set_error(FI_ERR_UNSUPPORTED_SHAPE, "MMA path: k must be a multiple of %d and m <= %d", kMmaKStep,
                      kMmaMaxM);
   if (a.splits < 1 || a.splits > a.k / kMmaKStep || (a.splits > 1 && !a.partials))
     return set_error(FI_ERR_INVALID_ARG, "MMA path: %d splits for k=%lld", a.splits, (long long)a.k);
-  if (a.op_stages < 2 || a.op_stages > kMmaMaxOpStages || (int64_t)a.stage_bytes != mma_stage_bytes(a.m_pad))
+  const bool resident = a.act_resident != 0;
+  if (resident) {
+    if (!mma_act_resident(a.m_pad, a.k, a.splits) || a.op_stages != kMmaMaxOpStages || a.stage_bytes != 0 ||
+        (int64_t)a.act_bytes != mma_resident_act_bytes(a.m_pad, a.k, a.splits) ||
+        (int64_t)a.act_extra_bytes != mma_resident_extra_bytes(a.m_pad))
+      return set_error(FI_ERR_INVALID_ARG, "MMA path: resident activations do not fit m_pad=%d, k=%lld, %d splits",
+                       a.m_pad, (long long)a.k, a.splits);
+  } else if (a.op_stages < 2 || a.op_stages > kMmaMaxOpStages || (int64_t)a.stage_bytes != mma_stage_bytes(a.m_pad) ||
+             a.act_bytes != 0 || a.act_extra_bytes != 0) {
     return set_error(FI_ERR_INVALID_ARG, "MMA path: %d operand stages of %u bytes do not match m_pad=%d", a.op_stages,
                      a.stage_bytes, a.m_pad);
+  }
   CUtensorMap tmap_a, tmap_w;
-  // activations: f16 [m_pad, k], box 64 k x m_pad rows, 128-byte swizzle (the MMA's B operand)
-  int rc = encode_2d(&tmap_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.a16, (uint64_t)a.k, (uint64_t)a.m_pad,
-                     (uint64_t)a.k * 2, kMmaKStep, (uint32_t)a.m_pad, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (rc != FI_OK) return rc;
+  int rc = FI_OK;
+  if (resident) {
+    // activations: bf16 [m, k] as they come, box 64 k x m_pad rows (rows past m read as zero),
+    // 128-byte swizzle: the layout of the MMA's B operand, converted in place by the kernel
+    rc = encode_2d(&tmap_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.A, (uint64_t)a.k, (uint64_t)a.m, (uint64_t)a.k * 2,
+                   kMmaKStep, (uint32_t)a.m_pad, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != FI_OK) return rc;
+  } else {
+    // activations: f16 [m_pad, k], box 64 k x m_pad rows, 128-byte swizzle (the MMA's B operand)
+    rc = encode_2d(&tmap_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.a16, (uint64_t)a.k, (uint64_t)a.m_pad,
+                   (uint64_t)a.k * 2, kMmaKStep, (uint32_t)a.m_pad, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != FI_OK) return rc;
+  }
   // packed codes: u8 [n, k/2], box 32 bytes x 256 rows (rows past n read as zero codes)
   rc = encode_2d(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, (uint64_t)(a.k / 2), (uint64_t)a.n,
                  (uint64_t)(a.k / 2), 32, kMmaTileRows, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -559,21 +689,24 @@ int launch_mma(const MmaArgs& a, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
 
-  cudaLaunchConfig_t pre = {};
-  pre.gridDim = dim3((unsigned)a.m_pad);
-  pre.blockDim = dim3(256);
-  pre.stream = stream;
-  pre.attrs = attr;
-  pre.numAttrs = 1;
-  if (cudaLaunchKernelEx(&pre, act_to_f16_kernel, a.A, a.m, a.k, a.a16, a.rs) != cudaSuccess)
-    return set_cuda_error("act_to_f16_kernel launch");
+  if (!resident) {
+    cudaLaunchConfig_t pre = {};
+    pre.gridDim = dim3((unsigned)a.m_pad, (unsigned)a.splits);
+    pre.blockDim = dim3(256);
+    pre.stream = stream;
+    pre.attrs = attr;
+    pre.numAttrs = 1;
+    if (cudaLaunchKernelEx(&pre, act_to_f16_kernel, a.A, a.m, a.k, a.a16, a.rs) != cudaSuccess)
+      return set_cuda_error("act_to_f16_kernel launch");
+  }
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((a.n + kMmaTileRows - 1) / kMmaTileRows), (unsigned)a.splits);
   cfg.blockDim = dim3(kMmaThreads);
   // at most one CTA per SM: with the weights in tensor memory a CTA takes all 512 columns, and
   // a second CTA on the SM would wait in its allocation
-  cfg.dynamicSmemBytes = (size_t)std::max<int64_t>(mma_smem_bytes(a.m_pad), kSmemBudget / 2 + 4096);
+  const int64_t smem = resident ? mma_resident_smem_bytes(a.m_pad, a.k, a.splits) : mma_smem_bytes(a.m_pad);
+  cfg.dynamicSmemBytes = (size_t)std::max<int64_t>(smem, kSmemBudget / 2 + 4096);
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;

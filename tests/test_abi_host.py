@@ -217,9 +217,20 @@ def test_mma_tactic_resolution():
     assert info["kind"] == fi.KIND_MMA and info["splits"] == 1
     assert info["grid_x"] == 152064 // 256 and info["threads"] == 24 * 32
     assert 0 < info["smem_bytes"] <= 227 * 1024
-    # workspace: f16 activations [256, k] then 256 fp32 row scales
+    # m = 256 (above the tensor-memory operand's 128 rows): the prepass conversion, whose
+    # workspace is the f16 activations [256, k] then 256 fp32 (row, split) scales
+    assert info["variant"] == 1
     assert info["workspace_bytes"] == 256 * 5120 * 2 + 256 * 4
-    assert fi.resolve_tactic(33, 100, 64, t, B200_SMS)["workspace_bytes"] == 48 * 64 * 2 + 48 * 4
+    prepass = fi.make_tactic(fi.KIND_MMA, 1, 0, 1)
+    assert fi.resolve_tactic(33, 100, 64, prepass, B200_SMS)["workspace_bytes"] == 48 * 64 * 2 + 48 * 4
+    # resident activations (variant 2, converted in the kernel): no activation copy in the
+    # workspace; the automatic variant takes them for m_pad = 16 (here 16 rows, one step)
+    res = fi.resolve_tactic(33, 100, 64, fi.make_tactic(fi.KIND_MMA, 1, 0, 2), B200_SMS)
+    assert (res["variant"], res["workspace_bytes"]) == (2, 0)
+    assert fi.resolve_tactic(33, 100, 64, t, B200_SMS)["variant"] == 1
+    assert fi.resolve_tactic(16, 100, 64, t, B200_SMS) == fi.resolve_tactic(16, 100, 64, res_t := fi.make_tactic(
+        fi.KIND_MMA, 1, 0, 2), B200_SMS)
+    assert fi.resolve_tactic(16, 100, 64, res_t, B200_SMS)["variant"] == 2
     # the built-in rules take the GEMV up to m = 4 and the MMA (device-sized split) above (a shape
     # the generated table does not list); the table's picks for 4096 x 4096 agree on the kind
     assert fi.resolve_tactic(5, 4096, 4096, fi.TACTIC_DEFAULT, B200_SMS)["kind"] == fi.KIND_MMA
@@ -235,7 +246,9 @@ def test_mma_tactic_resolution():
     (257, 64, 64, fi.make_tactic(1, 1, 0, 0), -2),   # m beyond 256
     (64, 64, 96, fi.make_tactic(1, 1, 0, 0), -2),    # k not a multiple of 64
     (64, 64, 64, fi.make_tactic(1, 2, 0, 0), -1),    # no split-K on the MMA path
-    (64, 64, 64, fi.make_tactic(1, 1, 0, 3), -1),    # no variants
+    (64, 64, 64, fi.make_tactic(1, 1, 0, 3), -1),    # variants 0 (automatic), 1 (prepass), 2 (resident)
+    (129, 64, 64, fi.make_tactic(1, 1, 0, 2), -2),   # resident activations need m <= 128
+    (16, 64, 64 * 97, fi.make_tactic(1, 1, 0, 2), -2),  # 97 steps x 16 rows x 128 B exceed shared memory
 ])
 def test_mma_resolve_rejects(m, n, k, tactic, status):
     with pytest.raises(fi.FiError) as e:
@@ -253,8 +266,10 @@ def test_mma_device_sized_split_follows_the_wave_step_model():
         info = fi.resolve_tactic(m, n, k, mma, B200_SMS)
         assert info["splits"] == S and info["grid_y"] == S, (m, n, k, info)
         assert info["grid_x"] == -(-n // 256)
-        if S > 1:  # f16 activations, their row scales, then the partials at a 256-byte boundary
+        if S > 1 and info["variant"] == 1:  # f16 activations, their scales, then the partials
             assert info["workspace_bytes"] >= S * m * n * 4 + 2 * 16 * k
+        elif S > 1:  # resident activations: the partials only
+            assert info["workspace_bytes"] == S * m * n * 4
     # explicit splits are kept, up to k / 64 steps
     assert fi.resolve_tactic(64, 4096, 4096, fi.make_tactic(fi.KIND_MMA, 3, 0, 0), B200_SMS)["splits"] == 3
     with pytest.raises(fi.FiError):
@@ -388,3 +403,32 @@ def test_tuned_table_picks_are_the_defaults_and_valid_for_their_whole_bucket():
             assert fi.default_tactic(m, n, k, sms) == t, (n, k, m)
             splits.add(fi.resolve_tactic(m, n, k, t, sms)["splits"])
         assert len(splits) == 1, (n, k, m_lo, m_hi, splits)
+
+
+def test_mma_resident_activations_fit_rule():
+    """Resident activations (variant 2): the largest split's slice, ceil(k/64 / S) steps of
+    m_pad rows x 128 bytes, plus the raw-code ring, the row scales and the barriers must fit the
+    226 KB of dynamic shared memory the kernel asks for; m_pad <= 128. The automatic variant
+    takes it for one-wave grids (tiles x S <= SMs) with m_pad = 16 and at most 16 steps per
+    split, where the B200 measurements favour it."""
+    ring = 1024 + 4 * 256 * 32
+    for m, n, k, S in [(8, 4096, 14336, 0), (32, 4096, 14336, 8), (1, 4096, 4096, 1), (16, 4096, 6144, 1),
+                       (16, 4096, 6208, 1), (64, 152064, 5120, 1), (128, 4096, 14336, 16), (112, 2048, 7168, 4),
+                       (16, 152064, 5120, 1), (8, 40000, 4096, 1), (32, 5120, 17408, 7), (8, 4096, 4096, 8),
+                       (12, 4096, 4096, 4), (8, 4096, 4096, 0), (4, 14336, 4096, 8), (8, 2048, 1024, 1)]:
+        info = fi.resolve_tactic(m, n, k, fi.make_tactic(fi.KIND_MMA, S, 0, 0), B200_SMS)
+        m_pad = -(-m // 16) * 16
+        steps = -(-(k // 64) // info["splits"])
+        need = ring + steps * m_pad * 128 + -(-m_pad * 4 // 16) * 16 + 23 * 8
+        fits = m_pad <= 128 and need <= 226 * 1024
+        auto = fits and info["grid_x"] * info["splits"] <= B200_SMS and m_pad == 16 and steps <= 16
+        assert info["variant"] == (2 if auto else 1), (m, n, k, S, need)
+        if auto:
+            assert info["smem_bytes"] == need
+        explicit = fi.make_tactic(fi.KIND_MMA, info["splits"], 0, 2)
+        if fits:
+            assert fi.resolve_tactic(m, n, k, explicit, B200_SMS)["smem_bytes"] == need
+        else:
+            with pytest.raises(fi.FiError):
+                fi.resolve_tactic(m, n, k, explicit, B200_SMS)
+

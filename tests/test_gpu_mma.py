@@ -89,8 +89,14 @@ def test_k_not_multiple_of_64_is_refused():
     assert e.value.status == -2
 
 
-def test_stalled_producer_reports_timeout_and_recovers():
+@pytest.mark.parametrize("variant", [1, 2])
+def test_stalled_producer_reports_timeout_and_recovers(variant):
+    """Both activation modes (1: prepass conversion, 2: converted in the kernel): with the
+    producers issuing nothing, every wait runs out, the error word is set, and the next call is
+    correct."""
     m, n, k = 64, 512, 1024
+    t = fi.make_tactic(fi.KIND_MMA, 1, 0, variant)
+    assert fi.resolve_tactic(m, n, k, t)["variant"] == variant
     A = inputs.activations(m, k, seed=12)
     W, (Wq, Ws, g) = _gpu.weights(n, k, 12)
     ref = oracle.mm(A, Wq, Ws, g)
@@ -99,15 +105,50 @@ def test_stalled_producer_reports_timeout_and_recovers():
     fi.debug_set(fi.DEBUG_WAIT_TIMEOUT_NS, 20_000_000)
     fi.debug_set(fi.DEBUG_STALL_PRODUCER, 1)
     try:
-        _mm(A, dw)
+        _mm(A, dw, t)
         code = fi.get_device_error()
         assert code != 0, code
         assert fi.get_device_error() == 0
     finally:
         fi.debug_set(fi.DEBUG_STALL_PRODUCER, 0)
         fi.debug_set(fi.DEBUG_WAIT_TIMEOUT_NS, 1_000_000_000)
-    _gpu.assert_within_tolerance(_mm(A, dw), ref, "after recovery")
+    _gpu.assert_within_tolerance(_mm(A, dw, t), ref, "after recovery")
     assert fi.get_device_error() == 0
+
+
+def _split_skewed_activations(m, k, seed):
+    """Activations whose K splits have very different ranges: outliers, one row scaled by 2^40 in
+    its first 64 k only, one row zero over its second half, one row of tiny values."""
+    A = inputs.activations_f32(m, k, seed=seed, outliers=True)
+    A[0, :64] *= np.float32(2.0 ** 40)
+    if m > 1:
+        A[1, k // 2:] = 0.0
+    if m > 2:
+        A[2] *= np.float32(2.0 ** -100)
+    return inputs.to_bf16_bits(A)
+
+
+@pytest.mark.parametrize("m,n,k,S", [(1, 256, 512, 1), (8, 1000, 2048, 3), (17, 257, 320, 1), (40, 300, 4096, 0),
+                                     (100, 1000, 1024, 2), (128, 768, 1024, 16), (16, 4096, 6144, 1)])
+def test_resident_and_prepass_activations_give_the_same_bits(m, n, k, S):
+    """Variant 2 converts each split's activations in the kernel's decode warps (shared memory),
+    variant 1 in a prepass kernel (workspace); both scale per (row, split) with the same
+    arithmetic, so outputs (bf16 and f16) are identical bit for bit, and within the oracle's
+    tolerance."""
+    A = _split_skewed_activations(m, k, seed=m + k)
+    W, (Wq, Ws, g) = _gpu.weights(n, k, m + 3)
+    dw = _gpu.device_weights(n, k, m + 3)
+    res, pre = fi.make_tactic(fi.KIND_MMA, S, 0, 2), fi.make_tactic(fi.KIND_MMA, S, 0, 1)
+    assert fi.resolve_tactic(m, n, k, res)["splits"] == fi.resolve_tactic(m, n, k, pre)["splits"]
+    got_res = _mm(A, dw, res)
+    assert np.array_equal(got_res, _mm(A, dw, pre))
+    Wq_d, Ws_d, g_d = dw
+    a = _gpu.dev_bf16(A)
+    f16 = [fi.mm_bf16_fp4(a, Wq_d, Ws_d, g_d, tactic=t, out_dtype=torch.float16) for t in (res, pre)]
+    torch.cuda.synchronize()
+    assert torch.equal(f16[0], f16[1])
+    ref = oracle.mm(A, Wq, Ws, g)
+    _gpu.assert_within_tolerance(got_res, ref, f"resident {m}x{n}x{k} S={S}")
 
 
 @pytest.mark.parametrize("m,n,k,S", [(8, 1000, 2048, 3), (40, 300, 4096, 0), (1, 256, 512, 2), (128, 768, 1024, 16)])

@@ -90,10 +90,10 @@ def test_partials_beyond_the_static_scratch_are_refused():
 
 
 def test_default_tactic_falls_back_to_a_split_that_fits():
-    """4096 x 14336 at m = 32: the default (the tensor-core path with 9 K splits) needs more
-    scratch than the static array holds; the allocation-free entry point takes the largest
-    smaller split that fits and stays within tolerance."""
-    m, n, k = 32, 4096, 14336
+    """5120 x 17408 (a Qwen3.6-27B down projection) at m = 32: the default (the tensor-core path
+    with 7 K splits) needs more scratch than the static array holds; the allocation-free entry
+    point takes the largest smaller split that fits and stays within tolerance."""
+    m, n, k = 32, 5120, 17408
     assert fi.workspace_bytes(m, n, k) > 4 << 20
     A_bits = inputs.activations(m, k, seed=3)
     W, (Wq_o, Ws_o, g_o) = _gpu.weights(n, k, 3)
@@ -109,11 +109,12 @@ def test_default_tactic_falls_back_to_a_split_that_fits():
 
 
 def test_default_falls_back_to_a_single_split_gemv():
-    """lm_head-like 152064 x 5120 at m = 4: the default (GEMV with two K splits) needs about
-    4.9 MB of partials; the only smaller split, S = 1, needs no scratch at all and must be the
-    one taken. Its bits equal the allocating call's with that tactic, and it stays within
-    tolerance of the oracle on sampled columns."""
-    m, n, k = 4, 152064, 5120
+    """150016 x 5120 at m = 4 (a shape the generated tactic table does not list, so the built-in
+    rules decide): the default (GEMV with two K splits) needs about 4.8 MB of partials; the only
+    smaller split, S = 1, needs no scratch at all and must be the one taken. Its bits equal the
+    allocating call's with that tactic, and it stays within tolerance of the oracle on sampled
+    columns."""
+    m, n, k = 4, 150016, 5120
     info = fi.resolve_tactic(m, n, k, fi.TACTIC_DEFAULT)
     assert info["kind"] == fi.KIND_GEMV and info["splits"] > 1 and info["workspace_bytes"] > SCRATCH_BYTES
     fallback = fi.make_tactic(fi.KIND_GEMV, 1, 0, 0)  # the automatic pipeline: any S = 1 GEMV gives these bits
