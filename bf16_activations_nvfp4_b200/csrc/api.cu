@@ -465,9 +465,10 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
 // converts its split's slice while its decode warps start on the weights; that saves the
 // prepass launch (about 3 us in a chained sequence of calls on B200) but costs the CTA time in
 // proportion to m_pad x its steps, once per wave. Measured on B200 (4096 x 4096 at m = 8, S = 8:
-// 10.1 against 11.4 us; 4096 x 14336 at m = 32, S = 8: 28.4 against 24.4 us), so automatic
-// takes it only for one-wave grids (tiles x S <= SMs) with m_pad = 16 and at most 16 steps per
-// split. Needs m <= 256 and k a multiple of 64; the workspace holds the f16
+// 10.0 against 11.0 us; 4096 x 14336 at m = 8, S = 8 (28 steps): 19.6 against 20.4 us; at
+// m = 32: 26.6 against 23.0 us; 14336 x 4096 at m = 8, S = 2 (32 steps): 20.7 against 20.3 us),
+// so automatic takes it only for one-wave grids (tiles x S <= SMs) with m_pad = 16 and at most
+// 28 steps per split. Needs m <= 256 and k a multiple of 64; the workspace holds the f16
 // activations and their (row, split) scales in prepass mode, then the [S, m, n] fp32 partials
 // when S > 1. Both modes give the same bits.
 static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var, int sms,
@@ -512,7 +513,7 @@ static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req,
                      "MMA resident activations: m=%lld rows of %lld k over %lld splits do not fit shared memory",
                      (long long)m, (long long)k, (long long)S);
   const int64_t steps = (KS + S - 1) / S;
-  const bool resident = var == 2 || (var == 0 && fits && tiles * S <= sms && m_pad == 16 && steps <= 16);
+  const bool resident = var == 2 || (var == 0 && fits && tiles * S <= sms && m_pad == 16 && steps <= 28);
   out->kind = FI_KIND_MMA;
   out->splits = (int32_t)S;
   out->ctas_per_sm = 1;

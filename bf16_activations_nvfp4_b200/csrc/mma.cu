@@ -152,6 +152,34 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   return d;
 }
 
+// The four bytes of a 32-bit word (8 E2M1 codes, low nibble first) as four f16x2 pairs, in
+// order, with one unpack of the word for all four conversions.
+__device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t& h0, uint32_t& h1, uint32_t& h2,
+                                                  uint32_t& h3) {
+  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
+      " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+      : "r"(w));
+}
+
+// One thread's 32 k of a step: 16 code bytes (blocks 2hb, 2hb+1 of the row) and the two E4M3
+// scales in the low 16 bits of sc2 -> 16 f16 pairs (code value times its block scale, exact).
+__device__ __forceinline__ void decode_step(const uint4 c0, uint32_t sc2, uint32_t (&hv)[16]) {
+  const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
+#pragma unroll
+  for (int bb = 0; bb < 2; ++bb) {  // 16-k block 2hb + bb: words 2bb, 2bb+1
+    const uint32_t sf2 = e4m3x2_to_f16x2(__byte_perm(sc2, 0u, (uint32_t)(bb | (bb << 4))));
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t h[4];
+      e2m1x8_to_f16x2x4(words[2 * bb + q], h[0], h[1], h[2], h[3]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) hv[8 * bb + 4 * q + i] = hmul2(h[i], sf2);
+    }
+  }
+}
+
 // Wait that ignores the abort flag (used to drain copies and MMAs in flight before exit).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, unsigned* err) {
   volatile int never = 0;
@@ -436,45 +464,70 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       return v;
     };
     uint4 sg0 = load_group(0), sg1 = load_group(1), sg2 = load_group(2);
-    int os = 0;        // operand stage of step s
-    uint32_t eph = 0;  // phase of op_empty[os] to wait for (steps s >= NST)
-    for (int s = 0; s < KS; ++s) {
-      const int rsn = s % kRawStages;
-      const int sj = s & 3;
-      const uint32_t sc4 = sj == 0 ? sg0.x : (sj == 1 ? sg0.y : (sj == 2 ? sg0.z : sg0.w));
-      if (sj == 3) {
+    if constexpr (TA) {
+      // Four operand stages (the host guarantees NST == kRawStages == 4 here), so the loop runs
+      // over groups of 4 steps with the step's stage, barriers, scale word and tensor-memory
+      // columns fixed at compile time; a group's 4 scale words were loaded 8-11 steps ahead.
+      // The decode warps' instruction issue paces a step at small m (B200 counters: cutting
+      // the integer work per step from 63 to 28 instructions per thread took 4096 x 14336 at
+      // m = 8 from 22.0 to 20.4 us), so the per-step bookkeeping is kept to a minimum.
+      static_assert(kRawStages == 4 && kMmaMaxOpStages == 4, "one group = one pass over both rings");
+      const uint32_t raw_row = base + (uint32_t)r * 32u + (uint32_t)hb * 16u;
+      const uint32_t tm_row = tmem + ((uint32_t)(tq * 32) << 16) + a_col(0, r >> 7) + (uint32_t)hb * 16u;
+      bool run = true;
+      for (int s0 = 0; s0 < KS && run; s0 += 4) {
+        const uint32_t par = (uint32_t)((s0 >> 2) & 1);  // raw_full phase; op_empty waits for par ^ 1
+        const uint4 scg = sg0;
         sg0 = sg1;
         sg1 = sg2;
-        sg2 = load_group(s / 4 + 3);
-      }
-      // every lane waits; the warp continues only if all of them saw both phases (a timeout is
-      // seen lane by lane, and the warp must stay converged for __syncwarp below)
-      const bool ok =
-          mbar_wait_bounded(&raw_full[rsn], (uint32_t)((s / kRawStages) & 1), &abort_flag, p.timeout_ns, p.err, 1u) &&
-          (s < NST || mbar_wait_bounded(&op_empty[os], eph, &abort_flag, p.timeout_ns, p.err, 1u));
-      if (!__all_sync(0xffffffffu, ok)) break;
-      const uint4 c0 = lds_v4m(raw_addr(rsn) + (uint32_t)r * 32u + (uint32_t)hb * 16u);
-      const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
-      const uint32_t sc2 = hb ? (sc4 >> 16) : sc4;  // the scales of blocks 2hb, 2hb+1
-      uint32_t hv[16];  // the 32 k of this thread as f16 pairs, in k order
+        sg2 = load_group(s0 / 4 + 3);
 #pragma unroll
-      for (int bb = 0; bb < 2; ++bb) {  // 16-k block b = 2hb + bb: words 2bb, 2bb+1
-        const uint32_t sf2 = e4m3x2_to_f16x2(__byte_perm(sc2, 0u, (uint32_t)(bb | (bb << 4))));
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const uint32_t wd = words[2 * bb + q];
-          hv[8 * bb + 4 * q + 0] = hmul2(e2m1x2_byte_to_f16x2<0>(wd), sf2);
-          hv[8 * bb + 4 * q + 1] = hmul2(e2m1x2_byte_to_f16x2<1>(wd), sf2);
-          hv[8 * bb + 4 * q + 2] = hmul2(e2m1x2_byte_to_f16x2<2>(wd), sf2);
-          hv[8 * bb + 4 * q + 3] = hmul2(e2m1x2_byte_to_f16x2<3>(wd), sf2);
+        for (int j = 0; j < 4; ++j) {
+          if (s0 + j >= KS) break;
+          // every lane waits; the warp continues only if all of them saw both phases (one step
+          // per pass: pairing two steps per wait and store cut instructions but lost overlap)
+          const bool ok = mbar_wait_bounded(&raw_full[j], par, &abort_flag, p.timeout_ns, p.err, 1u) &&
+                          (s0 == 0 || mbar_wait_bounded(&op_empty[j], par ^ 1u, &abort_flag, p.timeout_ns, p.err, 1u));
+          if (!__all_sync(0xffffffffu, ok)) {
+            run = false;
+            break;
+          }
+          const uint4 c0 = lds_v4m(raw_row + (uint32_t)j * kRawBytes);
+          const uint32_t sc4 = j == 0 ? scg.x : (j == 1 ? scg.y : (j == 2 ? scg.z : scg.w));
+          uint32_t hv[16];
+          decode_step(c0, hb ? (sc4 >> 16) : sc4, hv);
+          // lane r & 127 of half r >> 7: columns a_col + 16 hb .. + 15 hold k 32 hb .. 32 hb + 31
+          tmem_st16(tm_row + (uint32_t)j * 64u, hv);
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&op_full[j]);
+            mbar_arrive(&raw_empty[j]);
+          }
         }
       }
-      if constexpr (TA) {
-        // lane r & 127 of half r >> 7: columns a_col + 16 hb .. + 15 hold k 32 hb .. 32 hb + 31
-        tmem_st16(tmem + ((uint32_t)(tq * 32) << 16) + a_col(os, r >> 7) + (uint32_t)hb * 16u, hv);
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-      } else {
+    } else {
+      int os = 0;        // operand stage of step s
+      uint32_t eph = 0;  // phase of op_empty[os] to wait for (steps s >= NST)
+      for (int s = 0; s < KS; ++s) {
+        const int rsn = s % kRawStages;
+        const int sj = s & 3;
+        const uint32_t sc4 = sj == 0 ? sg0.x : (sj == 1 ? sg0.y : (sj == 2 ? sg0.z : sg0.w));
+        if (sj == 3) {
+          sg0 = sg1;
+          sg1 = sg2;
+          sg2 = load_group(s / 4 + 3);
+        }
+        // every lane waits; the warp continues only if all of them saw both phases (a timeout is
+        // seen lane by lane, and the warp must stay converged for __syncwarp below)
+        const bool ok =
+            mbar_wait_bounded(&raw_full[rsn], (uint32_t)((s / kRawStages) & 1), &abort_flag, p.timeout_ns, p.err, 1u) &&
+            (s < NST || mbar_wait_bounded(&op_empty[os], eph, &abort_flag, p.timeout_ns, p.err, 1u));
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const uint4 c0 = lds_v4m(raw_addr(rsn) + (uint32_t)r * 32u + (uint32_t)hb * 16u);
+        uint32_t hv[16];  // the 32 k of this thread as f16 pairs, in k order
+        decode_step(c0, hb ? (sc4 >> 16) : sc4, hv);
         const uint32_t dst = wop_addr(os) + wdst;
 #pragma unroll
         for (int c = 0; c < 4; ++c)  // chunk 4hb + c of the row (8 k each), 128-byte swizzle
@@ -482,15 +535,15 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                  hv[4 * c + 3]);
         // make the generic-proxy stores visible to the tensor core (async proxy)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&op_full[os]);
-        mbar_arrive(&raw_empty[rsn]);
-      }
-      if (++os == NST) {
-        os = 0;
-        if (s >= NST) eph ^= 1u;
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&op_full[os]);
+          mbar_arrive(&raw_empty[rsn]);
+        }
+        if (++os == NST) {
+          os = 0;
+          if (s >= NST) eph ^= 1u;
+        }
       }
     }
   } else if (warp == kWarpMma || warp == kWarpMma2) {
@@ -645,6 +698,9 @@ int launch_mma(const MmaArgs& a, cudaStream_t stream) {
   if (a.splits < 1 || a.splits > a.k / kMmaKStep || (a.splits > 1 && !a.partials))
     return set_error(FI_ERR_INVALID_ARG, "MMA path: %d splits for k=%lld", a.splits, (long long)a.k);
   const bool resident = a.act_resident != 0;
+  if (a.m_pad <= kMmaTmemMaxM && a.op_stages != kMmaMaxOpStages)
+    return set_error(FI_ERR_INVALID_ARG, "MMA path: weights in tensor memory need %d operand stages, got %d",
+                     kMmaMaxOpStages, a.op_stages);
   if (resident) {
     if (!mma_act_resident(a.m_pad, a.k, a.splits) || a.op_stages != kMmaMaxOpStages || a.stage_bytes != 0 ||
         (int64_t)a.act_bytes != mma_resident_act_bytes(a.m_pad, a.k, a.splits) ||
