@@ -464,11 +464,13 @@ static int resolve_gemv(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req
 // into shared memory, "resident"; only where the split's slice fits, m <= 128). Every CTA then
 // converts its split's slice while its decode warps start on the weights; that saves the
 // prepass launch (about 3 us in a chained sequence of calls on B200) but costs the CTA time in
-// proportion to m_pad x its steps, once per wave. Measured on B200 (4096 x 4096 at m = 8, S = 8:
-// 10.0 against 11.0 us; 4096 x 14336 at m = 8, S = 8 (28 steps): 19.6 against 20.4 us; at
-// m = 32: 26.6 against 23.0 us; 14336 x 4096 at m = 8, S = 2 (32 steps): 20.7 against 20.3 us),
-// so automatic takes it only for one-wave grids (tiles x S <= SMs) with m_pad = 16 and at most
-// 28 steps per split. Needs m <= 256 and k a multiple of 64; the workspace holds the f16
+// proportion to its rows x steps, once per wave. Measured on B200 (resident against prepass,
+// us per call): 4096 x 4096, S = 8: 9.5 / 10.9 at m = 4, 10.0 / 11.0 at m = 8, 11.0 / 11.7 at
+// m = 16; 4096 x 14336, S = 8 (28 steps): 18.9 / 20.1 at m = 4, 19.6 / 20.4 at m = 8, 22.0 /
+// 21.2 at m = 16, 26.6 / 23.0 at m = 32; 2048 x 7168, S = 8: 11.7 / 12.5 at m = 4, 14.8 / 12.9
+// at m = 16; 14336 x 4096, S = 2 (32 steps): 20.7 / 20.3 at m = 8. So automatic takes it for
+// one-wave grids (tiles x S <= SMs) with m <= 8 and at most 28 steps per split. Needs m <= 256
+// and k a multiple of 64; the workspace holds the f16
 // activations and their (row, split) scales in prepass mode, then the [S, m, n] fp32 partials
 // when S > 1. Both modes give the same bits.
 static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req, int var, int sms,
@@ -513,7 +515,7 @@ static int resolve_mma(int64_t m, int64_t n, int64_t k, int S_req, int ctas_req,
                      "MMA resident activations: m=%lld rows of %lld k over %lld splits do not fit shared memory",
                      (long long)m, (long long)k, (long long)S);
   const int64_t steps = (KS + S - 1) / S;
-  const bool resident = var == 2 || (var == 0 && fits && tiles * S <= sms && m_pad == 16 && steps <= 28);
+  const bool resident = var == 2 || (var == 0 && fits && tiles * S <= sms && m <= 8 && steps <= 28);
   out->kind = FI_KIND_MMA;
   out->splits = (int32_t)S;
   out->ctas_per_sm = 1;

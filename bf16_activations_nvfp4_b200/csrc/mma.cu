@@ -153,7 +153,7 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
 }
 
 // The four bytes of a 32-bit word (8 E2M1 codes, low nibble first) as four f16x2 pairs, in
-// order, with one unpack of the word for all four conversions.
+// byte order, with one unpack of the word for all four conversions. Exact.
 __device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t& h0, uint32_t& h1, uint32_t& h2,
                                                   uint32_t& h3) {
   asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"

@@ -224,13 +224,14 @@ def test_mma_tactic_resolution():
     prepass = fi.make_tactic(fi.KIND_MMA, 1, 0, 1)
     assert fi.resolve_tactic(33, 100, 64, prepass, B200_SMS)["workspace_bytes"] == 48 * 64 * 2 + 48 * 4
     # resident activations (variant 2, converted in the kernel): no activation copy in the
-    # workspace; the automatic variant takes them for m_pad = 16 (here 16 rows, one step)
+    # workspace; the automatic variant takes them for m <= 8 (here one step)
     res = fi.resolve_tactic(33, 100, 64, fi.make_tactic(fi.KIND_MMA, 1, 0, 2), B200_SMS)
     assert (res["variant"], res["workspace_bytes"]) == (2, 0)
     assert fi.resolve_tactic(33, 100, 64, t, B200_SMS)["variant"] == 1
-    assert fi.resolve_tactic(16, 100, 64, t, B200_SMS) == fi.resolve_tactic(16, 100, 64, res_t := fi.make_tactic(
-        fi.KIND_MMA, 1, 0, 2), B200_SMS)
-    assert fi.resolve_tactic(16, 100, 64, res_t, B200_SMS)["variant"] == 2
+    res_t = fi.make_tactic(fi.KIND_MMA, 1, 0, 2)
+    assert fi.resolve_tactic(8, 100, 64, t, B200_SMS) == fi.resolve_tactic(8, 100, 64, res_t, B200_SMS)
+    assert fi.resolve_tactic(8, 100, 64, res_t, B200_SMS)["variant"] == 2
+    assert fi.resolve_tactic(9, 100, 64, t, B200_SMS)["variant"] == 1
     # the built-in rules take the GEMV up to m = 4 and the MMA (device-sized split) above (a shape
     # the generated table does not list); the table's picks for 4096 x 4096 agree on the kind
     assert fi.resolve_tactic(5, 4096, 4096, fi.TACTIC_DEFAULT, B200_SMS)["kind"] == fi.KIND_MMA
@@ -409,8 +410,8 @@ def test_mma_resident_activations_fit_rule():
     """Resident activations (variant 2): the largest split's slice, ceil(k/64 / S) steps of
     m_pad rows x 128 bytes, plus the raw-code ring, the row scales and the barriers must fit the
     226 KB of dynamic shared memory the kernel asks for; m_pad <= 128. The automatic variant
-    takes it for one-wave grids (tiles x S <= SMs) with m_pad = 16 and at most 28 steps per
-    split, where the B200 measurements favour it."""
+    takes it for one-wave grids (tiles x S <= SMs) with m <= 8 and at most 28 steps per split,
+    where the B200 measurements favour it."""
     ring = 1024 + 4 * 256 * 32
     for m, n, k, S in [(8, 4096, 14336, 0), (32, 4096, 14336, 8), (1, 4096, 4096, 1), (16, 4096, 6144, 1),
                        (16, 4096, 6208, 1), (64, 152064, 5120, 1), (128, 4096, 14336, 16), (112, 2048, 7168, 4),
@@ -421,7 +422,7 @@ def test_mma_resident_activations_fit_rule():
         steps = -(-(k // 64) // info["splits"])
         need = ring + steps * m_pad * 128 + -(-m_pad * 4 // 16) * 16 + 23 * 8
         fits = m_pad <= 128 and need <= 226 * 1024
-        auto = fits and info["grid_x"] * info["splits"] <= B200_SMS and m_pad == 16 and steps <= 28
+        auto = fits and info["grid_x"] * info["splits"] <= B200_SMS and m <= 8 and steps <= 28
         assert info["variant"] == (2 if auto else 1), (m, n, k, S, need)
         if auto:
             assert info["smem_bytes"] == need
