@@ -516,15 +516,39 @@ def run_extra_shapes(dev, stream, peaks) -> dict:
 
 
 def mma_wave(args) -> None:
-    """Profiling case for the tensor-core path: one wave of CTAs (n = 148 x 256 rows, k = 5120,
-    the lm_head-like k) at m = 64 and 256, each timed over 10 eager calls after 3 warm-up
-    calls. Small enough for a multi-pass ncu capture of single launches."""
+    """Profiling cases for the tensor-core path, each timed over 10 eager calls after 3 warm-up
+    calls with the default tactic, small enough for a multi-pass ncu capture of single
+    launches: first the small-batch decode GEMM 4096 x 14336 at m = 8 (mma_nvfp4 launches 1-13),
+    then one wave of CTAs (n = 148 x 256 rows, k = 5120, the lm_head-like k) at m = 64
+    (launches 14-26) and m = 256 (launches 27-39)."""
     import torch
 
     import bf16_activations_nvfp4_b200 as fi
     from bf16_activations_nvfp4_b200 import inputs
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    n, k = inputs.SMALL_BATCH_NK
+    W = torch.from_numpy(inputs.weights(n, k, seed=0)).to(dev)
+    Wq, Ws, g = fi.pack_weights(W)
+    del W
+    m = 8
+    fi.set_workspace(torch.empty(fi.workspace_bytes(m, n, k) // 4 + 64, dtype=torch.float32, device=dev))
+    A = torch.from_numpy(inputs.activations(m, k, seed=0).view(np.int16)).view(torch.bfloat16).to(dev)
+    out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        fi.mm_bf16_fp4(A, Wq, Ws, g, out=out)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(10):
+        fi.mm_bf16_fp4(A, Wq, Ws, g, out=out)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / 10
+    info = fi.resolve_tactic(m, n, k)
+    print(json.dumps({"n": n, "k": k, "m": m, "kind": info["kind"], "splits": info["splits"],
+                      "variant": info["variant"], "us": round(us, 2)}), flush=True)
+    del Wq, Ws, A, out
     n, k = 148 * 256, LM_HEAD[1]
     W = torch.from_numpy(inputs.weights(n, k, seed=0)).to(dev)
     Wq, Ws, g = fi.pack_weights(W)

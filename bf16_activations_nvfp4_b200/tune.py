@@ -11,8 +11,9 @@ calls are chained by programmatic dependent launch inside one CUDA graph, and th
 graph replays is taken. The fastest tactic of a bucket over the bucket's sample m values wins; a
 bucket's tactic is one code for all of its m, so the default stays batch-invariant inside it.
 
-Buckets of m: {1}, {2..4}, {5..32}, {33..256}. Candidates are the codes fi_list_tactics offers at
-every sample m of the bucket. The table is keyed by (n, k, SM count); shapes and devices it
+Buckets of m: {1}, {2}, {3..4}, {5..32}, {33..256} ({2} apart: on B200 the GEMV's register
+pipeline wins at m = 2 where the tensor-core path wins at m = 4 on the 4096 x 14336 class of
+shapes). Candidates are the codes fi_list_tactics offers at every sample m of the bucket. The table is keyed by (n, k, SM count); shapes and devices it
 does not list fall back to the library's built-in rules.
 """
 from __future__ import annotations
@@ -30,7 +31,7 @@ ROOT = os.path.dirname(PKG)
 OUT = os.path.join(PKG, "csrc", "tactic_table.inc")
 
 # (m_lo, m_hi, sample m values timed for the bucket)
-BUCKETS = [(1, 1, (1,)), (2, 4, (2, 4)), (5, 32, (8, 32)), (33, 256, (64, 256))]
+BUCKETS = [(1, 1, (1,)), (2, 2, (2,)), (3, 4, (4,)), (5, 32, (8, 32)), (33, 256, (64, 256))]
 COLD_BYTES = 300 << 20  # weight copies per shape: more than twice the 126 MB L2
 
 
