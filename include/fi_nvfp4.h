@@ -82,8 +82,14 @@ typedef enum {
  *                an L2 prefetch of weights up to 40 MB; its CTAs-per-SM field is ignored;
  *                4 = weights loaded straight to registers, 1 or 2 rows per warp;
  *                5 = the lean form of 1 for m = 1: k % 256 == 0 and every split's k/32 chunks
- *                a multiple of 32, 1, 2 or 4 rows per item). MMA: 0. At m = 1 the automatic
- *                pipeline is 5 wherever it applies.
+ *                a multiple of 32, 1, 2 or 4 rows per item). At m = 1 the automatic pipeline is
+ *                5 wherever it applies.
+ *                MMA: where the activations are converted to the tensor core's f16 operand
+ *                (the same arithmetic and bits either way): 1 = a prepass kernel into the
+ *                workspace; 2 = inside the MMA kernel, into shared memory (m <= 128 and the
+ *                split's k range x 16-row-padded m fits next to the weight ring, else
+ *                FI_ERR_UNSUPPORTED_SHAPE); 0 = automatic: 2 for one-wave grids at m <= 8
+ *                with at most 28 64-k steps per split, else 1. Resolves to 1 or 2.
  *                The default table: for the shapes the library's cold-L2 tuner measured (the
  *                generated csrc/tactic_table.inc, per SM count and bucket of m), its pick;
  *                otherwise at m = 1, 3 for weights up to 12 MB, else 4 where k % 256 != 0, 5
@@ -116,12 +122,13 @@ typedef struct {
   int32_t kind;        /* FI_KIND_GEMV or FI_KIND_MMA */
   int32_t splits;      /* resolved S >= 1 */
   int32_t ctas_per_sm; /* resolved co-resident CTAs per SM */
-  int32_t variant;     /* resolved variant (GEMV: rows per warp | pipeline << 4; MMA: 0) */
+  int32_t variant;     /* resolved variant (GEMV: rows per warp | pipeline << 4; MMA: 1 prepass, 2 in-kernel) */
   int32_t grid_x;      /* CTAs along n */
   int32_t grid_y;      /* CTAs along k (= splits) */
   int32_t threads;     /* threads per CTA */
   int32_t smem_bytes;  /* dynamic shared memory per CTA */
-  int64_t workspace_bytes; /* scratch: GEMV fp32 partials (0 if S == 1); MMA f16 A, then partials if S > 1 */
+  int64_t workspace_bytes; /* scratch: GEMV fp32 partials (0 if S == 1); MMA variant 1: f16 A and its scales,
+                              then partials if S > 1; MMA variant 2: partials if S > 1 */
 } fi_tactic_info;
 
 /* Output element types (the op writes bf16 by default; PR #4038's commits add an fp16 output
@@ -162,8 +169,9 @@ FI_API int fi_nvfp4_pack_weights(const float* W, int64_t n, int64_t k, uint8_t* 
  * m <= 256 with k % 64 == 0 for MMA tactics (FI_ERR_UNSUPPORTED_SHAPE otherwise). m == 0
  * or n == 0 is a no-op; k == 0 writes zeros.
  * Workspace: a GEMV call with S > 1 needs fi_mm_workspace_bytes() bytes of device memory
- * for fp32 partials; an MMA call needs them for its f16 copy of A (each row times a power
- * of two), the per-row scales and, when S > 1, the fp32 partials. It uses the buffer registered with
+ * for fp32 partials; an MMA call with activation variant 1 needs them for its f16 copy of A
+ * (each row and K split times a power of two), those scales and, when S > 1, the fp32
+ * partials; variant 2 only for the partials. It uses the buffer registered with
  * fi_set_workspace() for the current device (FI_ERR_WORKSPACE if that is too small); if
  * none is registered, the library allocates one with cudaMalloc (growing it when needed)
  * and keeps it until process exit, except while `stream` is capturing a CUDA graph,
@@ -208,13 +216,13 @@ FI_API int fi_mm_bf16_fp4_out(const uint16_t* A, const uint8_t* Wq, const uint8_
  * as an operator plugin inside a serving engine that has already reserved the device's memory
  * for weights and the KV cache, or a component whose memory plan is fixed at start-up and
  * that owns no buffer it could pass to fi_mm_bf16_fp4_ex. fi_mm_bf16_fp4 would cudaMalloc its
- * workspace on first use; this variant keeps the workspace (the split-K fp32 partials, or
- * for MMA tactics the f16 copy of the activations) in a static device array compiled into
+ * workspace on first use; this variant keeps the workspace (the split-K fp32 partials, and
+ * for MMA tactics of variant 1 the f16 copy of the activations) in a static device array compiled into
  * the library instead: FI_NOALLOC_SCRATCH_BYTES (4 MiB) on every GPU that loads the library,
  * held until the process exits.
  * Arguments, tactics, preconditions and results are those of fi_mm_bf16_fp4.
  * Limit: the resolved tactic's fi_mm_workspace_bytes() (GEMV: 4 * splits * m * n; MMA: about
- * 2 * m * k, plus 4 * splits * m * n when split) must not exceed FI_NOALLOC_SCRATCH_BYTES; a
+ * 2 * m * k for variant 1, plus 4 * splits * m * n when split) must not exceed FI_NOALLOC_SCRATCH_BYTES; a
  * larger call returns FI_ERR_WORKSPACE and launches nothing. Single-split GEMV tactics use no
  * scratch. With FI_TACTIC_DEFAULT, a default whose scratch would not fit is replaced by the
  * same kind with the largest smaller split that fits (for a GEMV, with the default's pipeline
