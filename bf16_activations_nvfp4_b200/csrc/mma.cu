@@ -19,9 +19,12 @@
 //                  depend on the preceding kernel);
 //      warp 18     TMA producer of the f16 activation tiles (m_pad rows x 64 k, 128-byte
 //                  swizzled) into the operand stages (2 to 4, as many as shared memory holds);
-//                  with resident activations it converts them instead, with warps 19-22;
-//      warps 2-17  decode: two threads per weight row (32 k each), codes -> f16 (cvt.rn.f16x2.e2m1x2) times
-//                  the block scale (exact f16 multiply), stored in the 128-byte-swizzled
+//                  with resident activations it copies the split's bf16 tiles once instead and
+//                  converts them with warps 19-22;
+//      warps 2-17  decode: two threads per weight row (32 k each), codes -> f16
+//                  (cvt.rn.f16x2.e2m1x2) times the block scale (exact f16 multiply), written to
+//                  tensor memory (m_pad <= 128; the loop runs over groups of 4 steps with
+//                  compile-time stage indices) or to shared memory in the 128-byte-swizzled
 //                  K-major layout the MMA reads; the block scales are loaded 8-11 steps ahead;
 //      warps 1, 23 the MMAs, one thread each, one M = 128 half of the tile each (warp 1 also
 //                  allocates TMEM): per 64-k step 4 K=16 steps, N = m_pad, accumulating in
@@ -263,7 +266,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   __shared__ volatile int abort_flag;
   __shared__ uint32_t tmem_slot;
   // 1024-byte aligned base for the swizzled tiles: the raw-code ring, then NST operand stages
-  // (decoded weights, then activations, each stage stage_bytes), then the barriers
+  // (decoded weights, then activations, each stage stage_bytes; 0 with resident activations),
+  // then the resident slice and its row scales (act_bytes + act_extra_bytes, else 0), then
+  // the barriers
   const int NST = p.op_stages;
   const uint32_t stage_bytes = p.stage_bytes;
   const uint32_t raw_s = smem_addr(smem_raw);
