@@ -411,6 +411,24 @@ def test_tuned_table_picks_are_the_defaults_and_valid_for_their_whole_bucket():
         assert len(splits) == 1, (n, k, m_lo, m_hi, splits)
 
 
+def test_tuned_table_covers_every_m_once_per_shape():
+    """For every (n, k, SMs) the generated table lists, its buckets are the tuner's buckets and
+    tile m = 1..256 without gaps or overlaps, and the file was written by the tuner (its header)."""
+    import os
+    from bf16_activations_nvfp4_b200 import tune
+    path = os.path.join(os.path.dirname(fi.__file__), "csrc", "tactic_table.inc")
+    assert open(path).readline().startswith("// Default-tactic table: GENERATED by")
+    by_shape = {}
+    for n, k, m_lo, m_hi, sms, t in _tuned_entries():
+        by_shape.setdefault((n, k, sms), []).append((m_lo, m_hi))
+    assert by_shape
+    want = [(lo, hi) for lo, hi, _ in tune.BUCKETS]
+    for key, buckets in by_shape.items():
+        assert sorted(buckets) == want, (key, sorted(buckets))
+        assert want[0][0] == 1 and want[-1][1] == 256
+        assert all(a[1] + 1 == b[0] for a, b in zip(want, want[1:]))
+
+
 def test_mma_resident_activations_fit_rule():
     """Resident activations (variant 2): the largest split's slice, ceil(k/64 / S) steps of
     m_pad rows x 128 bytes, plus the raw-code ring, the row scales and the barriers must fit the
